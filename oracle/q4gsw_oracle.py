@@ -31,9 +31,10 @@ the design notes of the repository):
 * groups run along K: scale index g = floor(k / group_size), K % group_size == 0;
 * the forward is y[M, N] = x[M, K] @ dequant(W)[N, K]^T (the per-projection GEMM
   that the backward mirrors);
-* the 4-byte interleave and the position of the scales inside the packed blob
-  (``packed_layout``) are this library's own layout, not the Vulkan W_4X8 block
-  order, which the pages do not spell out;
+* the order of the bytes inside a pair row, the position of the scales and
+  the trailer of the packed blob (``packed_layout``) are this library's own
+  layout, not the Vulkan W_4X8 block order, which the pages do not spell out;
+  it needs K % 64 == 0;
 * a GPU tensor-core operand is the fp16 value fp16_RNE((code - 8) * scale): one
   correctly rounded product.  ``dequant_w16_bits`` gives it;
 * all outputs are fp32 on the GPU; here they are fp64 sums of exact fp32
@@ -52,10 +53,14 @@ import numpy as np
 ZERO_POINT = 8          # [P2] dequant(W[n, k]) = (code - 8) * scale
 CODE_MAX = 15           # 4-bit codes
 LAYOUT_VERSION = 1
-SCALES_ALIGN = 256      # byte alignment of the scales region inside the blob
+REGION_ALIGN = 256      # byte alignment of the scales region and the trailer
+TRAILER_BYTES = 64
+TRAILER_MAGIC = 0x53473451   # bytes "Q4GS"
 
-# Position of k within its aligned group of four bytes (k mod 4 -> byte slot).
-# Slots 0..3 of a group hold k = 4j+0, 4j+2, 4j+1, 4j+3: an own-layout choice.
+# Own-layout choices for the codes region (version 1), see ``packed_layout``:
+# inside each 64-byte block of a pair row, word slot w (4 bytes) holds the
+# columns 16*(w % 4) + 4*(w // 4) + 0..3, and inside a word the byte slots
+# 0, 1, 2, 3 hold the columns +0, +2, +1, +3.
 _SLOT_OF_K_MOD4 = (0, 2, 1, 3)
 
 
@@ -129,30 +134,45 @@ def _encode_one(x: float) -> int:
 # The packed blob (layout version 1)
 # ----------------------------------------------------------------------------
 def packed_layout(N: int, K: int, group_size: int) -> dict:
-    """Byte map of one packed weight.
+    """Byte map of one packed weight (layout version 1).
 
-    codes region, offset 0, N/2 * K bytes: the byte of (pair p, column k) holds
+    codes region, offset 0, N/2 * K bytes.  The byte of (pair p, column k) holds
       code[2p, k] in bits 0..3 and code[2p+1, k] in bits 4..7   ([P2] nibble rule)
-    and sits at offset p*K + 4*floor(k/4) + slot(k mod 4), slot = (0, 2, 1, 3).
+    and sits at ``codescodes_byte_offset(p, k, K)``: row p of K bytes, cut into
+    64-byte blocks (K % 64 == 0); in a block, column r = 16 i + 4 t + e
+    (i, t, e in 0..3) is in word slot 4 t + i, byte slot (0, 2, 1, 3)[e].
     scales region, offset round_up(N/2*K, 256): fp16 [G][N] row-major, G = K/gs
     ([P2] "[num_groups, N] scales"; fp16 per [P1]).
+    trailer, offset round_up(scales end, 256), 64 bytes of little-endian u32:
+    magic "Q4GS", layout version, N, K, group_size, range flag (1 if a code
+    exceeded 15 at packing time, else 0), then zeros.
     """
     G = K // group_size
     codes_bytes = (N // 2) * K
-    scales_offset = -(-codes_bytes // SCALES_ALIGN) * SCALES_ALIGN
+    scales_offset = -(-codes_bytes // REGION_ALIGN) * REGION_ALIGN
     scales_bytes = 2 * G * N
+    trailer_offset = -(-(scales_offset + scales_bytes) // REGION_ALIGN) * REGION_ALIGN
     return {
         "G": G,
         "codes_offset": 0,
         "codes_bytes": codes_bytes,
         "scales_offset": scales_offset,
         "scales_bytes": scales_bytes,
-        "total_bytes": scales_offset + scales_bytes,
+        "trailer_offset": trailer_offset,
+        "total_bytes": trailer_offset + TRAILER_BYTES,
     }
 
 
-def _byte_offset(p: int, k: int, K: int) -> int:
-    return p * K + 4 * (k // 4) + _SLOT_OF_K_MOD4[k % 4]
+def codes_byte_offset(p: int, k: int, K: int) -> int:
+    r = k % 64
+    i, t, e = r // 16, (r % 16) // 4, r % 4
+    return p * K + 64 * (k // 64) + 4 * (4 * t + i) + _SLOT_OF_K_MOD4[e]
+
+
+def _trailer(N: int, K: int, group_size: int, range_flag: int) -> np.ndarray:
+    words = np.zeros(TRAILER_BYTES // 4, dtype="<u4")
+    words[:6] = (TRAILER_MAGIC, LAYOUT_VERSION, N, K, group_size, range_flag)
+    return words.view(np.uint8)
 
 
 def pack(codes: np.ndarray, scale_bits: np.ndarray, group_size: int) -> np.ndarray:
@@ -167,10 +187,11 @@ def pack(codes: np.ndarray, scale_bits: np.ndarray, group_size: int) -> np.ndarr
         for k in range(K):
             lo = int(codes[2 * p, k])
             hi = int(codes[2 * p + 1, k])
-            blob[_byte_offset(p, k, K)] = lo | (hi << 4)
+            blob[codes_byte_offset(p, k, K)] = lo | (hi << 4)
     sb = np.ascontiguousarray(np.asarray(scale_bits, dtype=np.uint16))
     assert sb.shape == (lay["G"], N)
-    blob[lay["scales_offset"]:lay["total_bytes"]] = sb.view(np.uint8).reshape(-1)
+    blob[lay["scales_offset"]:lay["scales_offset"] + lay["scales_bytes"]] = sb.view(np.uint8).reshape(-1)
+    blob[lay["trailer_offset"]:] = _trailer(N, K, group_size, 0)
     return blob
 
 
@@ -180,7 +201,7 @@ def unpack_codes(blob: np.ndarray, N: int, K: int, group_size: int) -> np.ndarra
     codes = np.zeros((N, K), dtype=np.uint8)
     for p in range(N // 2):
         for k in range(K):
-            b = int(blob[_byte_offset(p, k, K)])
+            b = int(blob[codes_byte_offset(p, k, K)])
             codes[2 * p, k] = b & 0xF
             codes[2 * p + 1, k] = b >> 4
     return codes
@@ -188,12 +209,17 @@ def unpack_codes(blob: np.ndarray, N: int, K: int, group_size: int) -> np.ndarra
 
 def unpack_scale_bits(blob: np.ndarray, N: int, K: int, group_size: int) -> np.ndarray:
     lay = packed_layout(N, K, group_size)
-    raw = np.ascontiguousarray(np.asarray(blob, dtype=np.uint8)[lay["scales_offset"]:lay["total_bytes"]])
+    raw = np.ascontiguousarray(np.asarray(blob, dtype=np.uint8)[lay["scales_offset"]:lay["scales_offset"] + lay["scales_bytes"]])
     return raw.view(np.uint16).reshape(lay["G"], N).copy()
 
 
 # Vectorised versions of the two loops above, for the large configurations.
 # They compute the same byte map; the tests check them against the loops.
+def _codes_offset_table(K: int) -> np.ndarray:
+    """offset of column k inside its pair row, for k in [0, K)."""
+    return np.array([codes_byte_offset(0, k, K) for k in range(K)], dtype=np.int64)
+
+
 def pack_fast(codes: np.ndarray, scale_bits: np.ndarray, group_size: int) -> np.ndarray:
     codes = np.asarray(codes, dtype=np.uint8)
     N, K = codes.shape
@@ -201,29 +227,30 @@ def pack_fast(codes: np.ndarray, scale_bits: np.ndarray, group_size: int) -> np.
     if codes.max(initial=0) > CODE_MAX:
         raise ValueError("code out of range")
     byte_pk = (codes[0::2, :] | (codes[1::2, :] << 4)).astype(np.uint8)   # [N/2, K]
-    grouped = byte_pk.reshape(N // 2, K // 4, 4)
-    stored = np.empty_like(grouped)
-    for j in range(4):
-        stored[:, :, _SLOT_OF_K_MOD4[j]] = grouped[:, :, j]
+    rows = np.zeros((N // 2, K), dtype=np.uint8)
+    rows[:, _codes_offset_table(K)] = byte_pk
     blob = np.zeros(lay["total_bytes"], dtype=np.uint8)
-    blob[:lay["codes_bytes"]] = stored.reshape(-1)
+    blob[:lay["codes_bytes"]] = rows.reshape(-1)
     sb = np.ascontiguousarray(np.asarray(scale_bits, dtype=np.uint16))
     assert sb.shape == (lay["G"], N)
-    blob[lay["scales_offset"]:] = sb.view(np.uint8).reshape(-1)
+    blob[lay["scales_offset"]:lay["scales_offset"] + lay["scales_bytes"]] = sb.view(np.uint8).reshape(-1)
+    blob[lay["trailer_offset"]:] = _trailer(N, K, group_size, 0)
     return blob
 
 
 def unpack_codes_fast(blob: np.ndarray, N: int, K: int, group_size: int) -> np.ndarray:
     lay = packed_layout(N, K, group_size)
-    stored = np.asarray(blob, dtype=np.uint8)[:lay["codes_bytes"]].reshape(N // 2, K // 4, 4)
-    byte_pk = np.empty_like(stored)
-    for j in range(4):
-        byte_pk[:, :, j] = stored[:, :, _SLOT_OF_K_MOD4[j]]
-    byte_pk = byte_pk.reshape(N // 2, K)
+    rows = np.asarray(blob, dtype=np.uint8)[:lay["codes_bytes"]].reshape(N // 2, K)
+    byte_pk = rows[:, _codes_offset_table(K)]
     codes = np.empty((N, K), dtype=np.uint8)
     codes[0::2] = byte_pk & 0xF
     codes[1::2] = byte_pk >> 4
     return codes
+
+
+def trailer_words(blob: np.ndarray, N: int, K: int, group_size: int) -> np.ndarray:
+    lay = packed_layout(N, K, group_size)
+    return np.ascontiguousarray(np.asarray(blob, np.uint8)[lay["trailer_offset"]:]).view("<u4").copy()
 
 
 # ----------------------------------------------------------------------------

@@ -72,12 +72,24 @@ def test_fp16_encode_halfway_and_overflow_cases():
 
 # --------------------------------------------------------------------------- packing
 def test_pack_hand_example():
-    rows, _ = _read_fixture("nibble_pairs.txt")
-    codes = np.array([int(v) for v in rows["codes"]], np.uint8).reshape(2, 4)
-    want = np.array([int(v, 16) for v in rows["bytes"]], np.uint8)
-    blob = o.pack(codes, np.zeros((1, 2), np.uint16), 4)
-    assert np.array_equal(blob[:4], want)
-    assert np.array_equal(o.unpack_codes(blob, 2, 4, 4), codes)
+    _, lines = _read_fixture("nibble_pairs.txt")
+    codes = np.full((2, 64), 8, np.uint8)
+    want = np.full(64, 0x88, np.uint8)
+    for _, col, lo, hi, byte, off in (ln[:6] for ln in lines):
+        codes[0, int(col)], codes[1, int(col)] = int(lo), int(hi)
+        want[int(off)] = int(byte, 16)
+    blob = o.pack(codes, np.zeros((2, 2), np.uint16), 32)
+    assert np.array_equal(blob[:64], want)
+    assert np.array_equal(o.unpack_codes(blob, 2, 64, 32), codes)
+
+
+def test_codes_offsets_are_a_permutation_of_each_block():
+    K = 256
+    offs = [o.codes_byte_offset(0, k, K) for k in range(K)]
+    assert sorted(offs) == list(range(K))
+    for k in range(K):
+        assert offs[k] // 64 == k // 64          # a column never leaves its 64-byte block
+    assert o.codes_byte_offset(3, 5, K) == 3 * K + offs[5]
 
 
 def test_pack_every_byte_value_round_trips():
@@ -86,20 +98,28 @@ def test_pack_every_byte_value_round_trips():
     codes = np.stack([np.arange(K) & 15, np.arange(K) >> 4]).astype(np.uint8)
     blob = o.pack(codes, np.zeros((K // 32, 2), np.uint16), 32)
     for k in range(K):
-        assert blob[4 * (k // 4) + (0, 2, 1, 3)[k % 4]] == k
+        assert blob[o.codes_byte_offset(0, k, K)] == k
+    assert sorted(blob[:K].tolist()) == list(range(256))
     assert np.array_equal(o.unpack_codes(blob, 2, K, 32), codes)
 
 
-def test_pack_layout_sizes():
+def test_pack_layout_sizes_and_trailer():
     lay = o.packed_layout(14336, 4096, 128)
     assert lay["codes_bytes"] == 14336 // 2 * 4096
     assert lay["scales_offset"] % 256 == 0 and lay["scales_offset"] >= lay["codes_bytes"]
-    assert lay["total_bytes"] == lay["scales_offset"] + 2 * 32 * 14336
-    lay = o.packed_layout(8, 48, 16)     # codes region 192 B -> scales at 256
-    assert lay["scales_offset"] == 256
+    assert lay["trailer_offset"] % 256 == 0
+    assert lay["trailer_offset"] >= lay["scales_offset"] + 2 * 32 * 14336
+    assert lay["total_bytes"] == lay["trailer_offset"] + 64
+    lay = o.packed_layout(6, 64, 16)     # codes 192 B -> scales at 256, 48 B -> trailer at 512
+    assert (lay["scales_offset"], lay["trailer_offset"], lay["total_bytes"]) == (256, 512, 576)
+    codes = np.zeros((6, 64), np.uint8)
+    blob = o.pack(codes, np.ones((4, 6), np.uint16), 16)
+    tw = o.trailer_words(blob, 6, 64, 16)
+    assert bytes(blob[512:516]) == b"Q4GS"
+    assert list(tw[:6]) == [0x53473451, 1, 6, 64, 16, 0] and not tw[6:].any()
 
 
-@pytest.mark.parametrize("N,K,gs", [(2, 4, 4), (8, 64, 32), (64, 128, 32), (24, 96, 16)])
+@pytest.mark.parametrize("N,K,gs", [(2, 64, 64), (8, 64, 32), (64, 128, 32), (24, 192, 16)])
 def test_pack_fast_matches_loop(N, K, gs):
     rng = np.random.default_rng(N * K)
     codes = rng.integers(0, 16, (N, K), dtype=np.uint8)
@@ -112,7 +132,7 @@ def test_pack_fast_matches_loop(N, K, gs):
 
 def test_pack_rejects_out_of_range_codes():
     with pytest.raises(ValueError):
-        o.pack(np.full((2, 4), 16, np.uint8), np.zeros((1, 2), np.uint16), 4)
+        o.pack(np.full((2, 64), 16, np.uint8), np.zeros((1, 2), np.uint16), 64)
 
 
 # --------------------------------------------------------------------------- dequant
