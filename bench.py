@@ -1,0 +1,567 @@
+#!/usr/bin/env python
+"""Benchmark of the q4gsw linear layer on B200.
+
+One step = the adapter-training pass of one 1B-class decoder layer (hidden
+2048, 32 query / 8 key-value heads of width 64, MLP 8192) over a frozen q4gsw
+base, 512 tokens, group size 32:
+    fused Q/K/V forward   x[512,2048] -> y_q[512,2048], y_k[512,512], y_v[512,512]
+    MLP up forward        x[512,2048] -> y[512,8192]
+    MLP down forward      x[512,8192] -> y[512,2048]
+    MLP down input grad   d_out[512,2048] -> d_x[512,8192]
+    MLP up input grad     d_out[512,8192] -> d_x[512,2048]
+All inputs are seeded synthetic tensors (x ~ N(0,1), codes uniform 0..15,
+scales U[0.005, 0.02], d_out ~ N(0, 1e-2)), prepacked once (not timed).
+Between steps the weights and activations rotate over R copies whose total
+exceeds the 126 MB L2, so every step reads its weights from HBM.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+        python bench.py --sweep        (one JSON line per configuration shape)
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_group_quantized_q4gsw_b200 import workloads as wl  # noqa: E402
+
+METRIC = "q4gsw fwd+bwd_input TFLOP/s and weight GB/s on 1 B200, % of roofline"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4gsw base: "
+            "fused QKV fwd (K2048->2048+512+512) + MLP up fwd (2048->8192) + down fwd (8192->2048) "
+            "+ down and up input grads; M=512 tokens, group_size 32")
+
+# DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
+# dram__bytes_write.sum), with the hash of the kernel sources they were taken on.
+NCU_TRAFFIC = {"sources_sha": None, "bytes_per_launch": {}}
+
+
+def sources_sha() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "bit_group_quantized_q4gsw_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "tflops": d["bf16_tflops"], "tflops_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "tflops": 1590.0, "tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- the step
+def step_ops():
+    """(name, kind, shape) for the five operations of one step."""
+    qkv = wl.by_name("qkv_M512")
+    up, down = wl.adapter()
+    return [("qkv_fwd", "qkv", qkv), ("up_fwd", "fwd", up), ("down_fwd", "fwd", down),
+            ("down_bwd", "bwd", down), ("up_bwd", "bwd", up)]
+
+
+def op_flops(kind, sh, M=None):
+    M = sh.M if M is None else M
+    return 2.0 * M * sh.N * sh.K
+
+
+def op_bytes(kind, sh, M=None):
+    """Algorithmic bytes: packed codes + scales once, activations in, fp32 out."""
+    M = sh.M if M is None else M
+    w = sh.N * sh.K // 2 + 2 * (sh.K // sh.group_size) * sh.N
+    if kind == "bwd":
+        return w + 2 * M * sh.N + 4 * M * sh.K
+    return w + 2 * M * sh.K + 4 * M * sh.N
+
+
+def weight_bytes(sh):
+    return sh.N * sh.K // 2 + 2 * (sh.K // sh.group_size) * sh.N
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+               "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100}
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [k for k, v in self.REASONS.items() if bits & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+def oracle_sample_step(inputs, frac_cols: int):
+    """The five operations through the oracle on a sample: all tokens, and the
+    first 1/frac_cols of each operation's output features (whole groups).
+    Returns (seconds, flops of the sample)."""
+    import oracle as o
+    bits = lambda a: np.asarray(a, np.float16).view(np.uint16)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for name, kind, sh in step_ops():
+        inp = inputs[name]
+        M = inp.x.shape[0]
+        if kind in ("fwd", "qkv"):
+            n = max(8, (sh.N // frac_cols) // 8 * 8)
+            o.linear_fwd(bits(inp.x), inp.codes[:n], bits(inp.scales[:, :n]), sh.group_size)
+            flops += 2.0 * M * n * sh.K
+        else:
+            kk = max(sh.group_size, (sh.K // frac_cols) // sh.group_size * sh.group_size)
+            o.linear_bwd_input(bits(inp.d_out), inp.codes[:, :kk], bits(inp.scales[:kk // sh.group_size]),
+                               sh.group_size)
+            flops += 2.0 * M * sh.N * kk
+    return time.perf_counter() - t0, flops
+
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = [d for d in threadpool_info() if d.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def host_inputs():
+    out = {}
+    for name, kind, sh in step_ops():
+        out[name] = wl.make_inputs(sh)
+    return out
+
+
+def cpu_baseline(inputs, budget_s: float = 12.0):
+    t, _ = oracle_sample_step(inputs, 64)            # probe
+    frac = 64 if t > budget_s / 4 else max(1, int(64 * t / (budget_s / 4)))
+    frac = max(1, frac)
+    times, flops = [], 0.0
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or not times:
+        dt, flops = oracle_sample_step(inputs, frac)
+        times.append(dt)
+    value = flops / statistics.median(times) / 1e12
+    return {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"all 5 ops of the step, all 512 tokens, first 1/{frac} of each op's output features; "
+                      f"{len(times)} repetitions, median"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    inputs = host_inputs()
+    t, _ = oracle_sample_step(inputs, 64)
+    total_budget = 150.0
+    per_step = max(0.05, total_budget / max(1, args.steps + args.warmup))
+    frac = 64
+    while frac < 4096 and t > per_step:
+        frac *= 2
+        t /= 2
+    for _ in range(args.warmup):
+        oracle_sample_step(inputs, frac)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, flops = oracle_sample_step(inputs, frac)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms / 1e3) / 1e12
+    sample = (f"all 5 ops, 512 tokens, first 1/{frac} of each op's output features ({flops / 1e9:.3f} GFLOP per step)")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 512, "seq_len": 512, "parallelism": "replicas"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+class GpuStep:
+    """Device buffers for R rotating copies of the step's weights and activations."""
+
+    def __init__(self, inputs, copies, device):
+        import torch
+        import bit_group_quantized_q4gsw_b200 as q
+        self.q = q
+        self.torch = torch
+        self.lib = q.library()
+        self.dev = device
+        self.stream = torch.cuda.current_stream(device)
+        self.sptr = self.stream.cuda_stream
+        self.ops = step_ops()
+        self.copies = copies
+        self.packed, self.acts, self.outs = {}, {}, {}
+        for name, kind, sh in self.ops:
+            inp = inputs[name]
+            key = sh.name
+            if key not in self.packed:
+                codes = torch.from_numpy(inp.codes).to(device)
+                scales = torch.from_numpy(inp.scales).to(device)
+                first = q.q4gsw_prepack(codes, scales, sh.group_size)
+                self.packed[key] = [first] + [first.clone() for _ in range(copies - 1)]
+            src = inp.d_out if kind == "bwd" else inp.x
+            self.acts[name] = [torch.from_numpy(src).to(device) for _ in range(copies)]
+            if kind == "qkv":
+                Nq, Nk, Nv = sh.splits
+                self.outs[name] = [torch.empty((sh.M, n), dtype=torch.float32, device=device) for n in (Nq, Nk, Nv)]
+            elif kind == "fwd":
+                self.outs[name] = [torch.empty((sh.M, sh.N), dtype=torch.float32, device=device)]
+            else:
+                self.outs[name] = [torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)]
+        torch.cuda.synchronize(device)
+
+    def bytes_resident(self):
+        tot = 0
+        for v in self.packed.values():
+            tot += sum(t.numel() for t in v)
+        for v in self.acts.values():
+            tot += sum(t.numel() * t.element_size() for t in v)
+        return tot
+
+    def call(self, name, kind, sh, c):
+        """One operation through the C ABI on copy c (raw pointers, current stream)."""
+        lib, s = self.lib, self.sptr
+        pk = self.packed[sh.name][c].data_ptr()
+        a = self.acts[name][c].data_ptr()
+        o = self.outs[name]
+        if kind == "qkv":
+            Nq, Nk, Nv = sh.splits
+            st = lib.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, a, sh.M, o[0].data_ptr(), o[1].data_ptr(),
+                                   o[2].data_ptr(), s)
+        elif kind == "fwd":
+            st = lib.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a, sh.M, o[0].data_ptr(), s)
+        else:
+            st = lib.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a, sh.M, o[0].data_ptr(), s)
+        if st != 0:
+            raise RuntimeError(f"{name}: status {st} ({lib.q4gsw_status_str(st).decode()})")
+
+    def launches_per_call(self):
+        out = {}
+        for name, kind, sh in self.ops:
+            self.call(name, kind, sh, 0)
+            route = self.lib.q4gsw_last_route().decode()
+            n = 1
+            for tok in route.split():
+                if tok.startswith("launches="):
+                    n = int(tok.split("=")[1])
+            out[name] = (n, route)
+        self.torch.cuda.synchronize(self.dev)
+        return out
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    peaks = measured_peaks()
+    inputs = host_inputs()
+    ops = step_ops()
+    set_bytes = sum(weight_bytes(sh) for sh in {sh.name: sh for _, _, sh in ops}.values())
+    act_bytes = sum(inputs[n].x.nbytes if k != "bwd" else inputs[n].d_out.nbytes for n, k, _ in ops)
+    copies = args.copies or max(2, math.ceil(2.0 * L2_BYTES / (set_bytes + act_bytes)))
+    gs = GpuStep(inputs, copies, device)
+    per_call = gs.launches_per_call()
+    launches_per_step = sum(n for n, _ in per_call.values())
+    flops_step = sum(op_flops(k, sh) for _, k, sh in ops)
+    wbytes_step = sum(weight_bytes(sh) for _, _, sh in ops)
+
+    # ---- device-resident timed region
+    nops = len(ops)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(args.steps)]
+    for i in range(args.warmup):
+        for name, kind, sh in ops:
+            gs.call(name, kind, sh, i % copies)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record()
+        for i in range(args.steps):
+            c = (args.warmup + i) % copies
+            ev[i][0].record()
+            for j, (name, kind, sh) in enumerate(ops):
+                gs.call(name, kind, sh, c)
+                ev[i][j + 1].record()
+        end.record()
+        torch.cuda.synchronize(device)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    value = world * flops_step / (ms_step / 1e3) / 1e12
+    op_ms = {}
+    for j, (name, kind, sh) in enumerate(ops):
+        op_ms[name] = statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
+    clocks = sampler.summary()
+
+    # dominant op -> roofline
+    dom = max(op_ms, key=op_ms.get)
+    dkind, dsh = [(k, sh) for n, k, sh in ops if n == dom][0]
+    n_launch = per_call[dom][0]
+    fl = op_flops(dkind, dsh)
+    by = op_bytes(dkind, dsh)
+    ridge = peaks["tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if fl / by >= ridge:
+        achieved = fl / (op_ms[dom] / n_launch / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["tflops"], "unit": "TFLOP/s",
+                "peak_kind": f"bf16 dense burst ({peaks['source']})"}
+    else:
+        achieved = by / (op_ms[dom] / n_launch / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "peak_kind": f"HBM copy ({peaks['source']})"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    traffic = None
+    if NCU_TRAFFIC["sources_sha"] == sources_sha():
+        traffic = NCU_TRAFFIC["bytes_per_launch"].get(dom)
+    roof["traffic"] = traffic
+    roof["kernel"] = per_call[dom][1]
+    roof["op"] = dom
+
+    # ---- end to end through the public Python API with pinned host buffers
+    q = gs.q
+    host_in = {}
+    for name, kind, sh in ops:
+        src = inputs[name].d_out if kind == "bwd" else inputs[name].x
+        host_in[name] = torch.from_numpy(src).pin_memory()
+    host_out = {name: [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in gs.outs[name]] for name, _, _ in ops}
+    dev_in = {name: torch.empty(host_in[name].shape, dtype=torch.float16, device=device) for name, _, _ in ops}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for v in host_out.values() for t in v)
+    e2e_steps = max(1, min(args.steps, 50))
+
+    def e2e_step(c):
+        for name, kind, sh in ops:
+            dev_in[name].copy_(host_in[name], non_blocking=True)
+        for name, kind, sh in ops:
+            pk = gs.packed[sh.name][c]
+            o = gs.outs[name]
+            if kind == "qkv":
+                Nq, Nk, Nv = sh.splits
+                q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, dev_in[name], outs=o)
+            elif kind == "fwd":
+                q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, dev_in[name], y=o[0])
+            else:
+                q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, dev_in[name], d_x=o[0])
+        for name, _, _ in ops:
+            for hb, db in zip(host_out[name], gs.outs[name]):
+                hb.copy_(db, non_blocking=True)
+
+    for i in range(min(args.warmup, 3)):
+        e2e_step(i % copies)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e_step(i % copies)
+    e1.record()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e = {"value": world * flops_step / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16 inputs, f32 accumulate", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 512 * world, "seq_len": 512,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": f"rotating {copies} copies of weights+activations "
+                             f"({copies * (set_bytes + act_bytes) / 1e6:.0f} MB) > 126 MB L2"},
+            "weight_gbs": world * wbytes_step / (ms_step / 1e3) / 1e9,
+            "roofline": roof, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
+            "e2e": e2e,
+            "ops_ms": {k: round(v, 5) for k, v in op_ms.items()},
+            "ops_tflops": {n: op_flops(k, sh) / (op_ms[n] / 1e3) / 1e12 for n, k, sh in ops},
+            "routes": {k: v[1] for k, v in per_call.items()}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inputs)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- per-shape sweep
+def run_sweep(args):
+    import torch
+    import bit_group_quantized_q4gsw_b200 as q
+    device = torch.device("cuda", 0)
+    peaks = measured_peaks()
+    shapes = wl.tiny() + wl.decode() + wl.qkv() + wl.adapter() + wl.sweep()
+    if args.only:
+        shapes = [s for s in shapes if args.only in s.name]
+    for sh in shapes:
+        inp = wl.make_inputs(sh)
+        codes = torch.from_numpy(inp.codes).to(device)
+        scales = torch.from_numpy(inp.scales).to(device)
+        first = q.q4gsw_prepack(codes, scales, sh.group_size)
+        del codes, scales
+        wb = weight_bytes(sh)
+        R = max(2, math.ceil(3 * L2_BYTES / wb))
+        packs = [first] + [first.clone() for _ in range(R - 1)]
+        kinds = ["qkv"] if sh.splits else list(sh.directions)
+        for kind in kinds:
+            src = inp.d_out if kind == "bwd" else inp.x
+            a = torch.from_numpy(src).to(device)
+            if kind == "qkv":
+                Nq, Nk, Nv = sh.splits
+                outs = tuple(torch.empty((sh.M, n), dtype=torch.float32, device=device) for n in (Nq, Nk, Nv))
+                fn = lambda pk: q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, a, outs=outs)
+            elif kind == "fwd":
+                y = torch.empty((sh.M, sh.N), dtype=torch.float32, device=device)
+                fn = lambda pk: q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a, y=y)
+            else:
+                y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
+                fn = lambda pk: q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a, d_x=y)
+            for i in range(5):
+                fn(packs[i % R])
+            torch.cuda.synchronize()
+            iters = max(R, 50)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(iters):
+                    fn(packs[i % R])
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 3
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / (reps * iters) / 1e3
+            fl = op_flops(kind, sh)
+            by = op_bytes(kind, sh)
+            print(json.dumps({"shape": sh.name, "dir": kind, "M": sh.M, "N": sh.N, "K": sh.K, "gs": sh.group_size,
+                              "us": t * 1e6, "tflops": fl / t / 1e12, "gbs": by / t / 1e9,
+                              "weight_gbs": wb / t / 1e9, "frac_tc": fl / t / 1e12 / peaks["tflops"],
+                              "frac_hbm_measured": by / t / 1e9 / peaks["hbm_gbs"], "frac_hbm_8tbs": by / t / 8e12,
+                              "route": q.q4gsw_last_route(), "copies": R}), flush=True)
+            del g
+        del packs, first
+        torch.cuda.empty_cache()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--copies", type=int, default=0)
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--only", default="")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.sweep:
+        return run_sweep(args)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

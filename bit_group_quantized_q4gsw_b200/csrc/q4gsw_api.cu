@@ -1,0 +1,160 @@
+// q4gsw_api.cu - the extern "C" entry points declared in include/q4gsw.h:
+// argument checks, route choice and launches.  Nothing here computes a
+// result on the host; every number comes from the CUDA kernels.
+//
+// Route choice mirrors the geometry predicate of "[ExecuTorch][WebGPU] Replace
+// broad QKV fusion with BK64 kernel" (description of #21131): a route is taken
+// only for shapes it accepts, and the choice is made on the host per call.
+// Argument rules follow "[ExecuTorch][Vulkan] Add et_vk.linear_q4gsw_backward
+// kernel (4-bit input-grad)", PR description, "Constraints" (N, K, group_size
+// multiples of 4), tightened by the packed layout and TMA stride rules.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/q4gsw.h"
+#include "q4gsw_common.cuh"
+#include "q4gsw_internal.h"
+
+using namespace q4gsw;
+
+namespace {
+
+thread_local char g_route[160] = "none";
+
+void set_route(const char* s) {
+  std::strncpy(g_route, s, sizeof(g_route) - 1);
+  g_route[sizeof(g_route) - 1] = 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+// Shape rules shared by every entry point.
+q4gsw_status check_weight_shape(int N, int K, int gs) {
+  if (N <= 0 || K <= 0 || gs <= 0) return Q4GSW_ERR_SHAPE;
+  if (N % 4 || K % 4 || gs % 4) return Q4GSW_ERR_SHAPE;        // the page's constraints
+  if (N % 8 || K % 64) return Q4GSW_ERR_ALIGN;                  // layout blocks, 16-byte strides
+  if (!is_pow2(gs) || gs < 16 || gs > K) return Q4GSW_ERR_UNSUPPORTED;
+  return Q4GSW_OK;
+}
+
+q4gsw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? Q4GSW_OK : Q4GSW_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int q4gsw_layout_version(void) { return kLayoutVersion; }
+
+size_t q4gsw_packed_bytes(int N, int K, int group_size) {
+  if (check_weight_shape(N, K, group_size) != Q4GSW_OK) return 0;
+  return layout_of(N, K, group_size).total_bytes;
+}
+
+const char* q4gsw_last_route(void) { return g_route; }
+
+const char* q4gsw_status_str(q4gsw_status s) {
+  switch (s) {
+    case Q4GSW_OK: return "ok";
+    case Q4GSW_ERR_NULL: return "null pointer";
+    case Q4GSW_ERR_SHAPE: return "invalid shape";
+    case Q4GSW_ERR_ALIGN: return "misaligned pointer or shape (16-byte pointers, N % 8, K % 64)";
+    case Q4GSW_ERR_UNSUPPORTED: return "unsupported group size (power of two in [16, K])";
+    case Q4GSW_ERR_CODE_RANGE: return "code above 15";
+    case Q4GSW_ERR_CUDA: return "CUDA runtime error";
+    case Q4GSW_ERR_SIZE: return "buffer too small";
+  }
+  return "unknown status";
+}
+
+q4gsw_status q4gsw_prepack(const uint8_t* codes, const uint16_t* scales, int N, int K, int group_size,
+                           void* packed, size_t packed_bytes, q4gsw_stream_t stream) {
+  if (!codes || !scales || !packed) return Q4GSW_ERR_NULL;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(packed)) return Q4GSW_ERR_ALIGN;
+  if (packed_bytes < layout_of(N, K, group_size).total_bytes) return Q4GSW_ERR_SIZE;
+  uint32_t flag = 0;
+  set_route("prepack");
+  st = from_cuda(launch_prepack(codes, scales, N, K, group_size, packed, stream, &flag));
+  if (st != Q4GSW_OK) return st;
+  return flag ? Q4GSW_ERR_CODE_RANGE : Q4GSW_OK;
+}
+
+q4gsw_status q4gsw_linear_fwd(const void* packed, int N, int K, int group_size, const uint16_t* x, int M,
+                              float* y, q4gsw_stream_t stream) {
+  if (M < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed || !x || !y) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y)) return Q4GSW_ERR_ALIGN;
+  char route[160];
+  cudaError_t e = launch_gemv_fwd(packed, N, K, group_size, x, M, single_output(y, N), stream, route,
+                                  sizeof(route));
+  set_route(route);
+  return from_cuda(e);
+}
+
+q4gsw_status q4gsw_linear_bwd_input(const void* packed, int N, int K, int group_size, const uint16_t* d_out,
+                                    int M, float* d_x, q4gsw_stream_t stream) {
+  if (M < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed || !d_out || !d_x) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(d_out) || !aligned16(d_x)) return Q4GSW_ERR_ALIGN;
+  char route[160];
+  cudaError_t e = launch_gemv_bwd(packed, N, K, group_size, d_out, M, d_x, stream, route, sizeof(route));
+  set_route(route);
+  return from_cuda(e);
+}
+
+q4gsw_status q4gsw_qkv_fwd(const void* packed_qkv, int Nq, int Nk, int Nv, int K, int group_size,
+                           const uint16_t* x, int M, float* y_q, float* y_k, float* y_v,
+                           q4gsw_stream_t stream) {
+  if (M < 0 || Nq <= 0 || Nk <= 0 || Nv <= 0) return Q4GSW_ERR_SHAPE;
+  if ((long long)Nq + Nk + Nv > 0x7fffffffLL) return Q4GSW_ERR_SHAPE;
+  const int N = Nq + Nk + Nv;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (Nq % 4 || Nk % 4 || Nv % 4) return Q4GSW_ERR_SHAPE;
+  if (Nq % 8 || Nk % 8 || Nv % 8) return Q4GSW_ERR_ALIGN;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed_qkv || !x || !y_q || !y_k || !y_v) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed_qkv) || !aligned16(x) || !aligned16(y_q) || !aligned16(y_k) || !aligned16(y_v))
+    return Q4GSW_ERR_ALIGN;
+  OutSplit out{y_q, y_k, y_v, Nq, Nq + Nk, N};
+  char route[120];
+  cudaError_t e = launch_gemv_fwd(packed_qkv, N, K, group_size, x, M, out, stream, route, sizeof(route));
+  char full[160];
+  snprintf(full, sizeof(full), "qkv %s", route);
+  set_route(full);
+  return from_cuda(e);
+}
+
+q4gsw_status q4gsw_unpack(const void* packed, int N, int K, int group_size, uint8_t* codes,
+                          q4gsw_stream_t stream) {
+  if (!packed || !codes) return Q4GSW_ERR_NULL;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (!aligned16(packed) || !aligned16(codes)) return Q4GSW_ERR_ALIGN;
+  set_route("unpack");
+  return from_cuda(launch_unpack(packed, N, K, codes, stream));
+}
+
+q4gsw_status q4gsw_dequant(const void* packed, int N, int K, int group_size, float* w32, uint16_t* w16,
+                           q4gsw_stream_t stream) {
+  if (!packed || (!w32 && !w16)) return Q4GSW_ERR_NULL;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (!aligned16(packed) || (w32 && !aligned16(w32)) || (w16 && !aligned16(w16))) return Q4GSW_ERR_ALIGN;
+  set_route("dequant");
+  return from_cuda(launch_dequant(packed, N, K, group_size, w32, w16, stream));
+}
+
+}  // extern "C"

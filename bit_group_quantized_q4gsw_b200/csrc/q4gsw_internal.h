@@ -1,0 +1,35 @@
+// q4gsw_internal.h - launchers shared between the translation units of the
+// library.  Not part of the C ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace q4gsw {
+
+cudaError_t launch_prepack(const uint8_t* codes, const uint16_t* scales, int N, int K, int gs,
+                           void* packed, cudaStream_t stream, uint32_t* host_flag);
+cudaError_t launch_unpack(const void* packed, int N, int K, uint8_t* codes, cudaStream_t stream);
+cudaError_t launch_dequant(const void* packed, int N, int K, int gs, float* w32, uint16_t* w16,
+                           cudaStream_t stream);
+
+// Output columns [0, N) of a forward split over up to three row-major
+// buffers: n < n1 -> y0[m, n], n < n2 -> y1[m, n - n1], else y2[m, n - n2]
+// (the fused Q/K/V projection writes three distinct outputs).
+struct OutSplit {
+  float* y0;
+  float* y1;
+  float* y2;
+  int n1, n2, N;
+};
+
+__host__ __device__ inline OutSplit single_output(float* y, int N) { return OutSplit{y, y, y, N, N, N}; }
+
+// Tensor-core GEMV routes for small token counts.  `M` may exceed 16: token
+// chunks of 16 then run as grid z-slices (each re-reads the weight).
+cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M,
+                            OutSplit out, cudaStream_t stream, char* route, int route_len);
+cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M,
+                            float* d_x, cudaStream_t stream, char* route, int route_len);
+
+}  // namespace q4gsw

@@ -1,0 +1,164 @@
+/*
+ * q4gsw.h - C ABI of the q4gsw 4-bit group-symmetric weight-quantized linear
+ * layer for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the definitions (three web pages):
+ *   [P2] "[ExecuTorch][Vulkan] Add et_vk.linear_q4gsw_backward kernel (4-bit
+ *        input-grad)", pytorch/executorch pull request #20943, PR description:
+ *        the input gradient d_x[M,K] = d_out[M,N] @ dequant(W)[N,K] contracting
+ *        over N; dequant(W[n,k]) = (code - 8) * scale; "Key changes": even-N
+ *        code in the low nibble, odd-N code in the high nibble, [num_groups, N]
+ *        scales, one prepack shared by forward and backward; "Constraints":
+ *        N, K, group_size multiples of 4, fp32.
+ *   [P3] "[ExecuTorch][WebGPU] Replace broad QKV fusion with BK64 kernel",
+ *        pytorch/executorch pull request #21650, description of #21131: the
+ *        Q/K/V projection triple fused over one packing of the constant
+ *        weights and scales, scattered into three distinct outputs; outside the
+ *        accepted shapes the ordinary routes run.
+ *   [P1] "Upstream the Gemma 4 Vulkan support we carry on our ExecuTorch fork",
+ *        software-mansion/react-native-executorch issue #1361, comment of
+ *        Oct 20, 2026: fp16 weight scales.
+ *
+ * Notation: M tokens, K input features, N output features, gs = group_size,
+ * G = K / gs.  code[n,k] in 0..15, scale[g,n] fp16,
+ *     w[n,k] = (code[n,k] - 8) * scale[k / gs, n].
+ *
+ * Conventions for every entry point
+ *   - Every pointer argument is a DEVICE pointer on the current CUDA device,
+ *     except where stated.  The caller allocates and owns every buffer; the
+ *     library allocates no device memory and keeps no state besides a
+ *     thread-local route string.
+ *   - Dense operands are contiguous row-major.  fp16 values are passed as
+ *     uint16_t bit patterns; outputs are fp32.
+ *   - Device pointers must be 16-byte aligned (Q4GSW_ERR_ALIGN otherwise).
+ *   - Calls enqueue work on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return without waiting, except q4gsw_prepack (see there).
+ *   - Arguments are checked on the host before anything is enqueued; on an
+ *     error nothing is enqueued and outputs are untouched.  A launch failure
+ *     reported by the CUDA runtime returns Q4GSW_ERR_CUDA.
+ *   - No CPU fallback exists: every result is computed by this library's
+ *     CUDA kernels.  Calls are thread-safe and re-entrant.
+ *   - Shapes accepted: N > 0, N % 8 == 0; K > 0, K % 64 == 0; gs a power of
+ *     two with 16 <= gs <= K (so K % gs == 0).  [P2]'s own constraints
+ *     (multiples of 4) are a superset; the tighter ones come from the packed
+ *     layout (64-byte blocks) and from 16-byte TMA strides.  M == 0 is an empty
+ *     batch: nothing is enqueued and Q4GSW_OK is returned.
+ */
+#ifndef Q4GSW_H
+#define Q4GSW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define Q4GSW_API __attribute__((visibility("default")))
+#else
+#define Q4GSW_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *q4gsw_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+  Q4GSW_OK = 0,
+  Q4GSW_ERR_NULL = 1,         /* a required pointer is NULL */
+  Q4GSW_ERR_SHAPE = 2,        /* negative or zero sizes, [P2] multiple-of-4 rule, Q/K/V split mismatch */
+  Q4GSW_ERR_ALIGN = 3,        /* pointer not 16-byte aligned, N % 8 or K % 64 != 0 */
+  Q4GSW_ERR_UNSUPPORTED = 4,  /* group size not a power of two in [16, K] */
+  Q4GSW_ERR_CODE_RANGE = 5,   /* q4gsw_prepack saw a code > 15 */
+  Q4GSW_ERR_CUDA = 6,         /* the CUDA runtime reported an error */
+  Q4GSW_ERR_SIZE = 7          /* a byte count passed in is too small */
+} q4gsw_status;
+
+/* Version of the packed-weight byte layout written by q4gsw_prepack. */
+Q4GSW_API int q4gsw_layout_version(void);
+
+/*
+ * Bytes of the packed weight for (N, K, gs); 0 if the shape is not accepted.
+ * Layout version 1 (all offsets from the start of the blob):
+ *   codes   [0, N/2*K): for pair p = n/2 and column k, the byte
+ *           code[2p,k] | code[2p+1,k] << 4  ([P2] nibble rule) at
+ *           p*K + 64*(k/64) + 4*(4*t + i) + slot[e],  where k%64 = 16 i + 4 t + e
+ *           and slot = {0, 2, 1, 3}.
+ *   scales  at round_up(N/2*K, 256): fp16 [G][N] row-major ([P2] "[num_groups, N]").
+ *   trailer at round_up(scales end, 256), 64 bytes of little-endian uint32:
+ *           "Q4GS", version, N, K, gs, range flag, then zeros.
+ */
+Q4GSW_API size_t q4gsw_packed_bytes(int N, int K, int group_size);
+
+/*
+ * One-time packer ([P2] "Key changes": the prepack shared by forward and
+ * backward; [P3]: "packing the constant weights and scales once").
+ *   codes   uint8 [N, K], one code per byte, each in 0..15
+ *   scales  fp16  [K/gs, N]
+ *   packed  output, packed_bytes >= q4gsw_packed_bytes(N, K, gs)
+ * Writes the whole blob (codes, scales, trailer; padding zeroed).  It then
+ * waits for `stream` once, to read the range flag back: a code above 15
+ * returns Q4GSW_ERR_CODE_RANGE (the blob content is then unspecified).
+ */
+Q4GSW_API q4gsw_status q4gsw_prepack(const uint8_t *codes, const uint16_t *scales,
+                           int N, int K, int group_size,
+                           void *packed, size_t packed_bytes,
+                           q4gsw_stream_t stream);
+
+/*
+ * Forward: y[m,n] = sum_k x[m,k] * w[n,k], fp32 accumulation.
+ *   packed  a blob from q4gsw_prepack for the same (N, K, gs)
+ *   x       fp16 [M, K];   y  fp32 [M, N] (overwritten)
+ * Route: M <= 16 a tensor-core GEMV over the streamed packed weight; larger M
+ * a tcgen05 GEMM that dequantises into shared memory.
+ */
+Q4GSW_API q4gsw_status q4gsw_linear_fwd(const void *packed, int N, int K, int group_size,
+                              const uint16_t *x, int M, float *y,
+                              q4gsw_stream_t stream);
+
+/*
+ * Input gradient of the frozen base ([P2]):
+ *   d_x[m,k] = sum_n d_out[m,n] * w[n,k]   (contracts over N)
+ *   d_out fp16 [M, N];   d_x  fp32 [M, K] (overwritten)
+ * Reads the same packed blob as the forward (no re-pack, [P2]).
+ */
+Q4GSW_API q4gsw_status q4gsw_linear_bwd_input(const void *packed, int N, int K, int group_size,
+                                    const uint16_t *d_out, int M, float *d_x,
+                                    q4gsw_stream_t stream);
+
+/*
+ * Fused Q/K/V forward ([P3]).  packed_qkv is q4gsw_prepack of the
+ * row-concatenated codes [Nq+Nk+Nv, K] and scales [G, Nq+Nk+Nv].
+ *   y_q fp32 [M, Nq], y_k fp32 [M, Nk], y_v fp32 [M, Nv]: three distinct buffers.
+ * Nq, Nk, Nv > 0 and multiples of 8.
+ */
+Q4GSW_API q4gsw_status q4gsw_qkv_fwd(const void *packed_qkv, int Nq, int Nk, int Nv,
+                           int K, int group_size,
+                           const uint16_t *x, int M,
+                           float *y_q, float *y_k, float *y_v,
+                           q4gsw_stream_t stream);
+
+/* Debug export: codes uint8 [N, K] back out of a packed blob. */
+Q4GSW_API q4gsw_status q4gsw_unpack(const void *packed, int N, int K, int group_size,
+                          uint8_t *codes, q4gsw_stream_t stream);
+
+/*
+ * Debug export: the dequantised weight [N, K] as the kernels see it.
+ *   w32  fp32, (code - 8) * scale computed exactly (may be NULL)
+ *   w16  fp16 bits, the tensor-core operand fp16_RNE((code - 8) * scale)
+ *        (may be NULL; at least one of w32 / w16 must be given)
+ */
+Q4GSW_API q4gsw_status q4gsw_dequant(const void *packed, int N, int K, int group_size,
+                           float *w32, uint16_t *w16, q4gsw_stream_t stream);
+
+/* Thread-local description of the kernel route the last call on this thread
+ * enqueued (for example "gemv_fwd nt=1 splitk=8"); never NULL. */
+Q4GSW_API const char *q4gsw_last_route(void);
+
+/* Static text for a status code; never NULL. */
+Q4GSW_API const char *q4gsw_status_str(q4gsw_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4GSW_H */

@@ -1,0 +1,84 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every function that include/q4gsw.h declares, sizes blobs like the layout
+definition, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as o
+from bit_group_quantized_q4gsw_b200 import binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "q4gsw.h")).read()
+    return re.findall(r"Q4GSW_API\s+[\w\s\*]*?\b(q4gsw_\w+)\s*\(", text)
+
+
+def test_library_exports_every_declared_function():
+    lib = b.library()
+    names = declared_functions()
+    assert len(names) == 10
+    assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_is_the_in_tree_build():
+    lib = b.library()
+    assert os.path.samefile(lib._name, b.LIB_PATH)
+
+
+@pytest.mark.parametrize("N,K,gs", [(64, 128, 32), (2048, 2048, 32), (14336, 4096, 128), (8, 64, 64), (24, 192, 16)])
+def test_packed_bytes_matches_layout_definition(N, K, gs):
+    assert b.q4gsw_packed_bytes(N, K, gs) == o.packed_layout(N, K, gs)["total_bytes"]
+
+
+@pytest.mark.parametrize("N,K,gs,status", [
+    (0, 128, 32, 2), (64, 0, 32, 2), (62, 128, 32, 2), (64, 130, 32, 2), (64, 128, 30, 2),
+    (68, 128, 32, 3), (64, 96, 32, 3), (64, 128, 48, 4), (64, 128, 8, 4), (64, 128, 256, 4),
+])
+def test_bad_shapes_are_rejected_on_the_host(N, K, gs, status):
+    lib = b.library()
+    assert lib.q4gsw_packed_bytes(N, K, gs) == 0
+    fake = 0x100000  # never dereferenced: the shape check fails first
+    assert lib.q4gsw_linear_fwd(fake, N, K, gs, fake, 4, fake, None) == status
+    assert lib.q4gsw_linear_bwd_input(fake, N, K, gs, fake, 4, fake, None) == status
+
+
+def test_null_alignment_size_and_empty_batch():
+    lib = b.library()
+    fake = 0x100000
+    assert lib.q4gsw_linear_fwd(None, 64, 128, 32, fake, 4, fake, None) == 1
+    assert lib.q4gsw_linear_fwd(fake, 64, 128, 32, fake + 8, 4, fake, None) == 3
+    assert lib.q4gsw_linear_fwd(fake, 64, 128, 32, fake, -1, fake, None) == 2
+    assert lib.q4gsw_linear_fwd(None, 64, 128, 32, None, 0, None, None) == 0       # empty batch
+    assert b.q4gsw_last_route() == "empty"
+    assert lib.q4gsw_linear_bwd_input(fake, 64, 128, 32, None, 4, fake, None) == 1
+    assert lib.q4gsw_prepack(fake, fake, 64, 128, 32, fake, 100, None) == 7         # blob too small
+    assert lib.q4gsw_prepack(fake, None, 64, 128, 32, fake, 1 << 20, None) == 1
+    assert lib.q4gsw_prepack(fake + 4, fake, 64, 128, 32, fake, 1 << 20, None) == 3
+    assert lib.q4gsw_unpack(fake, 64, 128, 32, None, None) == 1
+    assert lib.q4gsw_dequant(fake, 64, 128, 32, None, None, None) == 1
+    assert lib.q4gsw_dequant(fake, 64, 128, 32, fake + 4, None, None) == 3
+
+
+def test_qkv_split_rules():
+    lib = b.library()
+    fake = 0x100000
+    q = lambda Nq, Nk, Nv, M=4: lib.q4gsw_qkv_fwd(fake, Nq, Nk, Nv, 128, 32, fake, M, fake, fake, fake, None)
+    assert q(0, 16, 16) == 2
+    assert q(64, 12, 16) == 2 or q(64, 12, 16) == 3
+    assert q(64, 20, 20) == 3          # multiples of 4 but not of 8
+    assert q(64, 16, 16, M=0) == 0
+    assert lib.q4gsw_qkv_fwd(fake, 64, 16, 16, 128, 32, fake, 4, fake, None, fake, None) == 1
+
+
+def test_status_strings_and_version():
+    assert b.q4gsw_layout_version() == o.LAYOUT_VERSION == 1
+    for s in range(8):
+        assert b.q4gsw_status_str(s)
+    assert b.q4gsw_status_str(99) == "unknown status"

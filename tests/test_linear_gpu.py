@@ -1,0 +1,221 @@
+"""GPU forward, input gradient and fused Q/K/V against the oracle.
+
+Floating-point results: every element within 4e-3 * sum |a||w| of the fp64
+oracle, and exactly 0 where that bound is 0.  Integer-exact inputs (all
+products and partial sums exact in fp32): bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+from bit_group_quantized_q4gsw_b200 import workloads as wl
+from helpers import assert_within_bound, bits, cuda, pack_on_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def q():
+    import bit_group_quantized_q4gsw_b200 as m
+    return m
+
+
+def run_fwd(inp, gs):
+    blob = pack_on_gpu(inp, gs)
+    N, K = inp.codes.shape
+    y = q().q4gsw_linear_fwd(blob, N, K, gs, cuda(inp.x))
+    torch.cuda.synchronize()
+    return y.cpu().numpy(), q().q4gsw_last_route()
+
+
+def run_bwd(inp, gs):
+    blob = pack_on_gpu(inp, gs)
+    N, K = inp.codes.shape
+    dx = q().q4gsw_linear_bwd_input(blob, N, K, gs, cuda(inp.d_out))
+    torch.cuda.synchronize()
+    return dx.cpu().numpy(), q().q4gsw_last_route()
+
+
+def check_fwd(inp, gs, rows=None):
+    y, route = run_fwd(inp, gs)
+    if rows is None:
+        ref, bnd = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), gs)
+    else:
+        ref, bnd = o.linear_fwd_rows(bits(inp.x), inp.codes, bits(inp.scales), gs, rows)
+        y = y[rows]
+    return assert_within_bound(y, ref, bnd, what=f"fwd {inp.shape.name} [{route}]")
+
+
+def check_bwd(inp, gs, rows=None):
+    dx, route = run_bwd(inp, gs)
+    if rows is None:
+        ref, bnd = o.linear_bwd_input(bits(inp.d_out), inp.codes, bits(inp.scales), gs)
+    else:
+        ref, bnd = o.linear_bwd_input_rows(bits(inp.d_out), inp.codes, bits(inp.scales), gs, rows)
+        dx = dx[rows]
+    return assert_within_bound(dx, ref, bnd, what=f"bwd {inp.shape.name} [{route}]")
+
+
+# ----------------------------------------------------------------------------- the five workloads
+def test_tiny_config_fwd_bwd():
+    sh = wl.tiny()[0]
+    inp = wl.make_inputs(sh)
+    check_fwd(inp, sh.group_size)
+    check_bwd(inp, sh.group_size)
+
+
+@pytest.mark.parametrize("sh", wl.decode(), ids=lambda s: s.name)
+def test_decode_config_fwd(sh):
+    check_fwd(wl.make_inputs(sh), sh.group_size)
+
+
+@pytest.mark.parametrize("sh", wl.adapter(), ids=lambda s: s.name)
+def test_adapter_config_fwd_bwd(sh):
+    inp = wl.make_inputs(sh)
+    check_fwd(inp, sh.group_size)
+    check_bwd(inp, sh.group_size)
+
+
+def _sample_rows(M, seed):
+    if M <= 1024:
+        return None
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([np.arange(8), np.arange(M - 8, M), rng.choice(M, 240, replace=False)]))
+
+
+@pytest.mark.parametrize("sh", wl.sweep(), ids=lambda s: s.name)
+def test_sweep_config_fwd_bwd(sh):
+    inp = wl.make_inputs(sh)
+    rows = _sample_rows(sh.M, sh.seed)
+    check_fwd(inp, sh.group_size, rows)
+    check_bwd(inp, sh.group_size, rows)
+
+
+@pytest.mark.parametrize("sh", wl.qkv(), ids=lambda s: s.name)
+def test_qkv_config(sh):
+    inp = wl.make_inputs(sh)
+    Nq, Nk, Nv = sh.splits
+    blob = pack_on_gpu(inp, sh.group_size)
+    yq, yk, yv = q().q4gsw_qkv_fwd(blob, Nq, Nk, Nv, sh.K, sh.group_size, cuda(inp.x))
+    torch.cuda.synchronize()
+    route = q().q4gsw_last_route()
+    assert route.startswith("qkv")
+    refs = o.qkv_fwd(bits(inp.x), inp.codes, bits(inp.scales), sh.group_size, Nq, Nk, Nv)
+    for got, (ref, bnd), name in zip((yq, yk, yv), refs, "qkv"):
+        assert_within_bound(got.cpu().numpy(), ref, bnd, what=f"qkv {name} M={sh.M} [{route}]")
+
+
+# ----------------------------------------------------------------------------- exact cases
+@pytest.mark.parametrize("M,N,K,gs", [(1, 64, 128, 32), (5, 136, 320, 64), (16, 64, 1024, 16),
+                                      (17, 128, 256, 32), (130, 256, 512, 128), (508, 192, 384, 32)])
+def test_integer_exact_inputs_are_bit_exact(M, N, K, gs):
+    inp = wl.integer_exact_inputs(M, N, K, gs, seed=M * 31 + N)
+    y, r1 = run_fwd(inp, gs)
+    ref, _ = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), gs)
+    assert np.array_equal(y.astype(np.float64), ref), r1
+    dx, r2 = run_bwd(inp, gs)
+    refb, _ = o.linear_bwd_input(bits(inp.d_out), inp.codes, bits(inp.scales), gs)
+    assert np.array_equal(dx.astype(np.float64), refb), r2
+
+
+@pytest.mark.parametrize("M", [1, 12, 200])
+def test_one_hot_probes(M):
+    N, K, gs = 64, 256, 32
+    rng = np.random.default_rng(M)
+    scales = rng.uniform(0.5, 2.0, (K // gs, N)).astype(np.float16)
+    for n0, k0 in ((0, 0), (1, 31), (2, 32), (17, 63), (40, 64), (63, 255), (33, 130)):
+        codes = np.full((N, K), 8, np.uint8)
+        codes[n0, k0] = 9
+        x = np.zeros((M, K), np.float16)
+        x[:, k0] = 1.0
+        d = np.zeros((M, N), np.float16)
+        d[:, n0] = 1.0
+        inp = wl.Inputs(x=x, codes=codes, scales=scales, d_out=d, shape=wl.Shape("probe", M, N, K, gs, 0))
+        y, _ = run_fwd(inp, gs)
+        want = np.zeros((M, N), np.float32)
+        want[:, n0] = np.float32(scales[k0 // gs, n0])
+        assert np.array_equal(y, want), (n0, k0)
+        dx, _ = run_bwd(inp, gs)
+        want = np.zeros((M, K), np.float32)
+        want[:, k0] = np.float32(scales[k0 // gs, n0])
+        assert np.array_equal(dx, want), (n0, k0)
+
+
+def test_zero_point_codes_give_exact_zeros():
+    inp = wl.random_inputs(24, 64, 256, 32, seed=3)
+    inp.codes[:] = 8
+    y, _ = run_fwd(inp, 32)
+    dx, _ = run_bwd(inp, 32)
+    assert not y.any() and not dx.any()
+
+
+def test_scale_homogeneity_is_exact():
+    inp = wl.random_inputs(6, 128, 512, 64, seed=4)
+    y1, _ = run_fwd(inp, 64)
+    inp.scales = (inp.scales * np.float16(2)).astype(np.float16)
+    y2, _ = run_fwd(inp, 64)
+    assert np.array_equal(y2, 2 * y1)
+
+
+@pytest.mark.parametrize("M", [3, 64])
+def test_adjoint_identity(M):
+    inp = wl.random_inputs(M, 256, 512, 32, seed=M)
+    y, _ = run_fwd(inp, 32)
+    dx, _ = run_bwd(inp, 32)
+    d = inp.d_out.astype(np.float64)
+    x = inp.x.astype(np.float64)
+    lhs = float(np.sum(d * y))
+    rhs = float(np.sum(dx * x))
+    w = np.abs(o.dequant_w32(inp.codes, bits(inp.scales), 32).astype(np.float64))
+    scale = float(np.sum((np.abs(d) @ w) * np.abs(x)))
+    assert abs(lhs - rhs) <= 4e-3 * scale
+
+
+def test_qkv_equals_three_separate_forwards():
+    Nq, Nk, Nv, K, gs, M = 128, 64, 64, 256, 32, 20
+    inp = wl.integer_exact_inputs(M, Nq + Nk + Nv, K, gs, seed=11)
+    blob = pack_on_gpu(inp, gs)
+    yq, yk, yv = q().q4gsw_qkv_fwd(blob, Nq, Nk, Nv, K, gs, cuda(inp.x))
+    for (lo, hi), got in zip(((0, Nq), (Nq, Nq + Nk), (Nq + Nk, Nq + Nk + Nv)), (yq, yk, yv)):
+        part = wl.Inputs(x=inp.x, codes=inp.codes[lo:hi].copy(), scales=inp.scales[:, lo:hi].copy(),
+                         d_out=inp.d_out, shape=inp.shape)
+        ysep, _ = run_fwd(part, gs)
+        assert np.array_equal(got.cpu().numpy(), ysep)
+
+
+# ----------------------------------------------------------------------------- edges
+def test_empty_batch_leaves_outputs_untouched():
+    m = q()
+    inp = wl.random_inputs(1, 64, 128, 32, seed=2)
+    blob = pack_on_gpu(inp, 32)
+    y = torch.full((0, 64), 1.0, device="cuda")
+    m.q4gsw_linear_fwd(blob, 64, 128, 32, torch.empty((0, 128), dtype=torch.float16, device="cuda"), y)
+    assert m.q4gsw_last_route() == "empty"
+
+
+@pytest.mark.parametrize("M", [1, 2, 7, 8, 9, 15, 16, 17, 33, 127, 129])
+def test_ragged_token_counts(M):
+    inp = wl.random_inputs(M, 72, 192, 64, seed=100 + M)
+    check_fwd(inp, 64)
+    check_bwd(inp, 64)
+
+
+@pytest.mark.parametrize("N,K,gs", [(8, 64, 64), (24, 64, 16), (40, 448, 64), (1032, 576, 32)])
+def test_odd_weight_shapes(N, K, gs):
+    inp = wl.random_inputs(9, N, K, gs, seed=N + K)
+    check_fwd(inp, gs)
+    check_bwd(inp, gs)
+
+
+def test_non_default_stream():
+    m = q()
+    inp = wl.random_inputs(4, 128, 256, 32, seed=8)
+    blob = pack_on_gpu(inp, 32)
+    s = torch.cuda.Stream()
+    x = cuda(inp.x)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        y = m.q4gsw_linear_fwd(blob, 128, 256, 32, x)
+    s.synchronize()
+    ref, bnd = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), 32)
+    assert_within_bound(y.cpu().numpy(), ref, bnd)
