@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libq4gsw.so")
 Q4GSW_OK = 0
 STATUS_NAMES = {0: "Q4GSW_OK", 1: "Q4GSW_ERR_NULL", 2: "Q4GSW_ERR_SHAPE", 3: "Q4GSW_ERR_ALIGN",
                 4: "Q4GSW_ERR_UNSUPPORTED", 5: "Q4GSW_ERR_CODE_RANGE", 6: "Q4GSW_ERR_CUDA",
-                7: "Q4GSW_ERR_SIZE"}
+                7: "Q4GSW_ERR_SIZE", 8: "Q4GSW_ERR_TIMEOUT"}
 
 # (name, restype, argtypes) of every function declared in include/q4gsw.h
 _VP, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -32,6 +32,7 @@ SIGNATURES = [
     ("q4gsw_linear_fwd", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
     ("q4gsw_linear_bwd_input", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
     ("q4gsw_qkv_fwd", _I, [_VP, _I, _I, _I, _I, _I, _VP, _I, _VP, _VP, _VP, _VP]),
+    ("q4gsw_device_error_check", _I, [_VP]),
     ("q4gsw_unpack", _I, [_VP, _I, _I, _I, _VP, _VP]),
     ("q4gsw_dequant", _I, [_VP, _I, _I, _I, _VP, _VP, _VP]),
     ("q4gsw_last_route", ctypes.c_char_p, []),
@@ -163,6 +164,13 @@ def q4gsw_qkv_fwd(packed_qkv: torch.Tensor, Nq: int, Nk: int, Nv: int, K: int, g
                                  _dev(yk, torch.float32, "y_k", 2), _dev(yv, torch.float32, "y_v", 2), _stream(x))
     _check("q4gsw_qkv_fwd", st)
     return yq, yk, yv
+
+
+def q4gsw_device_error_check(device=None) -> None:
+    """Raise Q4gswError(Q4GSW_ERR_TIMEOUT) if a kernel wait ran out since the last check."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = library().q4gsw_device_error_check(torch.cuda.current_stream(dev).cuda_stream)
+    _check("q4gsw_device_error_check", st)
 
 
 def q4gsw_unpack(packed: torch.Tensor, N: int, K: int, group_size: int) -> torch.Tensor:

@@ -44,6 +44,10 @@ q4gsw_status check_weight_shape(int N, int K, int gs) {
 
 q4gsw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? Q4GSW_OK : Q4GSW_ERR_CUDA; }
 
+// Token counts up to this run the tensor-core GEMV (weight streaming); above
+// it the tcgen05 GEMM.
+constexpr int kGemvMaxM = 16;
+
 }  // namespace
 
 extern "C" {
@@ -67,6 +71,7 @@ const char* q4gsw_status_str(q4gsw_status s) {
     case Q4GSW_ERR_CODE_RANGE: return "code above 15";
     case Q4GSW_ERR_CUDA: return "CUDA runtime error";
     case Q4GSW_ERR_SIZE: return "buffer too small";
+    case Q4GSW_ERR_TIMEOUT: return "a kernel wait ran out (results of the calls since the last check are invalid)";
   }
   return "unknown status";
 }
@@ -94,8 +99,11 @@ q4gsw_status q4gsw_linear_fwd(const void* packed, int N, int K, int group_size, 
   if (!packed || !x || !y) return Q4GSW_ERR_NULL;
   if (!aligned16(packed) || !aligned16(x) || !aligned16(y)) return Q4GSW_ERR_ALIGN;
   char route[160];
-  cudaError_t e = launch_gemv_fwd(packed, N, K, group_size, x, M, single_output(y, N), stream, route,
-                                  sizeof(route));
+  cudaError_t e = M <= kGemvMaxM
+                      ? launch_gemv_fwd(packed, N, K, group_size, x, M, single_output(y, N), stream, route,
+                                        sizeof(route))
+                      : launch_gemm_fwd(packed, N, K, group_size, x, M, single_output(y, N), stream, route,
+                                        sizeof(route));
   set_route(route);
   return from_cuda(e);
 }
@@ -109,7 +117,9 @@ q4gsw_status q4gsw_linear_bwd_input(const void* packed, int N, int K, int group_
   if (!packed || !d_out || !d_x) return Q4GSW_ERR_NULL;
   if (!aligned16(packed) || !aligned16(d_out) || !aligned16(d_x)) return Q4GSW_ERR_ALIGN;
   char route[160];
-  cudaError_t e = launch_gemv_bwd(packed, N, K, group_size, d_out, M, d_x, stream, route, sizeof(route));
+  cudaError_t e = M <= kGemvMaxM
+                      ? launch_gemv_bwd(packed, N, K, group_size, d_out, M, d_x, stream, route, sizeof(route))
+                      : launch_gemm_bwd(packed, N, K, group_size, d_out, M, d_x, stream, route, sizeof(route));
   set_route(route);
   return from_cuda(e);
 }
@@ -130,11 +140,19 @@ q4gsw_status q4gsw_qkv_fwd(const void* packed_qkv, int Nq, int Nk, int Nv, int K
     return Q4GSW_ERR_ALIGN;
   OutSplit out{y_q, y_k, y_v, Nq, Nq + Nk, N};
   char route[120];
-  cudaError_t e = launch_gemv_fwd(packed_qkv, N, K, group_size, x, M, out, stream, route, sizeof(route));
+  cudaError_t e = M <= kGemvMaxM ? launch_gemv_fwd(packed_qkv, N, K, group_size, x, M, out, stream, route, sizeof(route))
+                                 : launch_gemm_fwd(packed_qkv, N, K, group_size, x, M, out, stream, route, sizeof(route));
   char full[160];
   snprintf(full, sizeof(full), "qkv %s", route);
   set_route(full);
   return from_cuda(e);
+}
+
+q4gsw_status q4gsw_device_error_check(q4gsw_stream_t stream) {
+  unsigned int v = 0;
+  q4gsw_status st = from_cuda(read_and_clear_device_error(stream, &v));
+  if (st != Q4GSW_OK) return st;
+  return v ? Q4GSW_ERR_TIMEOUT : Q4GSW_OK;
 }
 
 q4gsw_status q4gsw_unpack(const void* packed, int N, int K, int group_size, uint8_t* codes,

@@ -1,0 +1,462 @@
+// q4gsw_gemm_sm100.cu - tcgen05 / tensor-memory GEMM route of the q4gsw linear
+// layer for larger token counts (sm_100a).
+//
+//   forward   y[m,n]   = sum_k x[m,k]     * w[n,k]     (w[n,k] = (code - 8) * s[k/gs, n])
+//   backward  d_x[m,k] = sum_n d_out[m,n] * w[n,k]
+// ("[ExecuTorch][Vulkan] Add et_vk.linear_q4gsw_backward kernel (4-bit
+// input-grad)", PR description; the fused Q/K/V forward of "[ExecuTorch][WebGPU]
+// Replace broad QKV fusion with BK64 kernel" is the forward with its output
+// columns scattered over three buffers.)
+//
+// One CTA computes a 128-token x 256-feature tile of the output, optionally for
+// one slice of the contraction (split-K, reduced in a cluster through
+// distributed shared memory).  Warp roles:
+//   warp 0       TMA producer: activation tile (fp16, 128-byte swizzle) and the
+//                packed-code tile of each 64-deep contraction stage;
+//   warp 1       allocates tensor memory and issues tcgen05.mma from one thread;
+//   warps 2..9   dequantise the stage's codes into fp16 (code - 8) * scale,
+//                written straight into the 128-byte-swizzled layout the MMA
+//                descriptors read, then run the epilogue (tcgen05.ld -> global).
+// The forward reads the weight tile [256 n][64 k] as a K-major B operand; the
+// backward writes the same kind of tile ([64 n][256 k], k contiguous) and reads
+// it as an MN-major B operand, so both directions use one packed blob and one
+// dequantisation routine.
+#include <cooperative_groups.h>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+
+#include "q4gsw_common.cuh"
+#include "q4gsw_internal.h"
+#include "q4gsw_sm100.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace q4gsw {
+
+// OR of the codes of waits that timed out (read and cleared by the host).
+__device__ unsigned int g_device_error = 0;
+
+namespace gemm {
+
+constexpr int BM = 128;                 // tokens per tile (MMA M)
+constexpr int BN = 256;                 // output features per tile (MMA N)
+constexpr int TK = 64;                  // contraction depth per stage
+constexpr int STAGES = 3;
+constexpr int kDequantWarps = 8;
+constexpr int kThreads = 32 * (2 + kDequantWarps);
+constexpr int A_BYTES = BM * TK * 2;    // activation tile, 16 KB
+constexpr int P_BYTES = BN / 2 * TK;    // packed codes, 8 KB
+constexpr int W_BYTES = BN * TK * 2;    // dequantised fp16 weights, 32 KB
+constexpr int STAGE_BYTES = A_BYTES + P_BYTES + W_BYTES;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr int TMEM_COLS = 256;
+
+static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+static_assert(BM * BN * 4 <= STAGES * STAGE_BYTES, "split-K staging must fit in the stage buffers");
+
+struct Args {
+  const uint8_t* packed;
+  OutSplit out;
+  int M, N, K, gs;
+  int out_cols;       // forward: N, backward: K
+  int stages_total;   // contraction / TK
+};
+
+struct SmemCtl {
+  uint64_t full[STAGES];
+  uint64_t wready[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t accfull;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ __half2 load_scale2(const __half* scales, int N, int g, int n, bool valid) {
+  if (!valid) return u32_as_h2(0u);
+  return u32_as_h2(ldg_nc_u32(scales + (size_t)g * N + n));
+}
+
+template <bool BWD>
+__global__ void __launch_bounds__(kThreads, 1)
+q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
+                  const Args args) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
+  volatile int* abort_flag = &ctl->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;    // first output feature of the tile
+  const int m0 = blockIdx.y * BM;    // first token of the tile
+  const int S = gridDim.z, split = blockIdx.z;
+  const int st_begin = (int)((long long)split * args.stages_total / S);
+  const int st_end = (int)((long long)(split + 1) * args.stages_total / S);
+  const int nit = st_end - st_begin;
+
+  auto stA = [&](int s) { return smem + s * STAGE_BYTES; };
+  auto stP = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+  auto stW = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + P_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->wready[s], kDequantWarps);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    mbar_init(&ctl->accfull, 1);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&map_act);
+    prefetch_tmap(&map_pk);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < nit; ++it) {
+        const int s = it % STAGES;
+        if (it >= STAGES && !mbar_wait(&ctl->empty[s], ((it / STAGES) - 1) & 1, abort_flag, &g_device_error, 1u))
+          break;
+        const int kc = (st_begin + it) * TK;
+        mbar_arrive_expect_tx(&ctl->full[s], A_BYTES + P_BYTES);
+        tma_load_2d(stA(s), &map_act, &ctl->full[s], kc, m0);
+        if (!BWD) {
+          tma_load_2d(stP(s), &map_pk, &ctl->full[s], kc, n0 / 2);
+        } else {
+          tma_load_2d(stP(s), &map_pk, &ctl->full[s], n0, kc / 2);
+          tma_load_2d(stP(s) + P_BYTES / 2, &map_pk, &ctl->full[s], n0 + 128, kc / 2);
+        }
+        issued = it + 1;
+      }
+      // never leave with copies in flight: wait for the last fill of each stage
+      for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
+        mbar_wait_teardown(&ctl->full[it % STAGES], (it / STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(BM, BN, BWD);
+      bool ok = true;
+      int done = 0;
+      for (int it = 0; it < nit && ok; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        ok = mbar_wait(&ctl->full[s], ph, abort_flag, &g_device_error, 2u) &&
+             mbar_wait(&ctl->wready[s], ph, abort_flag, &g_device_error, 4u);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(stA(s)), w0 = smem_u32(stW(s));
+#pragma unroll
+        for (int ks = 0; ks < TK / 16; ++ks) {
+          const uint64_t ad = smem_desc_sw128(a0 + 32 * ks, 16, 1024);
+          const uint64_t bd = BWD ? smem_desc_sw128(w0 + ks * 2048, 8192, 1024)
+                                  : smem_desc_sw128(w0 + 32 * ks, 16, 1024);
+          mma_f16_ss(tmem, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&ctl->empty[s]);
+        done = it + 1;
+      }
+      (void)done;
+      mma_commit(&ctl->accfull);
+      mma_commit(&ctl->drain);
+      mbar_wait_teardown(&ctl->drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ dequantisation
+    const int td = threadIdx.x - 64;
+    const Layout L = layout_of(args.N, args.K, args.gs);
+    const __half* scales = reinterpret_cast<const __half*>(args.packed + L.scales_offset);
+    int p, u, j = 0;
+    if (!BWD) {
+      p = td >> 1;
+      u = td & 1;
+    } else {
+      j = td >> 6;
+      p = (td & 63) >> 1;
+      u = td & 1;
+    }
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % STAGES;
+      const int kc = (st_begin + it) * TK;
+      // scales of this stage (issued before the wait to hide their latency)
+      __half2 sc[4];
+      int n_even;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (!BWD) {
+          n_even = n0 + 2 * p;
+          const int k = kc + 16 * i + 8 * u;
+          sc[i] = load_scale2(scales, args.N, k / args.gs, n_even, n_even < args.N);
+        } else {
+          n_even = kc + 2 * p;
+          const int k = n0 + 64 * j + 16 * i + 8 * u;
+          sc[i] = load_scale2(scales, args.N, k / args.gs, n_even, n_even < args.N && k < args.K);
+        }
+      }
+      if (!mbar_wait(&ctl->full[s], (it / STAGES) & 1, abort_flag, &g_device_error, 8u)) break;
+      uint4 c0, c1;
+      if (!BWD) {
+        const uint8_t* prow = stP(s) + p * 64;
+        const int sw = (p >> 1) & 3;
+        c0 = *reinterpret_cast<const uint4*>(prow + 16 * ((2 * u) ^ sw));
+        c1 = *reinterpret_cast<const uint4*>(prow + 16 * ((2 * u + 1) ^ sw));
+      } else {
+        const uint8_t* prow = stP(s) + (j >> 1) * (P_BYTES / 2) + p * 128;
+        const int cc = (j & 1) * 4 + 2 * u;
+        c0 = *reinterpret_cast<const uint4*>(prow + 16 * (cc ^ (p & 7)));
+        c1 = *reinterpret_cast<const uint4*>(prow + 16 * ((cc + 1) ^ (p & 7)));
+      }
+      const uint32_t wlo[4] = {c0.x, c0.y, c0.z, c0.w};
+      const uint32_t whi[4] = {c1.x, c1.y, c1.z, c1.w};
+      uint8_t* wt = BWD ? stW(s) + j * 8192 : stW(s);
+      const int re = 2 * p, ro = 2 * p + 1;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const RowPairs a = codes_minus8_rows(wlo[i]);   // columns +0..3 of this 8-column chunk
+        const RowPairs b = codes_minus8_rows(whi[i]);   // columns +4..7
+        const __half2 se = __low2half2(sc[i]), so = __high2half2(sc[i]);
+        const uint4 ve = make_uint4(h2_as_u32(__hmul2(a.ev01, se)), h2_as_u32(__hmul2(a.ev23, se)),
+                                    h2_as_u32(__hmul2(b.ev01, se)), h2_as_u32(__hmul2(b.ev23, se)));
+        const uint4 vo = make_uint4(h2_as_u32(__hmul2(a.od01, so)), h2_as_u32(__hmul2(a.od23, so)),
+                                    h2_as_u32(__hmul2(b.od01, so)), h2_as_u32(__hmul2(b.od23, so)));
+        const int chunk = 2 * i + u;
+        *reinterpret_cast<uint4*>(wt + re * 128 + 16 * (chunk ^ (re & 7))) = ve;
+        *reinterpret_cast<uint4*>(wt + ro * 128 + 16 * (chunk ^ (ro & 7))) = vo;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->wready[s]);
+    }
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  // Warps 2..9: warp w reads TMEM lanes 32 (w % 4) .. +31 (tokens) and columns
+  // [128 h, 128 h + 128) with h = (w - 2) / 4.
+  const bool epi = warp >= 2;
+  float* stage_f32 = reinterpret_cast<float*>(smem);   // split-K staging [128][256], 16-byte chunks swizzled
+  bool have_acc = false;
+  if (epi) have_acc = mbar_wait(&ctl->accfull, 0, abort_flag, &g_device_error, 16u);
+  if (epi && have_acc) {
+    tc_fence_after();
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    const int row = 32 * q + lane;
+    const int m = m0 + row;
+#pragma unroll 1
+    for (int c32 = 0; c32 < 4; ++c32) {
+      const int col = 128 * h + 32 * c32;
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, r);
+      tmem_wait_ld();
+      if (S == 1) {
+        if (m < args.M) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const int n = n0 + col + 4 * v;
+            if (n >= args.out_cols) break;
+            const float4 val = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            const OutSplit& o = args.out;
+            float* dst;
+            if (n < o.n1) dst = o.y0 + (size_t)m * o.n1 + n;
+            else if (n < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (n - o.n1);
+            else dst = o.y2 + (size_t)m * (o.N - o.n2) + (n - o.n2);
+            *reinterpret_cast<float4*>(dst) = val;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const int chunk = (col >> 2) + v;   // 16-byte chunk of the 1 KB row
+          const float4 val = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          *reinterpret_cast<float4*>(stage_f32 + row * 256 + 4 * (chunk ^ (row & 7))) = val;
+        }
+      }
+    }
+  }
+  if (S > 1) {
+    // every thread of every CTA of the cluster passes both barriers, aborted or not
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int r = (int)cluster.block_rank();
+    const int row_b = r * BM / S, row_e = (r + 1) * BM / S;
+    if (!*abort_flag) {
+      for (int idx = threadIdx.x; idx < (row_e - row_b) * 64; idx += kThreads) {
+        const int row = row_b + (idx >> 6), chunk = idx & 63;
+        const int m = m0 + row, n = n0 + 4 * chunk;
+        if (m >= args.M || n >= args.out_cols) continue;
+        const int off = row * 256 + 4 * (chunk ^ (row & 7));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < S; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, q) + off);
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const OutSplit& o = args.out;
+        float* dst;
+        if (n < o.n1) dst = o.y0 + (size_t)m * o.n1 + n;
+        else if (n < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (n - o.n1);
+        else dst = o.y2 + (size_t)m * (o.N - o.n2) + (n - o.n2);
+        *reinterpret_cast<float4*>(dst) = acc;
+      }
+    }
+    cluster.sync();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t dim0, uint64_t dim1,
+                        uint64_t stride1_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {dim0, dim1};
+  cuuint64_t strides[1] = {stride1_bytes};
+  cuuint32_t box[2] = {box0, box1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int sm_count_gemm() {
+  static int cached = 0;
+  if (!cached) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached = n > 0 ? n : 148;
+  }
+  return cached;
+}
+
+template <bool BWD>
+static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, const uint16_t* act, int M,
+                                    OutSplit out, cudaStream_t stream, char* route, int route_len) {
+  using namespace gemm;
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  CUtensorMap map_act, map_pk;
+  bool ok;
+  if (!BWD) {
+    ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, K, M, (uint64_t)K * 2, TK, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BN / 2, CU_TENSOR_MAP_SWIZZLE_64B);
+  } else {
+    ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, N, M, (uint64_t)N * 2, TK, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, TK / 2,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+
+  Args a;
+  a.packed = pk;
+  a.out = out;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.gs = gs;
+  a.out_cols = BWD ? K : N;
+  const int contraction = BWD ? N : K;
+  a.stages_total = (contraction + TK - 1) / TK;
+
+  const int tiles_n = (a.out_cols + BN - 1) / BN;
+  const int tiles_m = (M + BM - 1) / BM;
+  const int tiles = tiles_n * tiles_m;
+  int S = 1;
+  while (S < 8 && tiles * (S + 1) <= sm_count_gemm() && a.stages_total / (S + 1) >= 4) ++S;
+
+  auto kern = q4gsw_gemm_kernel<BWD>;
+  static bool attr_done[2][64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_done[BWD][dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_done[BWD][dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles_n, tiles_m, S);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = S;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, a);
+  if (route)
+    snprintf(route, route_len, "tcgen05_gemm_%s launches=1 tile=%dx%dx%d stages=%d grid=%dx%dx%d", BWD ? "bwd" : "fwd",
+             BM, BN, TK, STAGES, tiles_n, tiles_m, S);
+  return e;
+}
+
+cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
+                            cudaStream_t stream, char* route, int route_len) {
+  return launch_gemm_impl<false>(packed, N, K, gs, x, M, out, stream, route, route_len);
+}
+
+cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
+                            cudaStream_t stream, char* route, int route_len) {
+  return launch_gemm_impl<true>(packed, N, K, gs, d_out, M, single_output(d_x, K), stream, route, route_len);
+}
+
+cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int* host_value) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(host_value, g_device_error, sizeof(unsigned int), 0,
+                                            cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  if (*host_value) {
+    e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamSynchronize(stream);
+  }
+  return e;
+}
+
+}  // namespace q4gsw

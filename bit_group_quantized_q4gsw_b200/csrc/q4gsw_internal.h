@@ -32,4 +32,14 @@ cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint
 cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M,
                             float* d_x, cudaStream_t stream, char* route, int route_len);
 
+// tcgen05 GEMM routes (any M >= 1; used above the GEMV range).
+cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
+                            cudaStream_t stream, char* route, int route_len);
+cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
+                            cudaStream_t stream, char* route, int route_len);
+
+// Reads (and clears when set) the device word in which kernels record waits
+// that ran out; synchronises `stream`.
+cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int* host_value);
+
 }  // namespace q4gsw

@@ -70,7 +70,8 @@ typedef enum {
   Q4GSW_ERR_UNSUPPORTED = 4,  /* group size not a power of two in [16, K] */
   Q4GSW_ERR_CODE_RANGE = 5,   /* q4gsw_prepack saw a code > 15 */
   Q4GSW_ERR_CUDA = 6,         /* the CUDA runtime reported an error */
-  Q4GSW_ERR_SIZE = 7          /* a byte count passed in is too small */
+  Q4GSW_ERR_SIZE = 7,         /* a byte count passed in is too small */
+  Q4GSW_ERR_TIMEOUT = 8       /* a kernel's bounded wait ran out (q4gsw_device_error_check) */
 } q4gsw_status;
 
 /* Version of the packed-weight byte layout written by q4gsw_prepack. */
@@ -109,7 +110,7 @@ Q4GSW_API q4gsw_status q4gsw_prepack(const uint8_t *codes, const uint16_t *scale
  *   packed  a blob from q4gsw_prepack for the same (N, K, gs)
  *   x       fp16 [M, K];   y  fp32 [M, N] (overwritten)
  * Route: M <= 16 a tensor-core GEMV over the streamed packed weight; larger M
- * a tcgen05 GEMM that dequantises into shared memory.
+ * a tcgen05 GEMM that dequantises into shared memory (q4gsw_last_route()).
  */
 Q4GSW_API q4gsw_status q4gsw_linear_fwd(const void *packed, int N, int K, int group_size,
                               const uint16_t *x, int M, float *y,
@@ -136,6 +137,16 @@ Q4GSW_API q4gsw_status q4gsw_qkv_fwd(const void *packed_qkv, int Nq, int Nk, int
                            const uint16_t *x, int M,
                            float *y_q, float *y_k, float *y_v,
                            q4gsw_stream_t stream);
+
+/*
+ * Kernel health check.  Every wait inside this library's kernels is bounded
+ * (about one second); a wait that runs out makes its kernel stop early and
+ * record the event in a device-side status word instead of hanging.  This call
+ * waits for `stream`, reads that word for the current device and clears it:
+ * Q4GSW_ERR_TIMEOUT means the outputs of the calls since the previous check are
+ * not valid.  Returns Q4GSW_OK otherwise.
+ */
+Q4GSW_API q4gsw_status q4gsw_device_error_check(q4gsw_stream_t stream);
 
 /* Debug export: codes uint8 [N, K] back out of a packed blob. */
 Q4GSW_API q4gsw_status q4gsw_unpack(const void *packed, int N, int K, int group_size,

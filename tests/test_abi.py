@@ -21,7 +21,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = b.library()
     names = declared_functions()
-    assert len(names) == 10
+    assert len(names) == 11
     assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
     for n in names:
         assert hasattr(lib, n), n
@@ -79,6 +79,6 @@ def test_qkv_split_rules():
 
 def test_status_strings_and_version():
     assert b.q4gsw_layout_version() == o.LAYOUT_VERSION == 1
-    for s in range(8):
+    for s in range(9):
         assert b.q4gsw_status_str(s)
     assert b.q4gsw_status_str(99) == "unknown status"

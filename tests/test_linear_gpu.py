@@ -219,3 +219,32 @@ def test_non_default_stream():
     s.synchronize()
     ref, bnd = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), 32)
     assert_within_bound(y.cpu().numpy(), ref, bnd)
+
+
+# ----------------------------------------------------------------------------- tcgen05 GEMM route
+@pytest.mark.parametrize("M,N,K,gs", [(17, 256, 256, 32), (40, 72, 192, 64), (130, 1032, 576, 32),
+                                      (129, 264, 448, 16), (300, 520, 320, 64), (64, 256, 4096, 128)])
+def test_gemm_route_tails(M, N, K, gs):
+    inp = wl.random_inputs(M, N, K, gs, seed=M + N + K)
+    check_fwd(inp, gs)
+    assert q().q4gsw_last_route().startswith("tcgen05_gemm_fwd")
+    check_bwd(inp, gs)
+    assert q().q4gsw_last_route().startswith("tcgen05_gemm_bwd")
+
+
+def test_gemm_split_k_cluster_reduction():
+    # one 128x256 output tile and a long contraction: the route splits K over a cluster
+    inp = wl.integer_exact_inputs(100, 256, 4096, 64, seed=9)
+    y, route = run_fwd(inp, 64)
+    assert "x8" in route.split("grid=")[1], route
+    ref, _ = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), 64)
+    assert np.array_equal(y.astype(np.float64), ref)
+    inp = wl.integer_exact_inputs(100, 4096, 256, 64, seed=10)
+    dx, route = run_bwd(inp, 64)
+    assert "x8" in route.split("grid=")[1], route
+    ref, _ = o.linear_bwd_input(bits(inp.d_out), inp.codes, bits(inp.scales), 64)
+    assert np.array_equal(dx.astype(np.float64), ref)
+
+
+def test_no_kernel_wait_ran_out():
+    q().q4gsw_device_error_check()
