@@ -528,6 +528,33 @@ def run_sweep(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- profiling cases
+def run_case(args):
+    """Launch one operation `--iters` times (for ncu captures); no timing."""
+    import torch
+    import bit_group_quantized_q4gsw_b200 as q
+    device = torch.device("cuda", 0)
+    name, kind = args.case.rsplit(":", 1)
+    sh = wl.by_name(name)
+    M = args.case_m or sh.M
+    inp = wl.make_inputs(sh, M=M)
+    pk = q.q4gsw_prepack(torch.from_numpy(inp.codes).to(device), torch.from_numpy(inp.scales).to(device),
+                         sh.group_size)
+    a = torch.from_numpy(inp.d_out if kind == "bwd" else inp.x).to(device)
+    for _ in range(args.iters):
+        if kind == "qkv":
+            Nq, Nk, Nv = sh.splits
+            q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, a)
+        elif kind == "fwd":
+            q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a)
+        else:
+            q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a)
+    torch.cuda.synchronize()
+    q.q4gsw_device_error_check()
+    print(json.dumps({"case": args.case, "M": M, "iters": args.iters, "route": q.q4gsw_last_route()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -538,6 +565,9 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--only", default="")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default="", help="SHAPE:DIR, e.g. adapter_up_M512:fwd (profiling launches)")
+    ap.add_argument("--case-m", type=int, default=0)
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -548,6 +578,8 @@ def main():
         return run_reference(args, rank, world)
     if args.sweep:
         return run_sweep(args)
+    if args.case:
+        return run_case(args)
     if world > 1:
         import datetime
         import torch
