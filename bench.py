@@ -472,6 +472,7 @@ def run_sweep(args):
     device = torch.device("cuda", 0)
     peaks = measured_peaks()
     shapes = wl.tiny() + wl.decode() + wl.qkv() + wl.adapter() + wl.sweep()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     if args.only:
         shapes = [s for s in shapes if args.only in s.name]
     for sh in shapes:
@@ -515,13 +516,26 @@ def run_sweep(args):
             e1.record()
             torch.cuda.synchronize()
             t = e0.elapsed_time(e1) / (reps * iters) / 1e3
+            # one launch after an L2 flush (a 256 MB write), timed alone: the
+            # launch is enqueued while the flush still runs, so host launch
+            # latency stays outside the events
+            singles = []
+            for r in range(3):
+                torch.cuda.synchronize()
+                flush.fill_(r)
+                e0.record()
+                fn(packs[r % R])
+                e1.record()
+                torch.cuda.synchronize()
+                singles.append(e0.elapsed_time(e1) * 1e3)
+            t1 = sorted(singles)[1]
             fl = op_flops(kind, sh)
             by = op_bytes(kind, sh)
             print(json.dumps({"shape": sh.name, "dir": kind, "M": sh.M, "N": sh.N, "K": sh.K, "gs": sh.group_size,
                               "us": t * 1e6, "tflops": fl / t / 1e12, "gbs": by / t / 1e9,
                               "weight_gbs": wb / t / 1e9, "frac_tc": fl / t / 1e12 / peaks["tflops"],
                               "frac_hbm_measured": by / t / 1e9 / peaks["hbm_gbs"], "frac_hbm_8tbs": by / t / 8e12,
-                              "route": q.q4gsw_last_route(), "copies": R}), flush=True)
+                              "us_single_cold": t1, "route": q.q4gsw_last_route(), "copies": R}), flush=True)
             del g
         del packs, first
         torch.cuda.empty_cache()

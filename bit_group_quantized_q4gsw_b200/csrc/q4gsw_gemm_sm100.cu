@@ -44,52 +44,77 @@ namespace gemm {
 constexpr int BM = 128;                 // tokens per tile (MMA M)
 constexpr int BN = 256;                 // output features per tile (MMA N)
 constexpr int TK = 64;                  // contraction depth per stage
-constexpr int STAGES = 3;
-constexpr int kDequantWarps = 8;
+constexpr int ST = 4;                   // TMA ring: activation + codes + scales
+constexpr int WST = 3;                  // dequantised-weight ring
+constexpr int kGroupWarps = 8;          // warps of one dequantisation group
+constexpr int kGroups = 2;              // groups take alternate stages
+constexpr int kDequantWarps = kGroupWarps * kGroups;
 constexpr int kThreads = 32 * (2 + kDequantWarps);
 constexpr int A_BYTES = BM * TK * 2;    // activation tile, 16 KB
 constexpr int P_BYTES = BN / 2 * TK;    // packed codes, 8 KB
+constexpr int SC_BYTES = 2048;          // scale rows of one stage (at most)
 constexpr int W_BYTES = BN * TK * 2;    // dequantised fp16 weights, 32 KB
-constexpr int STAGE_BYTES = A_BYTES + P_BYTES + W_BYTES;
-constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr int OFF_A = 0;
+constexpr int OFF_P = OFF_A + ST * A_BYTES;
+constexpr int OFF_W = OFF_P + ST * P_BYTES;
+constexpr int OFF_SC = OFF_W + WST * W_BYTES;
+constexpr int OFF_CTL = OFF_SC + ST * SC_BYTES;
+constexpr int CTL_BYTES = 256;
+constexpr int SMEM_BYTES = OFF_CTL + CTL_BYTES + 1024;
 constexpr int TMEM_COLS = 256;
 
-static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
-static_assert(BM * BN * 4 <= STAGES * STAGE_BYTES, "split-K staging must fit in the stage buffers");
+static_assert(OFF_P % 1024 == 0 && OFF_W % 1024 == 0 && OFF_SC % 1024 == 0, "1024-byte aligned regions");
+static_assert(BM * BN * 4 <= OFF_SC, "split-K staging must fit below the scale buffers");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct Args {
-  const uint8_t* packed;
   OutSplit out;
   int M, N, K, gs;
   int out_cols;       // forward: N, backward: K
   int stages_total;   // contraction / TK
+  int sc_bytes;       // bytes of the scale box loaded per stage
 };
 
 struct SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t wready[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[ST];
+  uint64_t empty[ST];
+  uint64_t wready[WST];
+  uint64_t wempty[WST];
   uint64_t accfull;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(SmemCtl) <= CTL_BYTES, "control block");
 
-__device__ __forceinline__ __half2 load_scale2(const __half* scales, int N, int g, int n, bool valid) {
-  if (!valid) return u32_as_h2(0u);
-  return u32_as_h2(ldg_nc_u32(scales + (size_t)g * N + n));
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 template <bool BWD>
 __global__ void __launch_bounds__(kThreads, 1)
 q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
-                  const Args args) {
+                  const __grid_constant__ CUtensorMap map_sc, const Args args) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + OFF_CTL);
   volatile int* abort_flag = &ctl->abort;
+  const uint32_t sbase = smem_u32(smem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN;    // first output feature of the tile
@@ -99,15 +124,15 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
   const int st_end = (int)((long long)(split + 1) * args.stages_total / S);
   const int nit = st_end - st_begin;
 
-  auto stA = [&](int s) { return smem + s * STAGE_BYTES; };
-  auto stP = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
-  auto stW = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + P_BYTES; };
-
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ctl->full[s], 1);
-      mbar_init(&ctl->wready[s], kDequantWarps);
-      mbar_init(&ctl->empty[s], 1);
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], 1);
+    }
+    for (int i = 0; i < WST; ++i) {
+      mbar_init(&ctl->wready[i], kGroupWarps);
+      mbar_init(&ctl->wempty[i], 1);
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
@@ -115,6 +140,7 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
     fence_mbar_init();
     prefetch_tmap(&map_act);
     prefetch_tmap(&map_pk);
+    prefetch_tmap(&map_sc);
   }
   if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, TMEM_COLS);
@@ -128,40 +154,57 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued = 0;
-      for (int it = 0; it < nit; ++it) {
-        const int s = it % STAGES;
-        if (it >= STAGES && !mbar_wait(&ctl->empty[s], ((it / STAGES) - 1) & 1, abort_flag, &g_device_error, 1u))
-          break;
+      auto load_weights = [&](int it) {
+        const int s = it % ST;
         const int kc = (st_begin + it) * TK;
-        mbar_arrive_expect_tx(&ctl->full[s], A_BYTES + P_BYTES);
-        tma_load_2d(stA(s), &map_act, &ctl->full[s], kc, m0);
+        uint8_t* pk = smem + OFF_P + s * P_BYTES;
+        uint8_t* sc = smem + OFF_SC + s * SC_BYTES;
         if (!BWD) {
-          tma_load_2d(stP(s), &map_pk, &ctl->full[s], kc, n0 / 2);
+          tma_load_2d(pk, &map_pk, &ctl->full[s], kc, n0 / 2);
+          tma_load_2d(sc, &map_sc, &ctl->full[s], n0, kc >> (__ffs(args.gs) - 1));
         } else {
-          tma_load_2d(stP(s), &map_pk, &ctl->full[s], n0, kc / 2);
-          tma_load_2d(stP(s) + P_BYTES / 2, &map_pk, &ctl->full[s], n0 + 128, kc / 2);
+          tma_load_2d(pk, &map_pk, &ctl->full[s], n0, kc / 2);
+          tma_load_2d(pk + P_BYTES / 2, &map_pk, &ctl->full[s], n0 + 128, kc / 2);
+          tma_load_2d(sc, &map_sc, &ctl->full[s], kc, n0 >> (__ffs(args.gs) - 1));
         }
+      };
+      auto load_act = [&](int it) {
+        const int s = it % ST;
+        tma_load_2d(smem + OFF_A + s * A_BYTES, &map_act, &ctl->full[s], (st_begin + it) * TK, m0);
+      };
+      // The packed weight is constant: the first stages' codes and scales are
+      // requested before waiting for the previous kernel of the stream, which
+      // may still be producing the activations.
+      const int pre = nit < ST ? nit : ST;
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&ctl->full[it], A_BYTES + P_BYTES + args.sc_bytes);
+        load_weights(it);
+      }
+      griddep_wait();
+      for (int it = 0; it < pre; ++it) load_act(it);
+      int issued = pre;
+      for (int it = pre; it < nit; ++it) {
+        const int s = it % ST;
+        if (!mbar_wait(&ctl->empty[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
+        mbar_arrive_expect_tx(&ctl->full[s], A_BYTES + P_BYTES + args.sc_bytes);
+        load_weights(it);
+        load_act(it);
         issued = it + 1;
       }
       // never leave with copies in flight: wait for the last fill of each stage
-      for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
-        mbar_wait_teardown(&ctl->full[it % STAGES], (it / STAGES) & 1);
+      for (int it = (issued > ST ? issued - ST : 0); it < issued; ++it)
+        mbar_wait_teardown(&ctl->full[it % ST], (it / ST) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(BM, BN, BWD);
-      bool ok = true;
-      int done = 0;
-      for (int it = 0; it < nit && ok; ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        ok = mbar_wait(&ctl->full[s], ph, abort_flag, &g_device_error, 2u) &&
-             mbar_wait(&ctl->wready[s], ph, abort_flag, &g_device_error, 4u);
-        if (!ok) break;
+      for (int it = 0; it < nit; ++it) {
+        const int s = it % ST, w = it % WST;
+        if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 2u)) break;
+        if (!mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(stA(s)), w0 = smem_u32(stW(s));
+        const uint32_t a0 = sbase + OFF_A + s * A_BYTES, w0 = sbase + OFF_W + w * W_BYTES;
 #pragma unroll
         for (int ks = 0; ks < TK / 16; ++ks) {
           const uint64_t ad = smem_desc_sw128(a0 + 32 * ks, 16, 1024);
@@ -170,18 +213,19 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
           mma_f16_ss(tmem, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(&ctl->empty[s]);
-        done = it + 1;
+        mma_commit(&ctl->wempty[w]);
       }
-      (void)done;
       mma_commit(&ctl->accfull);
       mma_commit(&ctl->drain);
       mbar_wait_teardown(&ctl->drain, 0);
     }
   } else {
     // ------------------------------------------------------------ dequantisation
-    const int td = threadIdx.x - 64;
-    const Layout L = layout_of(args.N, args.K, args.gs);
-    const __half* scales = reinterpret_cast<const __half*>(args.packed + L.scales_offset);
+    // Group grp takes the iterations it == grp (mod 2); inside a group, thread
+    // td owns pair row p and half u of each 64-column block (backward: also
+    // the 64-column block j of the 256-column tile).
+    const int grp = (warp - 2) / kGroupWarps;
+    const int td = threadIdx.x - 64 - grp * 32 * kGroupWarps;
     int p, u, j = 0;
     if (!BWD) {
       p = td >> 1;
@@ -191,65 +235,76 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       p = (td & 63) >> 1;
       u = td & 1;
     }
-    for (int it = 0; it < nit; ++it) {
-      const int s = it % STAGES;
-      const int kc = (st_begin + it) * TK;
-      // scales of this stage (issued before the wait to hide their latency)
-      __half2 sc[4];
-      int n_even;
+    // Per-thread offsets, fixed for the whole contraction: packed-code chunks
+    // (64-byte swizzle forward, 128-byte backward), scale words (the scale
+    // row of each 8-column chunk is the same in every stage because stages
+    // start on 64-column boundaries), dequantised-tile chunks (128-byte swizzle).
+    const int gsl = __ffs(args.gs) - 1;
+    uint32_t pk_off0, pk_off1, sc_off[4];
+    if (!BWD) {
+      const int sz = (p >> 1) & 3;
+      pk_off0 = p * 64 + 16 * ((2 * u) ^ sz);
+      pk_off1 = p * 64 + 16 * ((2 * u + 1) ^ sz);
+      // stage base column kc: with gs >= 64 the 64 columns sit in one group,
+      // with gs < 64 the stage starts a group; either way the row is
+      // ((kc mod gs) + 16 i + 8 u) >> gsl = (16 i + 8 u) >> gsl for gs < 64, else 0
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (!BWD) {
-          n_even = n0 + 2 * p;
-          const int k = kc + 16 * i + 8 * u;
-          sc[i] = load_scale2(scales, args.N, k / args.gs, n_even, n_even < args.N);
-        } else {
-          n_even = kc + 2 * p;
-          const int k = n0 + 64 * j + 16 * i + 8 * u;
-          sc[i] = load_scale2(scales, args.N, k / args.gs, n_even, n_even < args.N && k < args.K);
-        }
-      }
-      if (!mbar_wait(&ctl->full[s], (it / STAGES) & 1, abort_flag, &g_device_error, 8u)) break;
-      uint4 c0, c1;
-      if (!BWD) {
-        const uint8_t* prow = stP(s) + p * 64;
-        const int sw = (p >> 1) & 3;
-        c0 = *reinterpret_cast<const uint4*>(prow + 16 * ((2 * u) ^ sw));
-        c1 = *reinterpret_cast<const uint4*>(prow + 16 * ((2 * u + 1) ^ sw));
-      } else {
-        const uint8_t* prow = stP(s) + (j >> 1) * (P_BYTES / 2) + p * 128;
-        const int cc = (j & 1) * 4 + 2 * u;
-        c0 = *reinterpret_cast<const uint4*>(prow + 16 * (cc ^ (p & 7)));
-        c1 = *reinterpret_cast<const uint4*>(prow + 16 * ((cc + 1) ^ (p & 7)));
-      }
+      for (int i = 0; i < 4; ++i) sc_off[i] = (args.gs < 64 ? ((16 * i + 8 * u) >> gsl) : 0) * 512 + 4 * p;
+    } else {
+      const int cc = (j & 1) * 4 + 2 * u;
+      pk_off0 = (j >> 1) * (P_BYTES / 2) + p * 128 + 16 * (cc ^ (p & 7));
+      pk_off1 = (j >> 1) * (P_BYTES / 2) + p * 128 + 16 * ((cc + 1) ^ (p & 7));
+      const int base = n0 & (args.gs - 1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sc_off[i] = ((base + 64 * j + 16 * i + 8 * u) >> gsl) * 128 + 4 * p;
+    }
+    const int re = 2 * p, ro = 2 * p + 1;
+    uint32_t st_off_e[4], st_off_o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int chunk = 2 * i + u;
+      st_off_e[i] = (BWD ? j * 8192 : 0) + re * 128 + 16 * (chunk ^ (re & 7));
+      st_off_o[i] = (BWD ? j * 8192 : 0) + ro * 128 + 16 * (chunk ^ (ro & 7));
+    }
+    for (int it = grp; it < nit; it += kGroups) {
+      const int s = it % ST, w = it % WST;
+      if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
+      if (it >= WST && !mbar_wait(&ctl->wempty[w], ((it / WST) - 1) & 1, abort_flag, &g_device_error, 32u)) break;
+      const uint32_t pk = sbase + OFF_P + s * P_BYTES;
+      const uint32_t sc = sbase + OFF_SC + s * SC_BYTES;
+      const uint4 c0 = lds128(pk + pk_off0);
+      const uint4 c1 = lds128(pk + pk_off1);
+      uint32_t sw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sw[i] = lds32(sc + sc_off[i]);
       const uint32_t wlo[4] = {c0.x, c0.y, c0.z, c0.w};
       const uint32_t whi[4] = {c1.x, c1.y, c1.z, c1.w};
-      uint8_t* wt = BWD ? stW(s) + j * 8192 : stW(s);
-      const int re = 2 * p, ro = 2 * p + 1;
+      const uint32_t wt = sbase + OFF_W + w * W_BYTES;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const RowPairs a = codes_minus8_rows(wlo[i]);   // columns +0..3 of this 8-column chunk
         const RowPairs b = codes_minus8_rows(whi[i]);   // columns +4..7
-        const __half2 se = __low2half2(sc[i]), so = __high2half2(sc[i]);
+        const __half2 s2 = u32_as_h2(sw[i]);
+        const __half2 se = __low2half2(s2), so = __high2half2(s2);
         const uint4 ve = make_uint4(h2_as_u32(__hmul2(a.ev01, se)), h2_as_u32(__hmul2(a.ev23, se)),
                                     h2_as_u32(__hmul2(b.ev01, se)), h2_as_u32(__hmul2(b.ev23, se)));
         const uint4 vo = make_uint4(h2_as_u32(__hmul2(a.od01, so)), h2_as_u32(__hmul2(a.od23, so)),
                                     h2_as_u32(__hmul2(b.od01, so)), h2_as_u32(__hmul2(b.od23, so)));
-        const int chunk = 2 * i + u;
-        *reinterpret_cast<uint4*>(wt + re * 128 + 16 * (chunk ^ (re & 7))) = ve;
-        *reinterpret_cast<uint4*>(wt + ro * 128 + 16 * (chunk ^ (ro & 7))) = vo;
+        sts128(wt + st_off_e[i], ve);
+        sts128(wt + st_off_o[i], vo);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->wready[s]);
+      if (lane == 0) mbar_arrive(&ctl->wready[w]);
     }
   }
 
   // ---------------------------------------------------------------- epilogue
-  // Warps 2..9: warp w reads TMEM lanes 32 (w % 4) .. +31 (tokens) and columns
-  // [128 h, 128 h + 128) with h = (w - 2) / 4.
+  // Warps 2..17: warp w reads TMEM lanes 32 (w % 4) .. +31 (tokens) and the 64
+  // accumulator columns [64 h, 64 h + 64) with h = (w - 2) / 4.
   const bool epi = warp >= 2;
   float* stage_f32 = reinterpret_cast<float*>(smem);   // split-K staging [128][256], 16-byte chunks swizzled
+  griddep_wait();   // outputs may still be read by the previous kernel of the stream
   bool have_acc = false;
   if (epi) have_acc = mbar_wait(&ctl->accfull, 0, abort_flag, &g_device_error, 16u);
   if (epi && have_acc) {
@@ -258,8 +313,8 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
     const int row = 32 * q + lane;
     const int m = m0 + row;
 #pragma unroll 1
-    for (int c32 = 0; c32 < 4; ++c32) {
-      const int col = 128 * h + 32 * c32;
+    for (int c32 = 0; c32 < 2; ++c32) {
+      const int col = 64 * h + 32 * c32;
       uint32_t r[32];
       tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, r);
       tmem_wait_ld();
@@ -303,8 +358,8 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
         if (m >= args.M || n >= args.out_cols) continue;
         const int off = row * 256 + 4 * (chunk ^ (row & 7));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < S; ++q) {
-          const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, q) + off);
+        for (int qq = 0; qq < S; ++qq) {
+          const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + off);
           acc.x += v.x;
           acc.y += v.y;
           acc.z += v.z;
@@ -375,22 +430,34 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
                                     OutSplit out, cudaStream_t stream, char* route, int route_len) {
   using namespace gemm;
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
-  CUtensorMap map_act, map_pk;
+  CUtensorMap map_act, map_pk, map_sc;
+  const Layout L = layout_of(N, K, gs);
+  const void* scales = pk + L.scales_offset;
+  const int G = K / gs;
   bool ok;
+  int sc_bytes;
   if (!BWD) {
+    const int rows = TK / gs > 1 ? TK / gs : 1;   // scale groups of one 64-column stage
+    sc_bytes = rows * BN * 2;
     ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, K, M, (uint64_t)K * 2, TK, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BN / 2, CU_TENSOR_MAP_SWIZZLE_64B);
+         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BN / 2, CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, BN, rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
+    const int rows = BN / gs > 1 ? BN / gs : 1;   // scale groups of one 256-column tile
+    sc_bytes = rows * TK * 2;
     ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, N, M, (uint64_t)N * 2, TK, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, TK / 2,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, TK, rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
   }
-  if (!ok) return cudaErrorInvalidValue;
+  if (!ok || sc_bytes > SC_BYTES) return cudaErrorInvalidValue;
 
   Args a;
-  a.packed = pk;
+  a.sc_bytes = sc_bytes;
   a.out = out;
   a.M = M;
   a.N = N;
@@ -420,17 +487,19 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = S;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, a);
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, a);
   if (route)
-    snprintf(route, route_len, "tcgen05_gemm_%s launches=1 tile=%dx%dx%d stages=%d grid=%dx%dx%d", BWD ? "bwd" : "fwd",
-             BM, BN, TK, STAGES, tiles_n, tiles_m, S);
+    snprintf(route, route_len, "tcgen05_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d",
+             BWD ? "bwd" : "fwd", BM, BN, TK, ST, WST, tiles_n, tiles_m, S);
   return e;
 }
 

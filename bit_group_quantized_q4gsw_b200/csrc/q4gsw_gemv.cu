@@ -22,6 +22,7 @@
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdio>
 
 #include "q4gsw_common.cuh"
@@ -37,17 +38,20 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // ---------------------------------------------------------------------------
 // Forward
 // ---------------------------------------------------------------------------
-// grid = (N/16 row tiles, S contraction splits, ceil(M/16) token slices),
-// cluster = (1, S, 1).  Warp u = split*4 + warp owns the 64-column blocks
-// [u*KB/U, (u+1)*KB/U) of its row tile (KB = K/64, U = 4 S).
+// grid = (ceil(N/16) row tiles, S contraction splits, ceil(M/16) token
+// slices), cluster = (1, S, 1).  Warp u = split*4 + warp owns the 64-column
+// blocks [u*KB/U, (u+1)*KB/U) of its row tile (KB = K/64, U = 4 S).
 // NT = number of 8-token MMA tiles (1: M <= 8 per slice, 2: M <= 16).
 // SPG = 16-column steps per scale group (1: gs 16, 2: gs 32, 4: gs >= 64).
+constexpr int kFwdPF = 2;   // 64-column blocks per pipeline chunk (two chunks in flight)
+
 template <int NT, int SPG>
-__global__ void __launch_bounds__(kGemvThreads) gemv_fwd_kernel(const uint8_t* __restrict__ packed,
-                                                                const __half* __restrict__ x, OutSplit out,
-                                                                int M, int N, int K, int gs) {
+__global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 8 : 5)
+gemv_fwd_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x, OutSplit out, int M, int N,
+                int K, int gs) {
   __shared__ float red[kGemvWarps][16][16];  // [warp][token][row]
   __shared__ float cta_part[16][16];         // [token][row]
+  griddep_launch_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -58,6 +62,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_fwd_kernel(const uint8_t* _
 
   const Layout L = layout_of(N, K, gs);
   const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
+  const int gsl = __ffs(gs) - 1;  // gs is a power of two
   const int p_raw = tile * 8 + g;  // nibble pair of this lane: rows 2p (even) and 2p+1 (odd)
   const bool pvalid = p_raw < (N >> 1);  // the last tile holds 4 pairs when N % 16 == 8
   const int p = pvalid ? p_raw : 0;
@@ -67,7 +72,45 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_fwd_kernel(const uint8_t* _
   const int U = S * kGemvWarps, u = split * kGemvWarps + warp;
   const int b_begin = (int)((long long)u * KB / U), b_end = (int)((long long)(u + 1) * KB / U);
 
-  // token rows this lane feeds into B (column g of each 8-token tile)
+  // Two partial-sum sets (even / odd 16-column steps) keep two independent
+  // MMA chains in flight; a finished group is scaled into acc in fp32.
+  float acc[NT][4], part[2][NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[j][c] = part[0][j][c] = part[1][j][c] = 0.f;
+
+  constexpr int PF = kFwdPF;
+  constexpr int NGB = (SPG == 4) ? 1 : 4 / SPG;    // scale groups per block
+  auto load_chunk = [&](int b0, uint4 (&w)[PF], uint32_t (&sc)[PF][NGB]) {
+#pragma unroll
+    for (int q = 0; q < PF; ++q) {
+      const int b = b0 + q;
+      const bool in = b < b_end;
+      w[q] = (in && pvalid) ? ldg_stream_v4(row + 64 * b) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int r = 0; r < NGB; ++r) {
+        const int col = 64 * b + r * (64 / NGB);
+        sc[q][r] = in ? ldg_nc_u32(scales + (size_t)(col >> gsl) * N + 2 * p) : 0u;
+      }
+    }
+  };
+  auto flush = [&](uint32_t s_word) {  // scale one finished group into acc
+    const __half2 s2 = u32_as_h2(s_word);
+    const float se = __low2float(s2), so = __high2float(s2);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      acc[j][0] = fmaf(part[0][j][0] + part[1][j][0], se, acc[j][0]);
+      acc[j][1] = fmaf(part[0][j][1] + part[1][j][1], se, acc[j][1]);
+      acc[j][2] = fmaf(part[0][j][2] + part[1][j][2], so, acc[j][2]);
+      acc[j][3] = fmaf(part[0][j][3] + part[1][j][3], so, acc[j][3]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) part[0][j][c] = part[1][j][c] = 0.f;
+    }
+  };
+
+  // x fragments of one 64-column block: lane (g, t) feeds token 8j + g with
+  // columns 64b + 16i + 4t .. +3 of step i (two LDG.64 per step, held for the block).
   const __half* xrow[NT];
   bool xvalid[NT];
 #pragma unroll
@@ -77,52 +120,45 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_fwd_kernel(const uint8_t* _
     xrow[j] = x + (size_t)(tok0 + (xvalid[j] ? tok : 0)) * K + 4 * t;
   }
 
-  float acc[NT][4], part[NT][4];
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[j][c] = part[j][c] = 0.f;
-
-  auto flush = [&](int col) {  // scale the group that holds column `col` into acc
-    const __half2 s2 = *reinterpret_cast<const __half2*>(scales + (size_t)(col / gs) * N + 2 * p);
-    const float se = __low2float(s2), so = __high2float(s2);
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      acc[j][0] = fmaf(part[j][0], se, acc[j][0]);
-      acc[j][1] = fmaf(part[j][1], se, acc[j][1]);
-      acc[j][2] = fmaf(part[j][2], so, acc[j][2]);
-      acc[j][3] = fmaf(part[j][3], so, acc[j][3]);
-      part[j][0] = part[j][1] = part[j][2] = part[j][3] = 0.f;
-    }
-  };
-
-  constexpr int PF = 4;  // 64-column blocks in flight per lane
-  for (int b0 = b_begin; b0 < b_end; b0 += PF) {
-    uint4 wv[PF];
-#pragma unroll
-    for (int q = 0; q < PF; ++q)
-      wv[q] = (b0 + q < b_end && pvalid) ? ldg_stream_v4(row + 64 * (b0 + q)) : make_uint4(0, 0, 0, 0);
+  auto compute_chunk = [&](int b0, const uint4 (&w)[PF], const uint32_t (&sc)[PF][NGB]) {
 #pragma unroll
     for (int q = 0; q < PF; ++q) {
       const int b = b0 + q;
       if (b >= b_end) break;
-      const uint32_t words[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
+      uint2 xv[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[j][i] = xvalid[j] ? ldg_nc_v2(xrow[j] + 64 * b + 16 * i) : make_uint2(0u, 0u);
+      const uint32_t words[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int col = 64 * b + 16 * i;  // first column of this 16-column step
         const RowPairs r = codes_minus8_rows(words[i]);
         const uint32_t a[4] = {h2_as_u32(r.ev01), h2_as_u32(r.od01), h2_as_u32(r.ev23), h2_as_u32(r.od23)};
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          uint2 xv = make_uint2(0u, 0u);
-          if (xvalid[j]) xv = ldg_nc_v2(xrow[j] + col);
-          const uint32_t bf[2] = {xv.x, xv.y};
-          mma_16816(part[j], a, bf);
+          const uint32_t bf[2] = {xv[j][i].x, xv[j][i].y};
+          mma_16816(part[i & 1][j], a, bf);
         }
-        if (SPG == 1 || (SPG == 2 && (i & 1))) flush(col);
+        if (SPG == 1) flush(sc[q][i]);
+        if (SPG == 2 && (i & 1)) flush(sc[q][i >> 1]);
       }
-      if (SPG == 4 && (((b + 1) * 64) % gs == 0 || b + 1 == b_end)) flush(64 * b);
+      if (SPG == 4 && ((((b + 1) * 64) & (gs - 1)) == 0 || b + 1 == b_end)) flush(sc[q][0]);
     }
+  };
+
+  // The packed weight is constant: its first chunk streams in before the
+  // wait for the previous kernel of the stream (which may produce x).
+  uint4 wA[PF], wB[PF];
+  uint32_t sA[PF][NGB], sB[PF][NGB];
+  load_chunk(b_begin, wA, sA);
+  griddep_wait();
+  for (int b0 = b_begin; b0 < b_end; b0 += 2 * PF) {
+    load_chunk(b0 + PF, wB, sB);
+    compute_chunk(b0, wA, sA);
+    if (b0 + PF >= b_end) break;
+    load_chunk(b0 + 2 * PF, wA, sA);
+    compute_chunk(b0 + PF, wB, sB);
   }
 
   // D fragment: rows g (even n) and g+8 (odd n), tokens 2t, 2t+1 of tile j.
@@ -162,21 +198,28 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_fwd_kernel(const uint8_t* _
 // ---------------------------------------------------------------------------
 // Backward (input gradient)
 // ---------------------------------------------------------------------------
+// MMA roles: A = weight^T tile (16 output columns k x 16 contraction rows n =
+// 8 nibble pairs; a register holds the (even n, odd n) half2 of ONE byte),
+// B = d_out^T (16 n x 8 tokens), D = 16 k x 8 tokens.
 // grid = (ceil(K/128) column tiles, S contraction splits, ceil(M/16) token
 // slices), cluster = (1, S, 1), kBwdWarps warps per CTA.  A column tile is two
 // 64-column blocks J = 2*tile + (g >> 2); lane (g, t) reads 16 bytes at offset
-// 16 (g & 3) of block J in pair rows pb+t and pb+t+4.  MMA (i, e) has output
-// column c <-> k = 64 J(c) + 16 i + 4 (c & 3) + e.  Warp u = split*W + warp
-// owns the 16-row contraction steps [u*NS/U, (u+1)*NS/U) (NS = N/16).
+// 16 (g & 3) of block J in pair rows pb+t and pb+t+4, i.e. columns
+// k = 64 J + 16 i + 4 (g & 3) + e.  MMA q = 2 i + h maps A row g to
+// e = 2h and row g+8 to e = 2h+1.  Warp u = split*W + warp owns the 16-row
+// contraction steps [u*NS/U, (u+1)*NS/U) (NS = N/16); the next step's loads are
+// issued before the current step is computed.
 constexpr int kBwdWarps = 8;
 constexpr int kBwdThreads = 32 * kBwdWarps;
 
-template <int SPB>  // scale groups per 64-column block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
+template <int NT, int SPB>  // NT 8-token tiles; SPB scale groups per block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
 __global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __restrict__ packed,
                                                                const __half* __restrict__ dout,
                                                                float* __restrict__ dx,
                                                                int M, int N, int K, int gs) {
-  __shared__ float cta_part[16 * 128];  // [token][local column]
+  extern __shared__ float red[];   // [warp][8 NT tokens][128 local columns]
+  float* cta_part = red;           // reused after the warp partials are summed (rank 0 reads peers' copies)
+  griddep_launch_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -186,6 +229,7 @@ __global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __
   const int KB = K >> 6;
   const int J = 2 * blockIdx.x + (g >> 2);  // this lane's 64-column block
   const bool jvalid = J < KB;
+  const int Jc = jvalid ? J : 0;            // lanes past the last block read block 0, never stored
 
   const Layout L = layout_of(N, K, gs);
   const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
@@ -194,94 +238,114 @@ __global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __
   const int U = S * kBwdWarps, u = split * kBwdWarps + warp;
   const int s_begin = (int)((long long)u * NS / U), s_end = (int)((long long)(u + 1) * NS / U);
 
-  // scale group of each 16-column step i of this lane's columns
-  // (lanes past the last block use block 0: their columns are never stored)
-  const int Jc = jvalid ? J : 0;
-  int grp[4];
+  int grp[SPB];   // scale group of the columns of step i (i = q * 4 / SPB .. )
 #pragma unroll
-  for (int i = 0; i < 4; ++i) grp[i] = (64 * Jc + 16 * i + 4 * (g & 3)) / gs;
+  for (int q = 0; q < SPB; ++q) grp[q] = (64 * Jc + 16 * (q * (4 / SPB)) + 4 * (g & 3)) >> (__ffs(gs) - 1);
 
-  const bool tv0 = g < Mz, tv1 = g + 8 < Mz;
-  const __half* drow0 = dout + (size_t)(tok0 + (tv0 ? g : 0)) * N;
-  const __half* drow1 = dout + (size_t)(tok0 + (tv1 ? g + 8 : 0)) * N;
+  bool tv[NT];
+  const __half* drow[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    tv[j] = 8 * j + g < Mz;
+    drow[j] = dout + (size_t)(tok0 + (tv[j] ? 8 * j + g : 0)) * N;
+  }
   const uint8_t* wcol = packed + 64 * Jc + 16 * (g & 3);
 
-  float acc[4][4][4];
+  float acc[NT][8][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int j = 0; j < NT; ++j)
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
+    for (int q = 0; q < 8; ++q)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[i][e][c] = 0.f;
+      for (int c = 0; c < 4; ++c) acc[j][q][c] = 0.f;
 
-  for (int st = s_begin; st < s_end; ++st) {
+  struct StepData {
+    uint4 va, vb;              // packed bytes of pairs pA and pB
+    uint32_t b[NT][2];         // d_out fragments
+    uint32_t sa[SPB], sb[SPB]; // scale half2 of pairs pA, pB per group
+  };
+  auto load_step = [&](int st, StepData& d) {
     const int pA = st * 8 + t;
-    const bool bvalid = pA + 4 < NP;
+    const bool in = st < s_end;
+    const bool bvalid = in && pA + 4 < NP;
     const int pB = bvalid ? pA + 4 : pA;
-    uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
-    if (jvalid) {
-      va = ldg_stream_v4(wcol + (size_t)pA * K);
-      if (bvalid) vb = ldg_stream_v4(wcol + (size_t)pB * K);
+    d.va = (in && jvalid) ? ldg_stream_v4(wcol + (size_t)pA * K) : make_uint4(0, 0, 0, 0);
+    d.vb = (bvalid && jvalid) ? ldg_stream_v4(wcol + (size_t)pB * K) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      d.b[j][0] = (in && tv[j]) ? ldg_nc_u32(drow[j] + 2 * pA) : 0u;
+      d.b[j][1] = (bvalid && tv[j]) ? ldg_nc_u32(drow[j] + 2 * pB) : 0u;
     }
-    uint32_t a[4] = {0u, 0u, 0u, 0u};
-    if (tv0) {
-      a[0] = ldg_nc_u32(drow0 + 2 * pA);
-      if (bvalid) a[2] = ldg_nc_u32(drow0 + 2 * pB);
-    }
-    if (tv1) {
-      a[1] = ldg_nc_u32(drow1 + 2 * pA);
-      if (bvalid) a[3] = ldg_nc_u32(drow1 + 2 * pB);
-    }
-    __half2 sa[SPB], sb[SPB];
 #pragma unroll
     for (int q = 0; q < SPB; ++q) {
-      const int gq = grp[q * (4 / SPB)];
-      sa[q] = u32_as_h2(ldg_nc_u32(scales + (size_t)gq * N + 2 * pA));
-      sb[q] = bvalid ? u32_as_h2(ldg_nc_u32(scales + (size_t)gq * N + 2 * pB)) : u32_as_h2(0u);
+      d.sa[q] = in ? ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pA) : 0u;
+      d.sb[q] = bvalid ? ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pB) : 0u;
     }
-    const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-    const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+  };
+  auto compute_step = [&](const StepData& d) {
+    const uint32_t wa[4] = {d.va.x, d.va.y, d.va.z, d.va.w};
+    const uint32_t wb[4] = {d.vb.x, d.vb.y, d.vb.z, d.vb.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int q = i / (4 / SPB);
+      const __half2 sa = u32_as_h2(d.sa[q]), sb = u32_as_h2(d.sb[q]);
       const ColPairs ca = codes_minus8_cols(wa[i]);
       const ColPairs cb = codes_minus8_cols(wb[i]);
       const __half2 la[4] = {ca.c0, ca.c1, ca.c2, ca.c3};
       const __half2 lb[4] = {cb.c0, cb.c1, cb.c2, cb.c3};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t bf[2] = {h2_as_u32(__hmul2(la[e], sa[q])), h2_as_u32(__hmul2(lb[e], sb[q]))};
-        mma_16816(acc[i][e], a, bf);
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t af[4] = {h2_as_u32(__hmul2(la[2 * h], sa)), h2_as_u32(__hmul2(la[2 * h + 1], sa)),
+                                h2_as_u32(__hmul2(lb[2 * h], sb)), h2_as_u32(__hmul2(lb[2 * h + 1], sb))};
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma_16816(acc[j][2 * i + h], af, d.b[j]);
       }
     }
+  };
+
+  // d_out may come from the previous kernel of the stream: wait before the
+  // first load (the step loads mix weights and d_out).
+  griddep_wait();
+  StepData dA, dB;
+  load_step(s_begin, dA);
+  for (int st = s_begin; st < s_end; st += 2) {
+    load_step(st + 1, dB);
+    compute_step(dA);
+    if (st + 1 >= s_end) break;
+    load_step(st + 2, dA);
+    compute_step(dB);
   }
 
-  // D fragment of MMA (i, e): rows g / g+8 = tokens, columns 2t, 2t+1;
-  // column c -> local output column 64 (c >> 2) + 16 i + 4 (c & 3) + e.
-  // Warps add their partials into cta_part one after another (fixed order).
-  for (int w = 0; w < kBwdWarps; ++w) {
-    if (warp == w) {
+  // Warp partials -> shared memory: D of MMA q = 2i + h, rows g / g+8 = columns
+  // 64 (g >> 2) + 16 i + 4 (g & 3) + 2h (+1), columns 2t, 2t+1 = tokens.
+  float* mine = red + warp * (8 * NT * 128);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+  for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int c = 2 * t + h;
-            const int kl = 64 * (c >> 2) + 16 * i + 4 * (c & 3) + e;
-            if (w == 0) {
-              cta_part[g * 128 + kl] = acc[i][e][h];
-              cta_part[(g + 8) * 128 + kl] = acc[i][e][2 + h];
-            } else {
-              cta_part[g * 128 + kl] += acc[i][e][h];
-              cta_part[(g + 8) * 128 + kl] += acc[i][e][2 + h];
-            }
-          }
+    for (int q = 0; q < 8; ++q) {
+      const int i = q >> 1, h = q & 1;
+      const int kl = 64 * (g >> 2) + 16 * i + 4 * (g & 3) + 2 * h;
+      const int tk = 8 * j + 2 * t;
+      mine[tk * 128 + kl] = acc[j][q][0];
+      mine[(tk + 1) * 128 + kl] = acc[j][q][1];
+      mine[tk * 128 + kl + 1] = acc[j][q][2];
+      mine[(tk + 1) * 128 + kl + 1] = acc[j][q][3];
     }
-    __syncthreads();
+  __syncthreads();
+  float sums[8 * NT * 128 / kBwdThreads];
+#pragma unroll
+  for (int r = 0; r < 8 * NT * 128 / kBwdThreads; ++r) {
+    const int idx = threadIdx.x + r * kBwdThreads;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kBwdWarps; ++w) s += red[w * (8 * NT * 128) + idx];
+    sums[r] = s;
   }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 8 * NT * 128 / kBwdThreads; ++r) cta_part[threadIdx.x + r * kBwdThreads] = sums[r];
   cg::cluster_group cluster = cg::this_cluster();
-  if (S > 1) cluster.sync();
+  if (S > 1) cluster.sync(); else __syncthreads();
   if (cluster.block_rank() == 0) {
     const int kbase = 128 * blockIdx.x;
     const int kw = min(128, K - kbase);
@@ -310,14 +374,22 @@ static int sm_count() {
   return cached;
 }
 
-// Contraction splits: grow S (cluster size) until the grid holds about
-// `warps_target` warps, keeping at least `min_units` contraction units per warp.
-static int pick_splits(long long tiles, int warps_per_cta, int units_per_tile, int min_units, int max_s,
-                       long long warps_target) {
-  int S = 1;
-  while (S * 2 <= max_s && tiles * S * warps_per_cta < warps_target &&
-         units_per_tile / (warps_per_cta * S * 2) >= min_units)
-    S *= 2;
+// Contraction splits S (the cluster size).  Measured on B200 for the decode,
+// MLP and 8B-layer shapes: the forward wants about four CTAs per SM in
+// flight and as little splitting as that allows; the input gradient, whose
+// output tile is narrow, wants about 320 CTAs.  At least `min_units`
+// contraction units stay with each warp.
+static int fwd_splits(long long tiles, int blocks_per_tile) {
+  int S = (int)lround(4.0 * sm_count() / (double)tiles);
+  S = S < 1 ? 1 : S > 8 ? 8 : S;
+  while (S > 1 && blocks_per_tile / (kGemvWarps * S) < 1) --S;
+  return S;
+}
+
+static int bwd_splits(long long tiles, int steps_per_tile, int warps_per_cta) {
+  int S = (int)lround(320.0 / (double)tiles);
+  S = S < 1 ? 1 : S > 16 ? 16 : S;
+  while (S > 1 && steps_per_tile / (warps_per_cta * S) < 2) --S;
   return S;
 }
 
@@ -333,52 +405,71 @@ static cudaError_t launch_cluster(Kern kernel, dim3 grid, int threads, int clust
   cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = cluster_y;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M,
                             OutSplit out, cudaStream_t stream, char* route, int route_len) {
   const int tiles = (N + 15) / 16;
-  const int S = pick_splits(tiles, kGemvWarps, K / 64, 1, 8, 24LL * sm_count());
+  const int zs = (M + 15) / 16;
   const int NT = (M <= 8) ? 1 : 2;
   const int spg = gs == 16 ? 1 : gs == 32 ? 2 : 4;
-  dim3 grid(tiles, S, (M + 15) / 16);
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
   const __half* xh = reinterpret_cast<const __half*>(x);
   cudaError_t err;
-#define Q4_FWD(NT_, SPG_) \
-  err = launch_cluster(gemv_fwd_kernel<NT_, SPG_>, grid, kGemvThreads, S, 0, stream, pk, xh, out, M, N, K, gs)
+  int S = 1;
+#define Q4_FWD(NT_, SPG_)                                                                                       \
+  do {                                                                                                          \
+    S = fwd_splits((long long)tiles * zs, K / 64);                                                             \
+    err = launch_cluster(gemv_fwd_kernel<NT_, SPG_>, dim3(tiles, S, zs), kGemvThreads, S, 0, stream, pk, xh, out, \
+                         M, N, K, gs);                                                                          \
+  } while (0)
   if (NT == 1) {
     if (spg == 1) Q4_FWD(1, 1); else if (spg == 2) Q4_FWD(1, 2); else Q4_FWD(1, 4);
   } else {
     if (spg == 1) Q4_FWD(2, 1); else if (spg == 2) Q4_FWD(2, 2); else Q4_FWD(2, 4);
   }
 #undef Q4_FWD
-  if (route) snprintf(route, route_len, "gemv_fwd launches=1 nt=%d splits=%d zslices=%d", NT, S, (M + 15) / 16);
+  if (route) snprintf(route, route_len, "gemv_fwd launches=1 nt=%d splits=%d zslices=%d", NT, S, zs);
   return err;
 }
 
 cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M,
                             float* d_x, cudaStream_t stream, char* route, int route_len) {
   const int tiles = (K + 127) / 128;
-  const int S = pick_splits(tiles, kBwdWarps, (N + 15) / 16, 2, 16, 24LL * sm_count());
+  const int zs = (M + 15) / 16;
+  const int NT = (M <= 8) ? 1 : 2;
   const int spb = gs >= 64 ? 1 : gs == 32 ? 2 : 4;
-  dim3 grid(tiles, S, (M + 15) / 16);
+  int S = 1;
+  const size_t smem = sizeof(float) * kBwdWarps * 8 * NT * 128;
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
   const __half* dh = reinterpret_cast<const __half*>(d_out);
   cudaError_t err;
-#define Q4_BWD(SPB_) \
-  err = launch_cluster(gemv_bwd_kernel<SPB_>, grid, kBwdThreads, S, 0, stream, pk, dh, d_x, M, N, K, gs)
-  if (spb == 1) Q4_BWD(1); else if (spb == 2) Q4_BWD(2); else Q4_BWD(4);
+#define Q4_BWD(NT_, SPB_)                                                                                         \
+  do {                                                                                                            \
+    err = cudaFuncSetAttribute(gemv_bwd_kernel<NT_, SPB_>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (err == cudaSuccess) {                                                                                     \
+      S = bwd_splits((long long)tiles * zs, (N + 15) / 16, kBwdWarps);                                           \
+      err = launch_cluster(gemv_bwd_kernel<NT_, SPB_>, dim3(tiles, S, zs), kBwdThreads, S, smem, stream, pk, dh,  \
+                           d_x, M, N, K, gs);                                                                     \
+    }                                                                                                             \
+  } while (0)
+  if (NT == 1) {
+    if (spb == 1) Q4_BWD(1, 1); else if (spb == 2) Q4_BWD(1, 2); else Q4_BWD(1, 4);
+  } else {
+    if (spb == 1) Q4_BWD(2, 1); else if (spb == 2) Q4_BWD(2, 2); else Q4_BWD(2, 4);
+  }
 #undef Q4_BWD
-  if (route) snprintf(route, route_len, "gemv_bwd launches=1 splits=%d zslices=%d", S, (M + 15) / 16);
+  if (route) snprintf(route, route_len, "gemv_bwd launches=1 nt=%d splits=%d zslices=%d", NT, S, zs);
   return err;
 }
 

@@ -109,7 +109,7 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ packed, float* __rest
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int k0 = 64 * b + 16 * i + 4 * t;  // columns k0 .. k0+3
-      const int g = k0 / gs;
+      const int g = k0 >> (__ffs(gs) - 1);
       const __half2 s2 = *reinterpret_cast<const __half2*>(scales + (size_t)g * N + 2 * p);
       const __half2 se = __low2half2(s2), so = __high2half2(s2);
       const RowPairs r = codes_minus8_rows(w[i]);

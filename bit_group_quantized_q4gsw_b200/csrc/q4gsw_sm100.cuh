@@ -55,7 +55,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // try_wait suspends the thread for a while inside the hardware before it
+    // reports "not yet", so the abort and clock checks run only every 8 tries
+#pragma unroll 1
+    for (int r = 0; r < 8; ++r)
+      if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) {
       *abort_flag = 1;

@@ -38,6 +38,13 @@
  *     reported by the CUDA runtime returns Q4GSW_ERR_CUDA.
  *   - No CPU fallback exists: every result is computed by this library's
  *     CUDA kernels.  Calls are thread-safe and re-entrant.
+ *   - The compute calls launch with programmatic dependent launch: a call may
+ *     start while the previous kernel on `stream` is still finishing.  It waits
+ *     for that kernel before reading activations or writing outputs, but the
+ *     packed weight is treated as a constant and may be read earlier.  So a
+ *     packed blob must not be written by the kernel enqueued immediately before
+ *     a call that reads it (q4gsw_prepack returns only after its own work is
+ *     done, so a blob it produced is always safe).
  *   - Shapes accepted: N > 0, N % 8 == 0; K > 0, K % 64 == 0; gs a power of
  *     two with 16 <= gs <= K (so K % gs == 0).  [P2]'s own constraints
  *     (multiples of 4) are a superset; the tighter ones come from the packed
