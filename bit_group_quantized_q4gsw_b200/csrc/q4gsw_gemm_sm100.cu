@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdio>
 
 #include "q4gsw_common.cuh"
@@ -44,7 +45,6 @@ namespace gemm {
 constexpr int BM = 128;                 // tokens per tile (MMA M)
 constexpr int BN = 256;                 // output features per tile (MMA N)
 constexpr int TK = 64;                  // contraction depth per stage
-constexpr int ST = 4;                   // TMA ring: activation + codes + scales
 constexpr int WST = 3;                  // dequantised-weight ring
 constexpr int kGroupWarps = 8;          // warps of one dequantisation group
 constexpr int kGroups = 2;              // groups take alternate stages
@@ -52,20 +52,24 @@ constexpr int kDequantWarps = kGroupWarps * kGroups;
 constexpr int kThreads = 32 * (2 + kDequantWarps);
 constexpr int A_BYTES = BM * TK * 2;    // activation tile, 16 KB
 constexpr int P_BYTES = BN / 2 * TK;    // packed codes, 8 KB
-constexpr int SC_BYTES = 2048;          // scale rows of one stage (at most)
 constexpr int W_BYTES = BN * TK * 2;    // dequantised fp16 weights, 32 KB
-constexpr int OFF_A = 0;
-constexpr int OFF_P = OFF_A + ST * A_BYTES;
-constexpr int OFF_W = OFF_P + ST * P_BYTES;
-constexpr int OFF_SC = OFF_W + WST * W_BYTES;
-constexpr int OFF_CTL = OFF_SC + ST * SC_BYTES;
 constexpr int CTL_BYTES = 256;
-constexpr int SMEM_BYTES = OFF_CTL + CTL_BYTES + 1024;
 constexpr int TMEM_COLS = 256;
 
-static_assert(OFF_P % 1024 == 0 && OFF_W % 1024 == 0 && OFF_SC % 1024 == 0, "1024-byte aligned regions");
-static_assert(BM * BN * 4 <= OFF_SC, "split-K staging must fit below the scale buffers");
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+// Shared-memory map for a TMA ring of ST stages whose scale slot holds SCB
+// bytes (the scale rows of one stage: 1 KB for gs >= 32, 2 KB for gs 16).
+template <int ST, int SCB>
+struct Smem {
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_P = OFF_A + ST * A_BYTES;
+  static constexpr int OFF_W = OFF_P + ST * P_BYTES;
+  static constexpr int OFF_SC = OFF_W + WST * W_BYTES;
+  static constexpr int OFF_CTL = OFF_SC + ST * SCB;
+  static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
+  static_assert(OFF_P % 1024 == 0 && OFF_W % 1024 == 0 && OFF_SC % 1024 == 0, "1024-byte aligned regions");
+  static_assert(BM * BN * 4 <= OFF_SC, "split-K staging must fit below the scale buffers");
+  static_assert(BYTES <= 232448, "shared memory per CTA");
+};
 
 struct Args {
   OutSplit out;
@@ -75,9 +79,10 @@ struct Args {
   int sc_bytes;       // bytes of the scale box loaded per stage
 };
 
+constexpr int kMaxST = 5;
 struct SmemCtl {
-  uint64_t full[ST];
-  uint64_t empty[ST];
+  uint64_t full[kMaxST];
+  uint64_t empty[kMaxST];
   uint64_t wready[WST];
   uint64_t wempty[WST];
   uint64_t accfull;
@@ -105,11 +110,14 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
-template <bool BWD>
+template <bool BWD, int ST, int SCB>
 __global__ void __launch_bounds__(kThreads, 1)
 q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
                   const __grid_constant__ CUtensorMap map_sc, const Args args) {
   using namespace sm100;
+  using SM = Smem<ST, SCB>;
+  constexpr int OFF_A = SM::OFF_A, OFF_P = SM::OFF_P, OFF_W = SM::OFF_W, OFF_SC = SM::OFF_SC,
+                OFF_CTL = SM::OFF_CTL, SC_BYTES = SCB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + OFF_CTL);
@@ -163,8 +171,8 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
           tma_load_2d(pk, &map_pk, &ctl->full[s], kc, n0 / 2);
           tma_load_2d(sc, &map_sc, &ctl->full[s], n0, kc >> (__ffs(args.gs) - 1));
         } else {
-          tma_load_2d(pk, &map_pk, &ctl->full[s], n0, kc / 2);
-          tma_load_2d(pk + P_BYTES / 2, &map_pk, &ctl->full[s], n0 + 128, kc / 2);
+#pragma unroll
+          for (int jb = 0; jb < 4; ++jb) tma_load_2d(pk + jb * (P_BYTES / 4), &map_pk, &ctl->full[s], n0 + 64 * jb, kc / 2);
           tma_load_2d(sc, &map_sc, &ctl->full[s], kc, n0 >> (__ffs(args.gs) - 1));
         }
       };
@@ -236,7 +244,7 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       u = td & 1;
     }
     // Per-thread offsets, fixed for the whole contraction: packed-code chunks
-    // (64-byte swizzle forward, 128-byte backward), scale words (the scale
+    // (64-byte swizzle), scale words (the scale
     // row of each 8-column chunk is the same in every stage because stages
     // start on 64-column boundaries), dequantised-tile chunks (128-byte swizzle).
     const int gsl = __ffs(args.gs) - 1;
@@ -251,9 +259,10 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
 #pragma unroll
       for (int i = 0; i < 4; ++i) sc_off[i] = (args.gs < 64 ? ((16 * i + 8 * u) >> gsl) : 0) * 512 + 4 * p;
     } else {
-      const int cc = (j & 1) * 4 + 2 * u;
-      pk_off0 = (j >> 1) * (P_BYTES / 2) + p * 128 + 16 * (cc ^ (p & 7));
-      pk_off1 = (j >> 1) * (P_BYTES / 2) + p * 128 + 16 * ((cc + 1) ^ (p & 7));
+      // block j is its own [32 pairs x 64 B] box with the 64-byte swizzle
+      const int sz = (p >> 1) & 3;
+      pk_off0 = j * (P_BYTES / 4) + p * 64 + 16 * ((2 * u) ^ sz);
+      pk_off1 = j * (P_BYTES / 4) + p * 64 + 16 * ((2 * u + 1) ^ sz);
       const int base = n0 & (args.gs - 1);
 #pragma unroll
       for (int i = 0; i < 4; ++i) sc_off[i] = ((base + 64 * j + 16 * i + 8 * u) >> gsl) * 128 + 4 * p;
@@ -414,15 +423,63 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
   return r == CUDA_SUCCESS;
 }
 
-static int sm_count_gemm() {
-  static int cached = 0;
-  if (!cached) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached = n > 0 ? n : 148;
+template <bool BWD, int ST, int SCB>
+static cudaError_t launch_gemm_variant(const CUtensorMap& map_act, const CUtensorMap& map_pk, const CUtensorMap& map_sc,
+                                       const gemm::Args& a, int tiles_n, int tiles_m, cudaStream_t stream, int* S_out) {
+  using namespace gemm;
+  auto kern = q4gsw_gemm_kernel<BWD, ST, SCB>;
+  constexpr int smem = Smem<ST, SCB>::BYTES;
+  static bool attr_done[64] = {};
+  static int max_clusters[64][9] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int d = (dev >= 0 && dev < 64) ? dev : 0;
+  if (!attr_done[d]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_done[d] = true;
   }
-  return cached;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+
+  // Split-K S: each candidate costs waves(S) * (stages / S + fixed overhead:
+  // 2 stages, or 8 with the cluster reduction), where waves(S) uses how many
+  // S-CTA clusters the device can hold at once (a GPC must host a whole cluster).
+  const int tiles = tiles_n * tiles_m;
+  int best_S = 1;
+  double best_cost = 1e30;
+  for (int S = 1; S <= 8; ++S) {
+    if (S > 1 && a.stages_total / S < 4) break;
+    if (!max_clusters[d][S]) {
+      attr[0].val.clusterDim.z = S;
+      cfg.gridDim = dim3(tiles_n, tiles_m, S);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = -1;
+      max_clusters[d][S] = n;
+    }
+    const int n = max_clusters[d][S];
+    if (n < 1) continue;
+    const double waves = ceil((double)tiles / n);
+    const double cost = waves * ((double)a.stages_total / S + (S > 1 ? 8.0 : 2.0));
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best_S = S;
+    }
+  }
+  attr[0].val.clusterDim.z = best_S;
+  cfg.gridDim = dim3(tiles_n, tiles_m, best_S);
+  *S_out = best_S;
+  return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, a);
 }
 
 template <bool BWD>
@@ -449,12 +506,12 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
     sc_bytes = rows * TK * 2;
     ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, N, M, (uint64_t)N * 2, TK, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, TK / 2,
-                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, TK / 2,
+                     CU_TENSOR_MAP_SWIZZLE_64B) &&
          make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, TK, rows,
                      CU_TENSOR_MAP_SWIZZLE_NONE);
   }
-  if (!ok || sc_bytes > SC_BYTES) return cudaErrorInvalidValue;
+  if (!ok || sc_bytes > 2048) return cudaErrorInvalidValue;
 
   Args a;
   a.sc_bytes = sc_bytes;
@@ -466,40 +523,20 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
   a.out_cols = BWD ? K : N;
   const int contraction = BWD ? N : K;
   a.stages_total = (contraction + TK - 1) / TK;
-
   const int tiles_n = (a.out_cols + BN - 1) / BN;
   const int tiles_m = (M + BM - 1) / BM;
-  const int tiles = tiles_n * tiles_m;
-  int S = 1;
-  while (S < 8 && tiles * (S + 1) <= sm_count_gemm() && a.stages_total / (S + 1) >= 4) ++S;
-
-  auto kern = q4gsw_gemm_kernel<BWD>;
-  static bool attr_done[2][64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_done[BWD][dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_done[BWD][dev] = true;
+  int S = 1, st = 0;
+  cudaError_t e;
+  if (sc_bytes <= 1024) {
+    st = 5;
+    e = launch_gemm_variant<BWD, 5, 1024>(map_act, map_pk, map_sc, a, tiles_n, tiles_m, stream, &S);
+  } else {
+    st = 4;
+    e = launch_gemm_variant<BWD, 4, 2048>(map_act, map_pk, map_sc, a, tiles_n, tiles_m, stream, &S);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(tiles_n, tiles_m, S);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = S;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, a);
   if (route)
     snprintf(route, route_len, "tcgen05_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d",
-             BWD ? "bwd" : "fwd", BM, BN, TK, ST, WST, tiles_n, tiles_m, S);
+             BWD ? "bwd" : "fwd", BM, BN, TK, st, WST, tiles_n, tiles_m, S);
   return e;
 }
 

@@ -43,8 +43,6 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // blocks [u*KB/U, (u+1)*KB/U) of its row tile (KB = K/64, U = 4 S).
 // NT = number of 8-token MMA tiles (1: M <= 8 per slice, 2: M <= 16).
 // SPG = 16-column steps per scale group (1: gs 16, 2: gs 32, 4: gs >= 64).
-constexpr int kFwdPF = 2;   // 64-column blocks per pipeline chunk (two chunks in flight)
-
 template <int NT, int SPG>
 __global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 8 : 5)
 gemv_fwd_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x, OutSplit out, int M, int N,
@@ -80,21 +78,6 @@ gemv_fwd_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[j][c] = part[0][j][c] = part[1][j][c] = 0.f;
 
-  constexpr int PF = kFwdPF;
-  constexpr int NGB = (SPG == 4) ? 1 : 4 / SPG;    // scale groups per block
-  auto load_chunk = [&](int b0, uint4 (&w)[PF], uint32_t (&sc)[PF][NGB]) {
-#pragma unroll
-    for (int q = 0; q < PF; ++q) {
-      const int b = b0 + q;
-      const bool in = b < b_end;
-      w[q] = (in && pvalid) ? ldg_stream_v4(row + 64 * b) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int r = 0; r < NGB; ++r) {
-        const int col = 64 * b + r * (64 / NGB);
-        sc[q][r] = in ? ldg_nc_u32(scales + (size_t)(col >> gsl) * N + 2 * p) : 0u;
-      }
-    }
-  };
   auto flush = [&](uint32_t s_word) {  // scale one finished group into acc
     const __half2 s2 = u32_as_h2(s_word);
     const float se = __low2float(s2), so = __high2float(s2);
@@ -109,56 +92,68 @@ gemv_fwd_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x
     }
   };
 
-  // x fragments of one 64-column block: lane (g, t) feeds token 8j + g with
-  // columns 64b + 16i + 4t .. +3 of step i (two LDG.64 per step, held for the block).
+  // Lanes whose rows or tokens do not exist read valid memory (row 0, token
+  // 0) and their results are never stored, so no load is predicated.  x rows
+  // of this lane: token 8j + g feeds column g of 8-token tile j.
   const __half* xrow[NT];
-  bool xvalid[NT];
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
     const int tok = 8 * j + g;
-    xvalid[j] = tok < Mz;
-    xrow[j] = x + (size_t)(tok0 + (xvalid[j] ? tok : 0)) * K + 4 * t;
+    xrow[j] = x + (size_t)(tok0 + (tok < Mz ? tok : 0)) * K + 4 * t;
   }
-
-  auto compute_chunk = [&](int b0, const uint4 (&w)[PF], const uint32_t (&sc)[PF][NGB]) {
+  constexpr int NGB = (SPG == 4) ? 1 : 4 / SPG;            // scale groups per block
+  const int bpg_mask = (SPG == 4) ? (gs >> 6) - 1 : 0;      // blocks per group - 1 (gs >= 64)
+  const __half* srow = scales + 2 * p;
+  auto load_scales = [&](int b, uint32_t (&sc)[NGB]) {
 #pragma unroll
-    for (int q = 0; q < PF; ++q) {
-      const int b = b0 + q;
-      if (b >= b_end) break;
-      uint2 xv[NT][4];
-#pragma unroll
-      for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) xv[j][i] = xvalid[j] ? ldg_nc_v2(xrow[j] + 64 * b + 16 * i) : make_uint2(0u, 0u);
-      const uint32_t words[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const RowPairs r = codes_minus8_rows(words[i]);
-        const uint32_t a[4] = {h2_as_u32(r.ev01), h2_as_u32(r.od01), h2_as_u32(r.ev23), h2_as_u32(r.od23)};
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          const uint32_t bf[2] = {xv[j][i].x, xv[j][i].y};
-          mma_16816(part[i & 1][j], a, bf);
-        }
-        if (SPG == 1) flush(sc[q][i]);
-        if (SPG == 2 && (i & 1)) flush(sc[q][i >> 1]);
-      }
-      if (SPG == 4 && ((((b + 1) * 64) & (gs - 1)) == 0 || b + 1 == b_end)) flush(sc[q][0]);
-    }
+    for (int r = 0; r < NGB; ++r) sc[r] = ldg_nc_u32(srow + (size_t)((64 * b + r * (64 / NGB)) >> gsl) * N);
   };
 
-  // The packed weight is constant: its first chunk streams in before the
-  // wait for the previous kernel of the stream (which may produce x).
-  uint4 wA[PF], wB[PF];
-  uint32_t sA[PF][NGB], sB[PF][NGB];
-  load_chunk(b_begin, wA, sA);
+  // Two-deep software pipeline over blocks: the weights and scales of blocks
+  // b+1 and b+2 are in flight while block b is dequantised and multiplied.
+  // The packed weight is constant, so the first loads precede the wait for
+  // the previous kernel of the stream (which may produce x).
+  const int b_last = b_end - 1;
+  uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
+  uint32_t s0[NGB], s1[NGB];
+  if (b_begin < b_end) {
+    w0 = ldg_stream_v4(row + 64 * b_begin);
+    w1 = ldg_stream_v4(row + 64 * min(b_begin + 1, b_last));
+    load_scales(b_begin, s0);
+    load_scales(min(b_begin + 1, b_last), s1);
+  }
   griddep_wait();
-  for (int b0 = b_begin; b0 < b_end; b0 += 2 * PF) {
-    load_chunk(b0 + PF, wB, sB);
-    compute_chunk(b0, wA, sA);
-    if (b0 + PF >= b_end) break;
-    load_chunk(b0 + 2 * PF, wA, sA);
-    compute_chunk(b0 + PF, wB, sB);
+  for (int b = b_begin; b < b_end; ++b) {
+    uint2 xv[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[j][i] = ldg_nc_v2(xrow[j] + 64 * b + 16 * i);
+    const uint4 w = w0;
+    uint32_t sc[NGB];
+#pragma unroll
+    for (int r = 0; r < NGB; ++r) sc[r] = s0[r];
+    w0 = w1;
+#pragma unroll
+    for (int r = 0; r < NGB; ++r) s0[r] = s1[r];
+    const int bn = min(b + 2, b_last);
+    w1 = ldg_stream_v4(row + 64 * bn);
+    load_scales(bn, s1);
+
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const RowPairs r = codes_minus8_rows(words[i]);
+      const uint32_t a[4] = {h2_as_u32(r.ev01), h2_as_u32(r.od01), h2_as_u32(r.ev23), h2_as_u32(r.od23)};
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const uint32_t bf[2] = {xv[j][i].x, xv[j][i].y};
+        mma_16816(part[i & 1][j], a, bf);
+      }
+      if (SPG == 1) flush(sc[i]);
+      if (SPG == 2 && (i & 1)) flush(sc[i >> 1]);
+    }
+    if (SPG == 4 && (((b + 1) & bpg_mask) == 0 || b == b_last)) flush(sc[0]);
   }
 
   // D fragment: rows g (even n) and g+8 (odd n), tokens 2t, 2t+1 of tile j.
@@ -242,13 +237,12 @@ __global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __
 #pragma unroll
   for (int q = 0; q < SPB; ++q) grp[q] = (64 * Jc + 16 * (q * (4 / SPB)) + 4 * (g & 3)) >> (__ffs(gs) - 1);
 
-  bool tv[NT];
+  // Rows, blocks and tokens that do not exist are read from valid places
+  // (token 0, block 0, pair pA) and their results are never stored; only the
+  // second pair of a ragged last step (N % 16 == 8) is zeroed explicitly.
   const __half* drow[NT];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    tv[j] = 8 * j + g < Mz;
-    drow[j] = dout + (size_t)(tok0 + (tv[j] ? 8 * j + g : 0)) * N;
-  }
+  for (int j = 0; j < NT; ++j) drow[j] = dout + (size_t)(tok0 + (8 * j + g < Mz ? 8 * j + g : 0)) * N;
   const uint8_t* wcol = packed + 64 * Jc + 16 * (g & 3);
 
   float acc[NT][8][4];
@@ -264,22 +258,24 @@ __global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __
     uint32_t b[NT][2];         // d_out fragments
     uint32_t sa[SPB], sb[SPB]; // scale half2 of pairs pA, pB per group
   };
+  const int s_last = s_end - 1;
   auto load_step = [&](int st, StepData& d) {
     const int pA = st * 8 + t;
-    const bool in = st < s_end;
-    const bool bvalid = in && pA + 4 < NP;
+    const bool bvalid = pA + 4 < NP;
     const int pB = bvalid ? pA + 4 : pA;
-    d.va = (in && jvalid) ? ldg_stream_v4(wcol + (size_t)pA * K) : make_uint4(0, 0, 0, 0);
-    d.vb = (bvalid && jvalid) ? ldg_stream_v4(wcol + (size_t)pB * K) : make_uint4(0, 0, 0, 0);
+    d.va = ldg_stream_v4(wcol + (size_t)pA * K);
+    d.vb = ldg_stream_v4(wcol + (size_t)pB * K);
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-      d.b[j][0] = (in && tv[j]) ? ldg_nc_u32(drow[j] + 2 * pA) : 0u;
-      d.b[j][1] = (bvalid && tv[j]) ? ldg_nc_u32(drow[j] + 2 * pB) : 0u;
+      d.b[j][0] = ldg_nc_u32(drow[j] + 2 * pA);
+      const uint32_t v = ldg_nc_u32(drow[j] + 2 * pB);
+      d.b[j][1] = bvalid ? v : 0u;
     }
 #pragma unroll
     for (int q = 0; q < SPB; ++q) {
-      d.sa[q] = in ? ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pA) : 0u;
-      d.sb[q] = bvalid ? ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pB) : 0u;
+      d.sa[q] = ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pA);
+      const uint32_t v = ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pB);
+      d.sb[q] = bvalid ? v : 0u;
     }
   };
   auto compute_step = [&](const StepData& d) {
@@ -306,14 +302,16 @@ __global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __
   // d_out may come from the previous kernel of the stream: wait before the
   // first load (the step loads mix weights and d_out).
   griddep_wait();
-  StepData dA, dB;
-  load_step(s_begin, dA);
-  for (int st = s_begin; st < s_end; st += 2) {
-    load_step(st + 1, dB);
-    compute_step(dA);
-    if (st + 1 >= s_end) break;
-    load_step(st + 2, dA);
-    compute_step(dB);
+  if (s_begin < s_end) {
+    StepData dA, dB;
+    load_step(s_begin, dA);
+    for (int st = s_begin; st < s_end; st += 2) {
+      load_step(min(st + 1, s_last), dB);
+      compute_step(dA);
+      if (st + 1 >= s_end) break;
+      load_step(min(st + 2, s_last), dA);
+      compute_step(dB);
+    }
   }
 
   // Warp partials -> shared memory: D of MMA q = 2i + h, rows g / g+8 = columns
