@@ -47,8 +47,9 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
             "+ down and up input grads; M=512 tokens, group_size 32")
 
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
-# dram__bytes_write.sum), with the hash of the kernel sources they were taken on.
-NCU_TRAFFIC = {"sources_sha": None, "bytes_per_launch": {}}
+# dram__bytes_write.sum; profiles/gemm_*.md), with the hash of the kernel
+# sources they were taken on: reported only while the sources still match.
+NCU_TRAFFIC = {"sources_sha": "540bb3eaf4e35eb1", "bytes_per_launch": {'up_fwd': 11581440, 'up_bwd': 17862400, 'qkv_fwd': 5671936}}
 
 
 def sources_sha() -> str:
