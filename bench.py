@@ -320,13 +320,22 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """Largest value over all ranks (every rank gets it); the job time of a
+    multi-GPU run is the slowest rank's.  Works on the nccl and gloo backends."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: float, ms_per_step_max: float, unit_scale: float = 1e12) -> float:
+    """Whole-job rate: the units all ranks processed per step over the slowest
+    rank's step time (replicas: every rank does the same step)."""
+    return world * units_per_rank / (ms_per_step_max / 1e3) / unit_scale
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -382,7 +391,7 @@ def run_gpu(args, rank, world, local_rank):
     ms_total = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
-    value = world * flops_step / (ms_step / 1e3) / 1e12
+    value = job_throughput(world, flops_step, ms_step)
     op_ms = {}
     for j, (name, kind, sh) in enumerate(ops):
         op_ms[name] = statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in ev)
@@ -457,7 +466,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize(device)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
-    e2e = {"value": world * flops_step / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+    e2e = {"value": job_throughput(world, flops_step, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
