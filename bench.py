@@ -498,7 +498,8 @@ def run_sweep(args):
     shapes = wl.tiny() + wl.decode() + wl.qkv() + wl.adapter() + wl.sweep()
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     if args.only:
-        shapes = [s for s in shapes if args.only in s.name]
+        import re
+        shapes = [s for s in shapes if re.search(args.only, s.name)]
     for sh in shapes:
         inp = wl.make_inputs(sh)
         codes = torch.from_numpy(inp.codes).to(device)

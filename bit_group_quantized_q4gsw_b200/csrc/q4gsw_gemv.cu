@@ -44,7 +44,7 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // NT = number of 8-token MMA tiles (1: M <= 8 per slice, 2: M <= 16).
 // SPG = 16-column steps per scale group (1: gs 16, 2: gs 32, 4: gs >= 64).
 template <int NT, int SPG>
-__global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 8 : 5)
+__global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 7 : 4)
 gemv_fwd_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x, OutSplit out, int M, int N,
                 int K, int gs) {
   __shared__ float red[kGemvWarps][16][16];  // [warp][token][row]
@@ -104,56 +104,72 @@ gemv_fwd_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x
   constexpr int NGB = (SPG == 4) ? 1 : 4 / SPG;            // scale groups per block
   const int bpg_mask = (SPG == 4) ? (gs >> 6) - 1 : 0;      // blocks per group - 1 (gs >= 64)
   const __half* srow = scales + 2 * p;
-  auto load_scales = [&](int b, uint32_t (&sc)[NGB]) {
-#pragma unroll
-    for (int r = 0; r < NGB; ++r) sc[r] = ldg_nc_u32(srow + (size_t)((64 * b + r * (64 / NGB)) >> gsl) * N);
-  };
 
-  // Two-deep software pipeline over blocks: the weights and scales of blocks
-  // b+1 and b+2 are in flight while block b is dequantised and multiplied.
-  // The packed weight is constant, so the first loads precede the wait for
-  // the previous kernel of the stream (which may produce x).
-  const int b_last = b_end - 1;
-  uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
-  uint32_t s0[NGB], s1[NGB];
-  if (b_begin < b_end) {
-    w0 = ldg_stream_v4(row + 64 * b_begin);
-    w1 = ldg_stream_v4(row + 64 * min(b_begin + 1, b_last));
-    load_scales(b_begin, s0);
-    load_scales(min(b_begin + 1, b_last), s1);
-  }
-  griddep_wait();
-  for (int b = b_begin; b < b_end; ++b) {
+  // One 64-column block of this lane: packed word quad, scale words, x fragments.
+  struct Blk {
+    uint4 w;
+    uint32_t s[NGB];
     uint2 xv[NT][4];
+  };
+  const int b_last = b_end - 1;
+  auto load_w = [&](int b, Blk& d) {
+    b = min(b, b_last);
+    d.w = ldg_stream_v4(row + 64 * b);
+#pragma unroll
+    for (int r = 0; r < NGB; ++r) d.s[r] = ldg_nc_u32(srow + (size_t)((64 * b + r * (64 / NGB)) >> gsl) * N);
+  };
+  auto load_x = [&](int b, Blk& d) {
+    b = min(b, b_last);
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xv[j][i] = ldg_nc_v2(xrow[j] + 64 * b + 16 * i);
-    const uint4 w = w0;
-    uint32_t sc[NGB];
-#pragma unroll
-    for (int r = 0; r < NGB; ++r) sc[r] = s0[r];
-    w0 = w1;
-#pragma unroll
-    for (int r = 0; r < NGB; ++r) s0[r] = s1[r];
-    const int bn = min(b + 2, b_last);
-    w1 = ldg_stream_v4(row + 64 * bn);
-    load_scales(bn, s1);
-
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+      for (int i = 0; i < 4; ++i) d.xv[j][i] = ldg_nc_v2(xrow[j] + 64 * b + 16 * i);
+  };
+  auto compute = [&](int b, const Blk& d) {
+    const uint32_t words[4] = {d.w.x, d.w.y, d.w.z, d.w.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const RowPairs r = codes_minus8_rows(words[i]);
       const uint32_t a[4] = {h2_as_u32(r.ev01), h2_as_u32(r.od01), h2_as_u32(r.ev23), h2_as_u32(r.od23)};
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
-        const uint32_t bf[2] = {xv[j][i].x, xv[j][i].y};
+        const uint32_t bf[2] = {d.xv[j][i].x, d.xv[j][i].y};
         mma_16816(part[i & 1][j], a, bf);
       }
-      if (SPG == 1) flush(sc[i]);
-      if (SPG == 2 && (i & 1)) flush(sc[i >> 1]);
+      if (SPG == 1) flush(d.s[i]);
+      if (SPG == 2 && (i & 1)) flush(d.s[i >> 1]);
     }
-    if (SPG == 4 && (((b + 1) & bpg_mask) == 0 || b == b_last)) flush(sc[0]);
+    if (SPG == 4 && (((b + 1) & bpg_mask) == 0 || b == b_last)) flush(d.s[0]);
+  };
+
+  // Three blocks rotate through three register sets (no copies): while one
+  // block is dequantised and multiplied, the next two are in flight.  The
+  // packed weight is constant, so its first loads precede the wait for the
+  // previous kernel of the stream (which may produce x).
+  if (b_begin < b_end) {
+    Blk A, B, C;
+    load_w(b_begin, A);
+    load_w(b_begin + 1, B);
+    load_w(b_begin + 2, C);
+    griddep_wait();
+    load_x(b_begin, A);
+    load_x(b_begin + 1, B);
+    load_x(b_begin + 2, C);
+    for (int b = b_begin; b < b_end; b += 3) {
+      compute(b, A);
+      if (b + 1 >= b_end) break;
+      load_w(b + 3, A);
+      load_x(b + 3, A);
+      compute(b + 1, B);
+      if (b + 2 >= b_end) break;
+      load_w(b + 4, B);
+      load_x(b + 4, B);
+      compute(b + 2, C);
+      load_w(b + 5, C);
+      load_x(b + 5, C);
+    }
+  } else {
+    griddep_wait();
   }
 
   // D fragment: rows g (even n) and g+8 (odd n), tokens 2t, 2t+1 of tile j.
@@ -372,15 +388,16 @@ static int sm_count() {
   return cached;
 }
 
-// Contraction splits S (the cluster size).  Measured on B200 for the decode,
-// MLP and 8B-layer shapes: the forward wants about four CTAs per SM in
-// flight and as little splitting as that allows; the input gradient, whose
-// output tile is narrow, wants about 320 CTAs.  At least `min_units`
-// contraction units stay with each warp.
-static int fwd_splits(long long tiles, int blocks_per_tile) {
-  int S = (int)lround(4.0 * sm_count() / (double)tiles);
+// Contraction splits S (the cluster size), from measurements on B200 over the
+// decode, MLP and 8B-layer shapes: the forward wants about six CTAs per SM and
+// no split that leaves a large weight's warps with fewer than 8 blocks; the
+// input gradient, whose output tile is narrow, wants about 320 CTAs.
+static int fwd_splits(long long tiles, int blocks_per_tile, size_t weight_bytes) {
+  int S = (int)lround(6.0 * sm_count() / (double)tiles);
   S = S < 1 ? 1 : S > 8 ? 8 : S;
-  while (S > 1 && blocks_per_tile / (kGemvWarps * S) < 1) --S;
+  // a large weight keeps at least 8 blocks (a few pipeline turns) per warp
+  const int min_blocks = weight_bytes >= ((size_t)16 << 20) ? 8 : 1;
+  while (S > 1 && blocks_per_tile / (kGemvWarps * S) < min_blocks) --S;
   return S;
 }
 
@@ -427,7 +444,7 @@ cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint
   int S = 1;
 #define Q4_FWD(NT_, SPG_)                                                                                       \
   do {                                                                                                          \
-    S = fwd_splits((long long)tiles * zs, K / 64);                                                             \
+    S = fwd_splits((long long)tiles * zs, K / 64, (size_t)N * K / 2);                                        \
     err = launch_cluster(gemv_fwd_kernel<NT_, SPG_>, dim3(tiles, S, zs), kGemvThreads, S, 0, stream, pk, xh, out, \
                          M, N, K, gs);                                                                          \
   } while (0)
