@@ -8,15 +8,19 @@
 // Replace broad QKV fusion with BK64 kernel" is the forward with its output
 // columns scattered over three buffers.)
 //
-// One CTA computes a 128-token x 256-feature tile of the output, optionally for
-// one slice of the contraction (split-K, reduced in a cluster through
-// distributed shared memory).  Warp roles:
+// One CTA computes a (128 or 256)-token x 256-feature tile of the output,
+// optionally for one slice of the contraction (split-K, reduced in a cluster
+// through distributed shared memory).  Warp roles:
 //   warp 0       TMA producer: activation tile (fp16, 128-byte swizzle) and the
 //                packed-code tile of each 64-deep contraction stage;
-//   warp 1       allocates tensor memory and issues tcgen05.mma from one thread;
-//   warps 2..9   dequantise the stage's codes into fp16 (code - 8) * scale,
+//   warp 1       allocates tensor memory and issues tcgen05.mma from one thread
+//                (one 128-token accumulator per 128 tokens of the tile);
+//   warps 2..17  dequantise every stage's codes into fp16 (code - 8) * scale,
 //                written straight into the 128-byte-swizzled layout the MMA
 //                descriptors read, then run the epilogue (tcgen05.ld -> global).
+// Every consumer waits on every phase of the barriers it uses: a waiter that
+// skipped a phase could mistake an older completion of the same parity for
+// the one it wants.
 // The forward reads the weight tile [256 n][64 k] as a K-major B operand; the
 // backward writes the same kind of tile ([64 n][256 k], k contiguous) and reads
 // it as an MN-major B operand, so both directions use one packed blob and one
@@ -28,6 +32,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 
 #include "q4gsw_common.cuh"
 #include "q4gsw_internal.h"
@@ -42,32 +47,34 @@ __device__ unsigned int g_device_error = 0;
 
 namespace gemm {
 
-constexpr int BM = 128;                 // tokens per tile (MMA M)
+constexpr int BM = 128;                 // tokens per MMA (M) and per accumulator
 constexpr int BN = 256;                 // output features per tile (MMA N)
 constexpr int TK = 64;                  // contraction depth per stage
 constexpr int WST = 3;                  // dequantised-weight ring
-constexpr int kGroupWarps = 8;          // warps of one dequantisation group
-constexpr int kGroups = 2;              // groups take alternate stages
-constexpr int kDequantWarps = kGroupWarps * kGroups;
+constexpr int kDequantWarps = 16;       // all of them dequantise every stage
 constexpr int kThreads = 32 * (2 + kDequantWarps);
 constexpr int A_BYTES = BM * TK * 2;    // activation tile, 16 KB
 constexpr int P_BYTES = BN / 2 * TK;    // packed codes, 8 KB
 constexpr int W_BYTES = BN * TK * 2;    // dequantised fp16 weights, 32 KB
 constexpr int CTL_BYTES = 256;
-constexpr int TMEM_COLS = 256;
 
-// Shared-memory map for a TMA ring of ST stages whose scale slot holds SCB
-// bytes (the scale rows of one stage: 1 KB for gs >= 32, 2 KB for gs 16).
-template <int ST, int SCB>
+// Shared-memory map for a TMA ring of ST stages (MSUB 128-row activation
+// tiles, packed codes, a scale slot of SCB bytes: 1 KB for gs >= 32, 2 KB for
+// gs 16) and a ring of WST dequantised-weight tiles.  One CTA computes MSUB
+// 128-token sub-tiles against each dequantised weight tile, so the
+// dequantisation work per multiply-add falls by MSUB.
+template <int ST, int SCB, int MSUB>
 struct Smem {
+  static constexpr int A_STAGE = MSUB * A_BYTES;
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_P = OFF_A + ST * A_BYTES;
+  static constexpr int OFF_P = OFF_A + ST * A_STAGE;
   static constexpr int OFF_W = OFF_P + ST * P_BYTES;
   static constexpr int OFF_SC = OFF_W + WST * W_BYTES;
   static constexpr int OFF_CTL = OFF_SC + ST * SCB;
   static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
+  static constexpr int TMEM_COLS = 256 * MSUB;
   static_assert(OFF_P % 1024 == 0 && OFF_W % 1024 == 0 && OFF_SC % 1024 == 0, "1024-byte aligned regions");
-  static_assert(BM * BN * 4 <= OFF_SC, "split-K staging must fit below the scale buffers");
+  static_assert(BM * BN * 4 <= OFF_SC, "split-K staging of one sub-tile must fit below the scale buffers");
   static_assert(BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -97,10 +104,9 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
-               : "memory");
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
   return v;
 }
 
@@ -110,14 +116,15 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
-template <bool BWD, int ST, int SCB>
+template <bool BWD, int ST, int SCB, int MSUB>
 __global__ void __launch_bounds__(kThreads, 1)
 q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
                   const __grid_constant__ CUtensorMap map_sc, const Args args) {
   using namespace sm100;
-  using SM = Smem<ST, SCB>;
+  using SM = Smem<ST, SCB, MSUB>;
   constexpr int OFF_A = SM::OFF_A, OFF_P = SM::OFF_P, OFF_W = SM::OFF_W, OFF_SC = SM::OFF_SC,
-                OFF_CTL = SM::OFF_CTL, SC_BYTES = SCB;
+                OFF_CTL = SM::OFF_CTL, SC_BYTES = SCB, A_STAGE = SM::A_STAGE,
+                TMEM_COLS = SM::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + OFF_CTL);
@@ -126,7 +133,7 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN;    // first output feature of the tile
-  const int m0 = blockIdx.y * BM;    // first token of the tile
+  const int m0 = blockIdx.y * BM * MSUB;    // first token of the tile
   const int S = gridDim.z, split = blockIdx.z;
   const int st_begin = (int)((long long)split * args.stages_total / S);
   const int st_end = (int)((long long)(split + 1) * args.stages_total / S);
@@ -139,7 +146,7 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       mbar_init(&ctl->empty[i], 1);
     }
     for (int i = 0; i < WST; ++i) {
-      mbar_init(&ctl->wready[i], kGroupWarps);
+      mbar_init(&ctl->wready[i], kDequantWarps);
       mbar_init(&ctl->wempty[i], 1);
     }
     mbar_init(&ctl->accfull, 1);
@@ -178,14 +185,14 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       };
       auto load_act = [&](int it) {
         const int s = it % ST;
-        tma_load_2d(smem + OFF_A + s * A_BYTES, &map_act, &ctl->full[s], (st_begin + it) * TK, m0);
+        tma_load_2d(smem + OFF_A + s * A_STAGE, &map_act, &ctl->full[s], (st_begin + it) * TK, m0);
       };
       // The packed weight is constant: the first stages' codes and scales are
       // requested before waiting for the previous kernel of the stream, which
       // may still be producing the activations.
       const int pre = nit < ST ? nit : ST;
       for (int it = 0; it < pre; ++it) {
-        mbar_arrive_expect_tx(&ctl->full[it], A_BYTES + P_BYTES + args.sc_bytes);
+        mbar_arrive_expect_tx(&ctl->full[it], A_STAGE + P_BYTES + args.sc_bytes);
         load_weights(it);
       }
       griddep_wait();
@@ -194,7 +201,7 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       for (int it = pre; it < nit; ++it) {
         const int s = it % ST;
         if (!mbar_wait(&ctl->empty[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
-        mbar_arrive_expect_tx(&ctl->full[s], A_BYTES + P_BYTES + args.sc_bytes);
+        mbar_arrive_expect_tx(&ctl->full[s], A_STAGE + P_BYTES + args.sc_bytes);
         load_weights(it);
         load_act(it);
         issued = it + 1;
@@ -212,13 +219,16 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
         if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 2u)) break;
         if (!mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
         tc_fence_after();
-        const uint32_t a0 = sbase + OFF_A + s * A_BYTES, w0 = sbase + OFF_W + w * W_BYTES;
+        const uint32_t a0 = sbase + OFF_A + s * A_STAGE, w0 = sbase + OFF_W + w * W_BYTES;
 #pragma unroll
         for (int ks = 0; ks < TK / 16; ++ks) {
-          const uint64_t ad = smem_desc_sw128(a0 + 32 * ks, 16, 1024);
           const uint64_t bd = BWD ? smem_desc_sw128(w0 + ks * 2048, 8192, 1024)
                                   : smem_desc_sw128(w0 + 32 * ks, 16, 1024);
-          mma_f16_ss(tmem, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+          for (int ms = 0; ms < MSUB; ++ms) {
+            const uint64_t ad = smem_desc_sw128(a0 + ms * A_BYTES + 32 * ks, 16, 1024);
+            mma_f16_ss(tmem + ms * 256, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+          }
         }
         mma_commit(&ctl->empty[s]);
         mma_commit(&ctl->wempty[w]);
@@ -229,78 +239,66 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
     }
   } else {
     // ------------------------------------------------------------ dequantisation
-    // Group grp takes the iterations it == grp (mod 2); inside a group, thread
-    // td owns pair row p and half u of each 64-column block (backward: also
-    // the 64-column block j of the 256-column tile).
-    const int grp = (warp - 2) / kGroupWarps;
-    const int td = threadIdx.x - 64 - grp * 32 * kGroupWarps;
-    int p, u, j = 0;
-    if (!BWD) {
-      p = td >> 1;
-      u = td & 1;
-    } else {
-      j = td >> 6;
-      p = (td & 63) >> 1;
-      u = td & 1;
-    }
-    // Per-thread offsets, fixed for the whole contraction: packed-code chunks
-    // (64-byte swizzle), scale words (the scale
-    // row of each 8-column chunk is the same in every stage because stages
-    // start on 64-column boundaries), dequantised-tile chunks (128-byte swizzle).
+    // Thread td owns pair row p (rows 2p, 2p+1 of the tile), half u of each
+    // 16-column step and the steps i = 2h, 2h+1 of each 64-column block; in the
+    // backward also the 64-column block j of the 256-column tile.  Lanes vary
+    // (u, h) fastest so that the 8-byte code loads of a half-warp and the
+    // 16-byte stores of a quarter-warp hit distinct banks.
+    const int td = threadIdx.x - 64;
+    const int u = td & 1, h = (td >> 1) & 1;
+    const int p = BWD ? ((td >> 2) & 31) : (td >> 2);
+    const int j = BWD ? (td >> 7) : 0;
+    // Per-thread offsets, fixed for the whole contraction: packed-code words
+    // (64-byte swizzle), scale words (the scale row of each 8-column chunk is
+    // the same in every stage because stages start on 64-column boundaries),
+    // dequantised-tile chunks (128-byte swizzle).
     const int gsl = __ffs(args.gs) - 1;
-    uint32_t pk_off0, pk_off1, sc_off[4];
-    if (!BWD) {
-      const int sz = (p >> 1) & 3;
-      pk_off0 = p * 64 + 16 * ((2 * u) ^ sz);
-      pk_off1 = p * 64 + 16 * ((2 * u + 1) ^ sz);
-      // stage base column kc: with gs >= 64 the 64 columns sit in one group,
-      // with gs < 64 the stage starts a group; either way the row is
-      // ((kc mod gs) + 16 i + 8 u) >> gsl = (16 i + 8 u) >> gsl for gs < 64, else 0
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sc_off[i] = (args.gs < 64 ? ((16 * i + 8 * u) >> gsl) : 0) * 512 + 4 * p;
-    } else {
-      // block j is its own [32 pairs x 64 B] box with the 64-byte swizzle
-      const int sz = (p >> 1) & 3;
-      pk_off0 = j * (P_BYTES / 4) + p * 64 + 16 * ((2 * u) ^ sz);
-      pk_off1 = j * (P_BYTES / 4) + p * 64 + 16 * ((2 * u + 1) ^ sz);
-      const int base = n0 & (args.gs - 1);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sc_off[i] = ((base + 64 * j + 16 * i + 8 * u) >> gsl) * 128 + 4 * p;
-    }
+    const int sz = (p >> 1) & 3;
+    const uint32_t pk_base = (BWD ? j * (P_BYTES / 4) : 0) + p * 64 + 8 * h;
+    const uint32_t pk_off0 = pk_base + 16 * ((2 * u) ^ sz);       // columns +0..3 of each step
+    const uint32_t pk_off1 = pk_base + 16 * ((2 * u + 1) ^ sz);   // columns +4..7
+    uint32_t sc_off[2], st_off_e[2], st_off_o[2];
     const int re = 2 * p, ro = 2 * p + 1;
-    uint32_t st_off_e[4], st_off_o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int ii = 0; ii < 2; ++ii) {
+      const int i = 2 * h + ii;
+      if (!BWD) {
+        // stage base column kc: with gs >= 64 the 64 columns sit in one group,
+        // with gs < 64 the stage starts a group; either way the row is
+        // ((kc mod gs) + 16 i + 8 u) >> gsl = (16 i + 8 u) >> gsl for gs < 64, else 0
+        sc_off[ii] = (args.gs < 64 ? ((16 * i + 8 * u) >> gsl) : 0) * 512 + 4 * p;
+      } else {
+        sc_off[ii] = (((n0 & (args.gs - 1)) + 64 * j + 16 * i + 8 * u) >> gsl) * 128 + 4 * p;
+      }
       const int chunk = 2 * i + u;
-      st_off_e[i] = (BWD ? j * 8192 : 0) + re * 128 + 16 * (chunk ^ (re & 7));
-      st_off_o[i] = (BWD ? j * 8192 : 0) + ro * 128 + 16 * (chunk ^ (ro & 7));
+      st_off_e[ii] = (BWD ? j * 8192 : 0) + re * 128 + 16 * (chunk ^ (re & 7));
+      st_off_o[ii] = (BWD ? j * 8192 : 0) + ro * 128 + 16 * (chunk ^ (ro & 7));
     }
-    for (int it = grp; it < nit; it += kGroups) {
+    for (int it = 0; it < nit; ++it) {
       const int s = it % ST, w = it % WST;
       if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
       if (it >= WST && !mbar_wait(&ctl->wempty[w], ((it / WST) - 1) & 1, abort_flag, &g_device_error, 32u)) break;
       const uint32_t pk = sbase + OFF_P + s * P_BYTES;
       const uint32_t sc = sbase + OFF_SC + s * SC_BYTES;
-      const uint4 c0 = lds128(pk + pk_off0);
-      const uint4 c1 = lds128(pk + pk_off1);
-      uint32_t sw[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sw[i] = lds32(sc + sc_off[i]);
-      const uint32_t wlo[4] = {c0.x, c0.y, c0.z, c0.w};
-      const uint32_t whi[4] = {c1.x, c1.y, c1.z, c1.w};
+      const uint2 c0 = lds64(pk + pk_off0);
+      const uint2 c1 = lds64(pk + pk_off1);
+      const uint32_t sw0 = lds32(sc + sc_off[0]), sw1 = lds32(sc + sc_off[1]);
+      const uint32_t wlo[2] = {c0.x, c0.y};
+      const uint32_t whi[2] = {c1.x, c1.y};
+      const uint32_t sw[2] = {sw0, sw1};
       const uint32_t wt = sbase + OFF_W + w * W_BYTES;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const RowPairs a = codes_minus8_rows(wlo[i]);   // columns +0..3 of this 8-column chunk
-        const RowPairs b = codes_minus8_rows(whi[i]);   // columns +4..7
-        const __half2 s2 = u32_as_h2(sw[i]);
+      for (int ii = 0; ii < 2; ++ii) {
+        const RowPairs a = codes_minus8_rows(wlo[ii]);   // columns +0..3 of this 8-column chunk
+        const RowPairs b = codes_minus8_rows(whi[ii]);   // columns +4..7
+        const __half2 s2 = u32_as_h2(sw[ii]);
         const __half2 se = __low2half2(s2), so = __high2half2(s2);
         const uint4 ve = make_uint4(h2_as_u32(__hmul2(a.ev01, se)), h2_as_u32(__hmul2(a.ev23, se)),
                                     h2_as_u32(__hmul2(b.ev01, se)), h2_as_u32(__hmul2(b.ev23, se)));
         const uint4 vo = make_uint4(h2_as_u32(__hmul2(a.od01, so)), h2_as_u32(__hmul2(a.od23, so)),
                                     h2_as_u32(__hmul2(b.od01, so)), h2_as_u32(__hmul2(b.od23, so)));
-        sts128(wt + st_off_e[i], ve);
-        sts128(wt + st_off_o[i], vo);
+        sts128(wt + st_off_e[ii], ve);
+        sts128(wt + st_off_o[ii], vo);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -310,79 +308,81 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
 
   // ---------------------------------------------------------------- epilogue
   // Warps 2..17: warp w reads TMEM lanes 32 (w % 4) .. +31 (tokens) and the 64
-  // accumulator columns [64 h, 64 h + 64) with h = (w - 2) / 4.
+  // accumulator columns [64 h, 64 h + 64) with h = (w - 2) / 4, for each of
+  // the MSUB accumulators (sub-tile ms holds tokens m0 + 128 ms ..).
   const bool epi = warp >= 2;
   float* stage_f32 = reinterpret_cast<float*>(smem);   // split-K staging [128][256], 16-byte chunks swizzled
   griddep_wait();   // outputs may still be read by the previous kernel of the stream
   bool have_acc = false;
   if (epi) have_acc = mbar_wait(&ctl->accfull, 0, abort_flag, &g_device_error, 16u);
-  if (epi && have_acc) {
-    tc_fence_after();
-    const int q = warp & 3, h = (warp - 2) >> 2;
-    const int row = 32 * q + lane;
-    const int m = m0 + row;
+  if (epi && have_acc) tc_fence_after();
+  auto store4 = [&](int m, int n, float4 val) {
+    const OutSplit& o = args.out;
+    float* dst;
+    if (n < o.n1) dst = o.y0 + (size_t)m * o.n1 + n;
+    else if (n < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (n - o.n1);
+    else dst = o.y2 + (size_t)m * (o.N - o.n2) + (n - o.n2);
+    *reinterpret_cast<float4*>(dst) = val;
+  };
 #pragma unroll 1
-    for (int c32 = 0; c32 < 2; ++c32) {
-      const int col = 64 * h + 32 * c32;
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, r);
-      tmem_wait_ld();
-      if (S == 1) {
-        if (m < args.M) {
+  for (int ms = 0; ms < MSUB; ++ms) {
+    const int mb = m0 + ms * BM;
+    if (epi && have_acc) {
+      const int q = warp & 3, h = (warp - 2) >> 2;
+      const int row = 32 * q + lane;
+      const int m = mb + row;
+#pragma unroll 1
+      for (int c32 = 0; c32 < 2; ++c32) {
+        const int col = 64 * h + 32 * c32;
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ms * 256 + col), r);
+        tmem_wait_ld();
+        if (S == 1) {
+          if (m < args.M) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const int n = n0 + col + 4 * v;
+              if (n >= args.out_cols) break;
+              store4(m, n, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                       __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+            }
+          }
+        } else {
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            const int n = n0 + col + 4 * v;
-            if (n >= args.out_cols) break;
+            const int chunk = (col >> 2) + v;   // 16-byte chunk of the 1 KB row
             const float4 val = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                            __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-            const OutSplit& o = args.out;
-            float* dst;
-            if (n < o.n1) dst = o.y0 + (size_t)m * o.n1 + n;
-            else if (n < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (n - o.n1);
-            else dst = o.y2 + (size_t)m * (o.N - o.n2) + (n - o.n2);
-            *reinterpret_cast<float4*>(dst) = val;
+            *reinterpret_cast<float4*>(stage_f32 + row * 256 + 4 * (chunk ^ (row & 7))) = val;
           }
         }
-      } else {
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const int chunk = (col >> 2) + v;   // 16-byte chunk of the 1 KB row
-          const float4 val = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-          *reinterpret_cast<float4*>(stage_f32 + row * 256 + 4 * (chunk ^ (row & 7))) = val;
-        }
       }
     }
-  }
-  if (S > 1) {
-    // every thread of every CTA of the cluster passes both barriers, aborted or not
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    const int r = (int)cluster.block_rank();
-    const int row_b = r * BM / S, row_e = (r + 1) * BM / S;
-    if (!*abort_flag) {
-      for (int idx = threadIdx.x; idx < (row_e - row_b) * 64; idx += kThreads) {
-        const int row = row_b + (idx >> 6), chunk = idx & 63;
-        const int m = m0 + row, n = n0 + 4 * chunk;
-        if (m >= args.M || n >= args.out_cols) continue;
-        const int off = row * 256 + 4 * (chunk ^ (row & 7));
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int qq = 0; qq < S; ++qq) {
-          const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + off);
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
+    if (S > 1) {
+      // every thread of every CTA of the cluster passes both barriers, aborted or not
+      cg::cluster_group cluster = cg::this_cluster();
+      cluster.sync();
+      const int r = (int)cluster.block_rank();
+      const int row_b = r * BM / S, row_e = (r + 1) * BM / S;
+      if (!*abort_flag) {
+        for (int idx = threadIdx.x; idx < (row_e - row_b) * 64; idx += kThreads) {
+          const int row = row_b + (idx >> 6), chunk = idx & 63;
+          const int m = mb + row, n = n0 + 4 * chunk;
+          if (m >= args.M || n >= args.out_cols) continue;
+          const int off = row * 256 + 4 * (chunk ^ (row & 7));
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int qq = 0; qq < S; ++qq) {
+            const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + off);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+          }
+          store4(m, n, acc);
         }
-        const OutSplit& o = args.out;
-        float* dst;
-        if (n < o.n1) dst = o.y0 + (size_t)m * o.n1 + n;
-        else if (n < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (n - o.n1);
-        else dst = o.y2 + (size_t)m * (o.N - o.n2) + (n - o.n2);
-        *reinterpret_cast<float4*>(dst) = acc;
       }
+      cluster.sync();
     }
-    cluster.sync();
   }
   tc_fence_before();
   __syncthreads();
@@ -423,12 +423,24 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
   return r == CUDA_SUCCESS;
 }
 
-template <bool BWD, int ST, int SCB>
-static cudaError_t launch_gemm_variant(const CUtensorMap& map_act, const CUtensorMap& map_pk, const CUtensorMap& map_sc,
-                                       const gemm::Args& a, int tiles_n, int tiles_m, cudaStream_t stream, int* S_out) {
+// Relative main-loop time of one 64-column stage: one 128-token accumulator
+// (1.0), or two sharing the dequantised tile (less than twice: the weight
+// tile's dequantisation, its shared-memory stores and the packed-code copy are
+// paid once).
+static double stage_time(int msub) { return msub == 2 ? 1.6 : 1.0; }
+
+// Chooses the split-K factor S of one kernel variant (and its cost), and
+// launches it when `launch` is set.  Each candidate S costs waves(S) *
+// (stages / S * stage time + fixed overhead: 2 stage times per accumulator, or
+// 8 with the cluster reduction), where waves(S) uses how many S-CTA clusters
+// the device can hold at once (a GPC must host a whole cluster).
+template <bool BWD, int ST, int SCB, int MSUB>
+static cudaError_t gemm_variant(const CUtensorMap& map_act, const CUtensorMap& map_pk, const CUtensorMap& map_sc,
+                                const gemm::Args& a, int tiles_n, cudaStream_t stream, bool launch, int* S_out,
+                                double* cost_out) {
   using namespace gemm;
-  auto kern = q4gsw_gemm_kernel<BWD, ST, SCB>;
-  constexpr int smem = Smem<ST, SCB>::BYTES;
+  auto kern = q4gsw_gemm_kernel<BWD, ST, SCB, MSUB>;
+  constexpr int smem = Smem<ST, SCB, MSUB>::BYTES;
   static bool attr_done[64] = {};
   static int max_clusters[64][9] = {};
   int dev = 0;
@@ -439,6 +451,7 @@ static cudaError_t launch_gemm_variant(const CUtensorMap& map_act, const CUtenso
     if (e != cudaSuccess) return e;
     attr_done[d] = true;
   }
+  const int tiles_m = (a.M + BM * MSUB - 1) / (BM * MSUB);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
@@ -452,10 +465,8 @@ static cudaError_t launch_gemm_variant(const CUtensorMap& map_act, const CUtenso
   cfg.attrs = attr;
   cfg.numAttrs = 2;
 
-  // Split-K S: each candidate costs waves(S) * (stages / S + fixed overhead:
-  // 2 stages, or 8 with the cluster reduction), where waves(S) uses how many
-  // S-CTA clusters the device can hold at once (a GPC must host a whole cluster).
   const int tiles = tiles_n * tiles_m;
+  const double t = stage_time(MSUB);
   int best_S = 1;
   double best_cost = 1e30;
   for (int S = 1; S <= 8; ++S) {
@@ -470,16 +481,25 @@ static cudaError_t launch_gemm_variant(const CUtensorMap& map_act, const CUtenso
     const int n = max_clusters[d][S];
     if (n < 1) continue;
     const double waves = ceil((double)tiles / n);
-    const double cost = waves * ((double)a.stages_total / S + (S > 1 ? 8.0 : 2.0));
+    const double cost = waves * ((double)a.stages_total / S * t + (S > 1 ? 8.0 : 2.0) * MSUB);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best_S = S;
     }
   }
+  *S_out = best_S;
+  *cost_out = best_cost;
+  if (!launch) return cudaSuccess;
   attr[0].val.clusterDim.z = best_S;
   cfg.gridDim = dim3(tiles_n, tiles_m, best_S);
-  *S_out = best_S;
   return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, a);
+}
+
+// Q4GSW_GEMM_MSUB=1 or 2 pins the number of 128-token accumulators per CTA
+// (for tuning and tests); unset or 0 lets the cost model choose.
+static int forced_msub() {
+  const char* e = getenv("Q4GSW_GEMM_MSUB");
+  return (e && (e[0] == '1' || e[0] == '2') && e[1] == 0) ? e[0] - '0' : 0;
 }
 
 template <bool BWD>
@@ -487,7 +507,7 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
                                     OutSplit out, cudaStream_t stream, char* route, int route_len) {
   using namespace gemm;
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
-  CUtensorMap map_act, map_pk, map_sc;
+  CUtensorMap map_pk, map_sc;
   const Layout L = layout_of(N, K, gs);
   const void* scales = pk + L.scales_offset;
   const int G = K / gs;
@@ -496,17 +516,13 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
   if (!BWD) {
     const int rows = TK / gs > 1 ? TK / gs : 1;   // scale groups of one 64-column stage
     sc_bytes = rows * BN * 2;
-    ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, K, M, (uint64_t)K * 2, TK, BM,
-                     CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BN / 2, CU_TENSOR_MAP_SWIZZLE_64B) &&
+    ok = make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BN / 2, CU_TENSOR_MAP_SWIZZLE_64B) &&
          make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, BN, rows,
                      CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
     const int rows = BN / gs > 1 ? BN / gs : 1;   // scale groups of one 256-column tile
     sc_bytes = rows * TK * 2;
-    ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, N, M, (uint64_t)N * 2, TK, BM,
-                     CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, TK / 2,
+    ok = make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, TK / 2,
                      CU_TENSOR_MAP_SWIZZLE_64B) &&
          make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, TK, rows,
                      CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -524,19 +540,36 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
   const int contraction = BWD ? N : K;
   a.stages_total = (contraction + TK - 1) / TK;
   const int tiles_n = (a.out_cols + BN - 1) / BN;
-  const int tiles_m = (M + BM - 1) / BM;
-  int S = 1, st = 0;
-  cudaError_t e;
-  if (sc_bytes <= 1024) {
-    st = 5;
-    e = launch_gemm_variant<BWD, 5, 1024>(map_act, map_pk, map_sc, a, tiles_n, tiles_m, stream, &S);
-  } else {
-    st = 4;
-    e = launch_gemm_variant<BWD, 4, 2048>(map_act, map_pk, map_sc, a, tiles_n, tiles_m, stream, &S);
+  // The activation box is re-encoded per variant (128 or 256 tokens high).
+  auto run = [&](int msub, bool launch, int* S, double* cost) -> cudaError_t {
+    CUtensorMap map_a;
+    const uint64_t act_cols = BWD ? (uint64_t)N : (uint64_t)K;
+    if (!make_map_2d(&map_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, act_cols, M, act_cols * 2, TK, BM * msub,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    if (sc_bytes <= 1024)
+      return msub == 2 ? gemm_variant<BWD, 3, 1024, 2>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost)
+                       : gemm_variant<BWD, 5, 1024, 1>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost);
+    return msub == 2 ? gemm_variant<BWD, 3, 2048, 2>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost)
+                     : gemm_variant<BWD, 4, 2048, 1>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost);
+  };
+  int msub = forced_msub();
+  int S = 1;
+  double cost = 0;
+  cudaError_t e = cudaSuccess;
+  if (msub == 0) {
+    int S1 = 1, S2 = 1;
+    double c1 = 0, c2 = 0;
+    e = run(1, false, &S1, &c1);
+    if (e == cudaSuccess) e = run(2, false, &S2, &c2);
+    if (e != cudaSuccess) return e;
+    msub = (M > BM && c2 < c1) ? 2 : 1;
   }
+  e = run(msub, true, &S, &cost);
+  const int st = msub == 2 ? 3 : (sc_bytes <= 1024 ? 5 : 4);
   if (route)
     snprintf(route, route_len, "tcgen05_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d",
-             BWD ? "bwd" : "fwd", BM, BN, TK, st, WST, tiles_n, tiles_m, S);
+             BWD ? "bwd" : "fwd", BM * msub, BN, TK, st, WST, tiles_n, (M + BM * msub - 1) / (BM * msub), S);
   return e;
 }
 

@@ -222,18 +222,35 @@ def test_non_default_stream():
 
 
 # ----------------------------------------------------------------------------- tcgen05 GEMM route
+@pytest.fixture(params=[1, 2], ids=["msub1", "msub2"])
+def msub(request, monkeypatch):
+    """Pins the GEMM variant: one or two 128-token accumulators per CTA."""
+    monkeypatch.setenv("Q4GSW_GEMM_MSUB", str(request.param))
+    return request.param
+
+
 @pytest.mark.parametrize("M,N,K,gs", [(17, 256, 256, 32), (40, 72, 192, 64), (130, 1032, 576, 32),
-                                      (129, 264, 448, 16), (300, 520, 320, 64), (64, 256, 4096, 128)])
-def test_gemm_route_tails(M, N, K, gs):
+                                      (129, 264, 448, 16), (300, 520, 320, 64), (64, 256, 4096, 128),
+                                      (520, 264, 192, 16)])
+def test_gemm_route_tails(M, N, K, gs, msub):
     inp = wl.random_inputs(M, N, K, gs, seed=M + N + K)
     check_fwd(inp, gs)
-    assert q().q4gsw_last_route().startswith("tcgen05_gemm_fwd")
+    route = q().q4gsw_last_route()
+    assert route.startswith("tcgen05_gemm_fwd") and f"tile={128 * msub}x" in route, route
     check_bwd(inp, gs)
-    assert q().q4gsw_last_route().startswith("tcgen05_gemm_bwd")
+    route = q().q4gsw_last_route()
+    assert route.startswith("tcgen05_gemm_bwd") and f"tile={128 * msub}x" in route, route
 
 
-def test_gemm_split_k_cluster_reduction():
-    # one 128x256 output tile and a long contraction: the route splits K over a cluster
+def test_gemm_variant_choice_is_automatic(monkeypatch):
+    monkeypatch.delenv("Q4GSW_GEMM_MSUB", raising=False)
+    inp = wl.random_inputs(100, 256, 256, 32, seed=5)
+    check_fwd(inp, 32)
+    assert "tile=128x" in q().q4gsw_last_route()   # fewer than 129 tokens: one accumulator
+
+
+def test_gemm_split_k_cluster_reduction(msub):
+    # one output tile and a long contraction: the route splits K over a cluster
     inp = wl.integer_exact_inputs(100, 256, 4096, 64, seed=9)
     y, route = run_fwd(inp, 64)
     assert "x8" in route.split("grid=")[1], route
