@@ -309,9 +309,13 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
   // ---------------------------------------------------------------- epilogue
   // Warps 2..17: warp w reads TMEM lanes 32 (w % 4) .. +31 (tokens) and the 64
   // accumulator columns [64 h, 64 h + 64) with h = (w - 2) / 4, for each of
-  // the MSUB accumulators (sub-tile ms holds tokens m0 + 128 ms ..).
+  // the MSUB accumulators (sub-tile ms holds tokens m0 + 128 ms ..), and parks
+  // them in shared memory (the operand rings are idle by now).  All threads
+  // then copy whole rows out, so each warp store covers 512 contiguous bytes
+  // of one output row; with split-K the copy-out also sums the S partial
+  // tiles of the cluster.
   const bool epi = warp >= 2;
-  float* stage_f32 = reinterpret_cast<float*>(smem);   // split-K staging [128][256], 16-byte chunks swizzled
+  float* stage_f32 = reinterpret_cast<float*>(smem);   // staging [128][256] fp32, 16-byte chunks swizzled
   griddep_wait();   // outputs may still be read by the previous kernel of the stream
   bool have_acc = false;
   if (epi) have_acc = mbar_wait(&ctl->accfull, 0, abort_flag, &g_device_error, 16u);
@@ -330,35 +334,34 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
     if (epi && have_acc) {
       const int q = warp & 3, h = (warp - 2) >> 2;
       const int row = 32 * q + lane;
-      const int m = mb + row;
 #pragma unroll 1
       for (int c32 = 0; c32 < 2; ++c32) {
         const int col = 64 * h + 32 * c32;
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ms * 256 + col), r);
         tmem_wait_ld();
-        if (S == 1) {
-          if (m < args.M) {
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const int n = n0 + col + 4 * v;
-              if (n >= args.out_cols) break;
-              store4(m, n, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                       __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const int chunk = (col >> 2) + v;   // 16-byte chunk of the 1 KB row
-            const float4 val = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-            *reinterpret_cast<float4*>(stage_f32 + row * 256 + 4 * (chunk ^ (row & 7))) = val;
-          }
+        for (int v = 0; v < 8; ++v) {
+          const int chunk = (col >> 2) + v;   // 16-byte chunk of the 1 KB row
+          const float4 val = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          *reinterpret_cast<float4*>(stage_f32 + row * 256 + 4 * (chunk ^ (row & 7))) = val;
         }
       }
     }
-    if (S > 1) {
+    if (S == 1) {
+      __syncthreads();
+      const int rows = args.M - mb < BM ? args.M - mb : BM;
+      if (!*abort_flag) {
+        for (int idx = threadIdx.x; idx < rows * 64; idx += kThreads) {
+          const int row = idx >> 6, chunk = idx & 63;
+          const int n = n0 + 4 * chunk;
+          if (n >= args.out_cols) continue;
+          store4(mb + row, n, *reinterpret_cast<const float4*>(stage_f32 + row * 256 + 4 * (chunk ^ (row & 7))));
+        }
+      }
+      __syncthreads();
+    } else {
       // every thread of every CTA of the cluster passes both barriers, aborted or not
       cg::cluster_group cluster = cg::this_cluster();
       cluster.sync();
