@@ -576,14 +576,35 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
   return e;
 }
 
+}  // namespace q4gsw
+
+#include "q4gsw_gemm_ts.cuh"
+
+namespace q4gsw {
+
+// Route between the two GEMM kernels.  Up to 512 tokens the weight tile lives
+// in tensor memory (its shared-memory traffic is lowest); above, the
+// shared-memory route with two 128-token accumulators per CTA re-reads each
+// activation tile half as often from L2 and wins (measured on B200 at 1024 and
+// 4096 tokens).  Q4GSW_GEMM_KIND=ss or ts pins the route (tests and tuning).
+static bool use_ss_route(int M) {
+  const char* e = getenv("Q4GSW_GEMM_KIND");
+  if (e && e[0] == 's' && e[1] == 's' && e[2] == 0) return true;
+  if (e && e[0] == 't' && e[1] == 's' && e[2] == 0) return false;
+  return M > 512;
+}
+
 cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
                             cudaStream_t stream, char* route, int route_len) {
-  return launch_gemm_impl<false>(packed, N, K, gs, x, M, out, stream, route, route_len);
+  if (use_ss_route(M)) return launch_gemm_impl<false>(packed, N, K, gs, x, M, out, stream, route, route_len);
+  return launch_gemm_ts_impl<false>(packed, N, K, gs, x, M, out, stream, route, route_len);
 }
 
 cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
                             cudaStream_t stream, char* route, int route_len) {
-  return launch_gemm_impl<true>(packed, N, K, gs, d_out, M, single_output(d_x, K), stream, route, route_len);
+  if (use_ss_route(M))
+    return launch_gemm_impl<true>(packed, N, K, gs, d_out, M, single_output(d_x, K), stream, route, route_len);
+  return launch_gemm_ts_impl<true>(packed, N, K, gs, d_out, M, single_output(d_x, K), stream, route, route_len);
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int* host_value) {

@@ -1,0 +1,482 @@
+// q4gsw_gemm_ts.cuh - tcgen05 GEMM route with the dequantised weight tile in
+// tensor memory (sm_100a).  Included once, by q4gsw_gemm_sm100.cu, which owns
+// the device error word and the tensor-map helpers.
+//
+// The same two products as the shared-memory route, transposed so that the
+// weight is the MMA's M side:
+//   forward   y^T[n, m]   = sum_k w[n, k]   x[m, k]        (A = w tile,   B = x tile)
+//   backward  d_x^T[k, m] = sum_n w^T[k, n] d_out[m, n]    (A = w^T tile, B = d_out tile)
+// with w[n, k] = (code[n, k] - 8) * s[k / gs, n] ("[ExecuTorch][Vulkan] Add
+// et_vk.linear_q4gsw_backward kernel (4-bit input-grad)", PR description).
+//
+// Why transposed: the dequantisation warps write the fp16 weight tile straight
+// into tensor memory (tcgen05.st), where tcgen05.mma reads it as the A operand.
+// Only the activation tile and the 4-bit codes pass through shared memory, so
+// per 128 x 256 x 64 step the shared-memory traffic is the 32 KB activation
+// copy in, the MMA's 32 KB read of it and 4 KB of codes, against 112 KB when
+// the dequantised tile is stored to and re-read from shared memory.
+//
+// One CTA computes 128 weight rows (output features) x bt tokens (bt <= 256,
+// a multiple of 16, chosen per launch to balance the token tiles), optionally
+// for one slice of the contraction (split-K, reduced in a cluster through
+// distributed shared memory).  Warp roles:
+//   warp 0       TMA producer: activation tile [bt][64] fp16 (128-byte
+//                swizzle), packed codes and scale rows of each 64-deep stage;
+//   warp 1       allocates tensor memory (fp32 accumulator in columns 0..255,
+//                a ring of WST dequantised stages of 32 columns after it) and
+//                issues tcgen05.mma from one thread;
+//   warps 2..17  warp w writes TMEM lanes 32 (w % 4) .. +31 (weight rows) and
+//                the 16-deep contraction slice (w - 2) / 4 of every stage, then
+//                runs the epilogue for the same lanes.
+// Every consumer waits on every phase of the barriers it uses.
+#pragma once
+
+namespace q4gsw {
+namespace ts {
+
+constexpr int BW = 128;                    // weight rows per tile (MMA M)
+constexpr int BT_MAX = 256;                // tokens per tile (MMA N)
+constexpr int TK = 64;                     // contraction depth per stage
+constexpr int WST = 4;                     // tensor-memory ring of dequantised stages
+constexpr int kDequantWarps = 16;
+constexpr int kThreads = 32 * (2 + kDequantWarps);
+constexpr int X_BYTES = BT_MAX * TK * 2;   // activation tile, 32 KB
+constexpr int P_BYTES = BW / 2 * TK;       // packed codes of one stage, 4 KB
+constexpr int SC_BYTES = 1024;             // scale rows of one stage (at most)
+constexpr int CTL_BYTES = 256;
+constexpr int ACC_COLS = 256;              // fp32 accumulator columns (tokens)
+constexpr int A_COLS = TK / 2;             // one dequantised stage: 64 fp16 per lane = 32 columns
+constexpr int TMEM_COLS = 512;
+static_assert(ACC_COLS + WST * A_COLS <= TMEM_COLS, "tensor memory budget");
+
+template <int ST>
+struct Smem {
+  static constexpr int OFF_X = 0;
+  static constexpr int OFF_P = OFF_X + ST * X_BYTES;
+  static constexpr int OFF_SC = OFF_P + ST * P_BYTES;
+  static constexpr int OFF_CTL = OFF_SC + ST * SC_BYTES;
+  static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
+  static_assert(OFF_P % 1024 == 0 && OFF_SC % 1024 == 0, "1024-byte aligned regions");
+  static_assert(BT_MAX * BW * 4 <= OFF_SC, "split-K staging must fit below the scale slots");
+  static_assert(BYTES <= 232448, "shared memory per CTA");
+};
+
+struct Args {
+  OutSplit out;
+  int M, N, K, gs;
+  int rows_out;       // weight-side extent of the output: N (forward) or K (backward)
+  int stages_total;
+  int sc_bytes;       // bytes of the scale box of one stage
+  int bt;             // tokens per tile
+};
+
+struct Ctl {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t wready[WST];
+  uint64_t wempty[WST];
+  uint64_t accfull;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Ctl) <= CTL_BYTES, "control block");
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// (1024 + lo nibble, 1024 + nibble at bits 16..19) -> exact (c - 8) half2
+__device__ __forceinline__ uint32_t nibbles_minus8(uint32_t v) {
+  const __half2 kSub = u32_as_h2(0x64086408u);   // 1032, 1032
+  return h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(v, 0x000F000Fu, 0x64006400u)), kSub));
+}
+
+template <bool BWD, int ST>
+__global__ void __launch_bounds__(kThreads, 1)
+q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
+                     const __grid_constant__ CUtensorMap map_sc, const Args args) {
+  using namespace sm100;
+  using SM = Smem<ST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + SM::OFF_CTL);
+  volatile int* abort_flag = &ctl->abort;
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f0 = blockIdx.x * BW;          // first weight row (output feature) of the tile
+  const int t0 = blockIdx.y * args.bt;     // first token of the tile
+  const int S = gridDim.z, split = blockIdx.z;
+  const int st_begin = (int)((long long)split * args.stages_total / S);
+  const int st_end = (int)((long long)(split + 1) * args.stages_total / S);
+  const int nit = st_end - st_begin;
+  const int gsl = __ffs(args.gs) - 1;
+
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], 1);
+    }
+    for (int i = 0; i < WST; ++i) {
+      mbar_init(&ctl->wready[i], kDequantWarps);
+      mbar_init(&ctl->wempty[i], 1);
+    }
+    mbar_init(&ctl->accfull, 1);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&map_act);
+    prefetch_tmap(&map_pk);
+    prefetch_tmap(&map_sc);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint32_t tx = (uint32_t)args.bt * TK * 2 + P_BYTES + args.sc_bytes;
+      auto load_weights = [&](int it) {
+        const int s = it % ST;
+        const int kc = (st_begin + it) * TK;
+        uint8_t* pk = smem + SM::OFF_P + s * P_BYTES;
+        uint8_t* sc = smem + SM::OFF_SC + s * SC_BYTES;
+        if (!BWD) {
+          tma_load_2d(pk, &map_pk, &ctl->full[s], kc, f0 / 2);       // [64 pairs][64 B]
+          tma_load_2d(sc, &map_sc, &ctl->full[s], f0, kc >> gsl);    // [rows][128 n]
+        } else {
+          tma_load_2d(pk, &map_pk, &ctl->full[s], f0, kc / 2);       // [32 pairs][128 B]
+          tma_load_2d(sc, &map_sc, &ctl->full[s], kc, f0 >> gsl);    // [rows][64 n]
+        }
+      };
+      auto load_act = [&](int it) {
+        const int s = it % ST;
+        tma_load_2d(smem + SM::OFF_X + s * X_BYTES, &map_act, &ctl->full[s], (st_begin + it) * TK, t0);
+      };
+      // The packed weight is constant: the first stages' codes and scales are
+      // requested before waiting for the previous kernel of the stream, which
+      // may still be producing the activations.
+      const int pre = nit < ST ? nit : ST;
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&ctl->full[it], tx);
+        load_weights(it);
+      }
+      griddep_wait();
+      for (int it = 0; it < pre; ++it) load_act(it);
+      int issued = pre;
+      for (int it = pre; it < nit; ++it) {
+        const int s = it % ST;
+        if (!mbar_wait(&ctl->empty[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
+        mbar_arrive_expect_tx(&ctl->full[s], tx);
+        load_weights(it);
+        load_act(it);
+        issued = it + 1;
+      }
+      // never leave with copies in flight: wait for the last fill of each stage
+      for (int it = (issued > ST ? issued - ST : 0); it < issued; ++it)
+        mbar_wait_teardown(&ctl->full[it % ST], (it / ST) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(BW, args.bt, false);
+      for (int it = 0; it < nit; ++it) {
+        const int s = it % ST, w = it % WST;
+        if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 2u)) break;
+        if (!mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
+        tc_fence_after();
+        const uint32_t x0 = sbase + SM::OFF_X + s * X_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < TK / 16; ++ks) {
+          const uint64_t bd = smem_desc_sw128(x0 + 32 * ks, 16, 1024);
+          mma_f16_ts(tmem, tmem + ACC_COLS + w * A_COLS + 8 * ks, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&ctl->empty[s]);
+        mma_commit(&ctl->wempty[w]);
+      }
+      mma_commit(&ctl->accfull);
+      mma_commit(&ctl->drain);
+      mbar_wait_teardown(&ctl->drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ dequantisation
+    // Thread = weight row r of the tile (its TMEM lane); the warp's slice kq
+    // covers contraction columns 16 kq .. 16 kq + 15 of each stage, i.e. the
+    // 8 TMEM columns 8 kq .. 8 kq + 7 of the stage (two fp16 per column, lower
+    // index in the low half).
+    const int q = warp & 3, kq = (warp - 2) >> 2;
+    const int r = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    uint32_t off[8];
+    uint32_t sc_off, shift = 0;
+    if (!BWD) {
+      // Row r = 2 p + odd of pair p.  Word kq of the 16-byte chunk t of the
+      // pair row holds columns 16 kq + 4 t + (0, 2, 1, 3) in its byte slots;
+      // the chunk sits at 16 (t ^ ((p >> 1) & 3)) under the 64-byte swizzle.
+      const int p = r >> 1;
+      shift = 4 * (r & 1);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) off[t] = p * 64 + 16 * (t ^ ((p >> 1) & 3)) + 4 * kq;
+      // the 16 columns share one scale: row ((kc mod gs) + 16 kq) >> gsl of
+      // the stage's box (stages start on 64-column boundaries)
+      sc_off = (args.gs < 64 ? ((16 * kq) >> gsl) : 0) * 256 + 2 * r;
+    } else {
+      // Row r = output feature k = f0 + r.  Pair row p (contraction rows 2p,
+      // 2p+1) holds it in byte column_offset(r) of its 128-byte box row; the
+      // scale of both rows sits in scale row ((f0 mod gs) + r) >> gsl.
+      const uint32_t boff = (uint32_t)column_offset(r);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) off[j] = (8 * kq + j) * 128 + boff;
+      sc_off = (uint32_t)((((f0 & (args.gs - 1)) + r) >> gsl) * 128 + 4 * 8 * kq);
+    }
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % ST, w = it % WST;
+      if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
+      if (it >= WST && !mbar_wait(&ctl->wempty[w], ((it / WST) - 1) & 1, abort_flag, &g_device_error, 32u)) break;
+      tc_fence_after();
+      const uint32_t pk = sbase + SM::OFF_P + s * P_BYTES;
+      const uint32_t sc = sbase + SM::OFF_SC + s * SC_BYTES;
+      uint32_t v[8];
+      if (!BWD) {
+        uint32_t wd[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) wd[t] = lds32(pk + off[t]);
+        const uint32_t sb = lds_u16(sc + sc_off);
+        const __half2 s2 = u32_as_h2(sb | (sb << 16));
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const uint32_t W = wd[t] >> shift;                                      // this row's nibbles
+          v[2 * t] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W)), s2));       // columns 4t, 4t+1
+          v[2 * t + 1] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W >> 8)), s2));  // 4t+2, 4t+3
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t b = lds_u8(pk + off[j]);                 // code[2p, k] | code[2p+1, k] << 4
+          const uint32_t s2 = lds32(sc + sc_off + 4 * j);          // s[g, 2p], s[g, 2p+1]
+          v[j] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(b * 0x1001u)), u32_as_h2(s2)));
+        }
+      }
+      tmem_st_32x32b_x8(tmem + lane_base + (uint32_t)(ACC_COLS + w * A_COLS + 8 * kq), v);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->wready[w]);
+    }
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  // Warp w (2..17) reads TMEM lanes 32 (w % 4) .. +31 (weight rows) and the
+  // token columns [64 c, 64 c + 64) with c = (w - 2) / 4.  Without split-K
+  // each lane stores its feature of 32 tokens, so a warp store covers 128
+  // contiguous bytes of one output row.  With split-K the tile is parked in
+  // shared memory as [token][128 features] and the cluster sums the S partial
+  // tiles row by row.
+  const bool epi = warp >= 2;
+  griddep_wait();   // outputs may still be read by the previous kernel of the stream
+  bool have_acc = false;
+  if (epi) {
+    have_acc = mbar_wait(&ctl->accfull, 0, abort_flag, &g_device_error, 16u);
+    have_acc = __all_sync(0xffffffffu, have_acc);
+    if (have_acc) tc_fence_after();
+  }
+  const OutSplit& o = args.out;
+  float* stage_f32 = reinterpret_cast<float*>(smem);   // split-K staging [256 tokens][128 features]
+  if (epi && have_acc) {
+    const int q = warp & 3, cb = (warp - 2) >> 2;
+    const int r = 32 * q + lane;
+    const int f = f0 + r;
+    float* base = nullptr;
+    size_t ld = 0;
+    if (S == 1 && f < args.rows_out) {
+      if (f < o.n1) { base = o.y0 + f; ld = (size_t)o.n1; }
+      else if (f < o.n2) { base = o.y1 + (f - o.n1); ld = (size_t)(o.n2 - o.n1); }
+      else { base = o.y2 + (f - o.n2); ld = (size_t)(o.N - o.n2); }
+    }
+#pragma unroll 1
+    for (int c32 = 0; c32 < 2; ++c32) {
+      const int col = 64 * cb + 32 * c32;
+      if (col >= args.bt) break;
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, v);
+      tmem_wait_ld();
+      if (S == 1) {
+        if (base) {
+          // tokens of this tile only: columns past bt hold no accumulator
+          const int mlim = min(args.M - (t0 + col), args.bt - col);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < mlim) base[(size_t)(t0 + col + j) * ld] = __uint_as_float(v[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage_f32[(col + j) * BW + r] = __uint_as_float(v[j]);
+      }
+    }
+  }
+  if (S > 1) {
+    // every thread of every CTA of the cluster passes both barriers, aborted or not
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int rk = (int)cluster.block_rank();
+    const int row_b = rk * args.bt / S, row_e = (rk + 1) * args.bt / S;
+    if (!*abort_flag) {
+      for (int idx = threadIdx.x; idx < (row_e - row_b) * (BW / 4); idx += kThreads) {
+        const int row = row_b + idx / (BW / 4), c4 = idx % (BW / 4);
+        const int m = t0 + row, f = f0 + 4 * c4;
+        if (m >= args.M || f >= args.rows_out) continue;
+        const int offs = row * BW + 4 * c4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int qq = 0; qq < S; ++qq) {
+          const float4 vv = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + offs);
+          acc.x += vv.x;
+          acc.y += vv.y;
+          acc.z += vv.z;
+          acc.w += vv.w;
+        }
+        float* dst;
+        if (f < o.n1) dst = o.y0 + (size_t)m * o.n1 + f;
+        else if (f < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (f - o.n1);
+        else dst = o.y2 + (size_t)m * (o.N - o.n2) + (f - o.n2);
+        *reinterpret_cast<float4*>(dst) = acc;
+      }
+    }
+    cluster.sync();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace ts
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+template <bool BWD>
+static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs, const uint16_t* act, int M,
+                                       OutSplit out, cudaStream_t stream, char* route, int route_len) {
+  using namespace ts;
+  constexpr int ST = 6;
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  const Layout L = layout_of(N, K, gs);
+  const void* scales = pk + L.scales_offset;
+  const int G = K / gs;
+  Args a;
+  a.out = out;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.gs = gs;
+  a.rows_out = BWD ? K : N;
+  const int contraction = BWD ? N : K;
+  a.stages_total = (contraction + TK - 1) / TK;
+  // token tiles: as few as fit 256 tokens, balanced, rounded up to 16
+  const int tiles_t = (M + BT_MAX - 1) / BT_MAX;
+  a.bt = (((M + tiles_t - 1) / tiles_t) + 15) / 16 * 16;
+  const int tiles_f = (a.rows_out + BW - 1) / BW;
+
+  CUtensorMap map_act, map_pk, map_sc;
+  bool ok = make_map_2d(&map_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act, (uint64_t)contraction, M,
+                        (uint64_t)contraction * 2, TK, a.bt, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!BWD) {
+    const int rows = TK / gs > 1 ? TK / gs : 1;   // scale groups of one 64-column stage
+    a.sc_bytes = rows * BW * 2;
+    ok = ok && make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BW / 2,
+                           CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, BW, rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+  } else {
+    const int rows = BW / gs > 1 ? BW / gs : 1;   // scale groups of one 128-feature tile
+    a.sc_bytes = rows * TK * 2;
+    ok = ok && make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, BW, TK / 2,
+                           CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, TK, rows,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  if (!ok || a.sc_bytes > SC_BYTES) return cudaErrorInvalidValue;
+
+  auto kern = q4gsw_gemm_ts_kernel<BWD, ST>;
+  constexpr int smem = Smem<ST>::BYTES;
+  static bool attr_done[64] = {};
+  static int max_clusters[64][9] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int d = (dev >= 0 && dev < 64) ? dev : 0;
+  if (!attr_done[d]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_done[d] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+
+  // Split-K S: each candidate costs waves(S) * (stages / S + fixed overhead:
+  // 2 stages, or 8 with the cluster reduction), where waves(S) uses how many
+  // S-CTA clusters the device can hold at once.
+  const int tiles = tiles_f * tiles_t;
+  int best_S = 1;
+  double best_cost = 1e30;
+  for (int S = 1; S <= 8; ++S) {
+    if (S > 1 && a.stages_total / S < 4) break;
+    if (!max_clusters[d][S]) {
+      attr[0].val.clusterDim.z = S;
+      cfg.gridDim = dim3(tiles_f, tiles_t, S);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = -1;
+      max_clusters[d][S] = n;
+    }
+    const int n = max_clusters[d][S];
+    if (n < 1) continue;
+    const double waves = ceil((double)tiles / n);
+    const double cost = waves * ((double)a.stages_total / S + (S > 1 ? 8.0 : 2.0));
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best_S = S;
+    }
+  }
+  attr[0].val.clusterDim.z = best_S;
+  cfg.gridDim = dim3(tiles_f, tiles_t, best_S);
+  if (route)
+    snprintf(route, route_len, "tcgen05_ts_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d",
+             BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, WST, tiles_f, tiles_t, best_S);
+  return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, a);
+}
+
+}  // namespace q4gsw

@@ -221,35 +221,59 @@ def test_non_default_stream():
     assert_within_bound(y.cpu().numpy(), ref, bnd)
 
 
-# ----------------------------------------------------------------------------- tcgen05 GEMM route
-@pytest.fixture(params=[1, 2], ids=["msub1", "msub2"])
-def msub(request, monkeypatch):
-    """Pins the GEMM variant: one or two 128-token accumulators per CTA."""
-    monkeypatch.setenv("Q4GSW_GEMM_MSUB", str(request.param))
-    return request.param
+# ----------------------------------------------------------------------------- tcgen05 GEMM routes
+@pytest.fixture(params=["ts", "ss1", "ss2"])
+def gemm_variant(request, monkeypatch):
+    """Pins the GEMM route: weight tile in tensor memory (ts, the default), or
+    dequantised into shared memory with one or two 128-token accumulators."""
+    v = request.param
+    monkeypatch.setenv("Q4GSW_GEMM_KIND", v[:2])
+    if v.startswith("ss"):
+        monkeypatch.setenv("Q4GSW_GEMM_MSUB", v[2])
+    return v
+
+
+def _route_ok(route, direction, variant):
+    if variant == "ts":
+        return route.startswith(f"tcgen05_ts_gemm_{direction}") and "tile=128x" in route
+    return route.startswith(f"tcgen05_gemm_{direction}") and f"tile={128 * int(variant[2])}x" in route
 
 
 @pytest.mark.parametrize("M,N,K,gs", [(17, 256, 256, 32), (40, 72, 192, 64), (130, 1032, 576, 32),
                                       (129, 264, 448, 16), (300, 520, 320, 64), (64, 256, 4096, 128),
-                                      (520, 264, 192, 16)])
-def test_gemm_route_tails(M, N, K, gs, msub):
+                                      (520, 264, 192, 16), (33, 136, 128, 128)])
+def test_gemm_route_tails(M, N, K, gs, gemm_variant):
     inp = wl.random_inputs(M, N, K, gs, seed=M + N + K)
     check_fwd(inp, gs)
     route = q().q4gsw_last_route()
-    assert route.startswith("tcgen05_gemm_fwd") and f"tile={128 * msub}x" in route, route
+    assert _route_ok(route, "fwd", gemm_variant), route
     check_bwd(inp, gs)
     route = q().q4gsw_last_route()
-    assert route.startswith("tcgen05_gemm_bwd") and f"tile={128 * msub}x" in route, route
+    assert _route_ok(route, "bwd", gemm_variant), route
 
 
-def test_gemm_variant_choice_is_automatic(monkeypatch):
+def test_gemm_default_routes(monkeypatch):
+    monkeypatch.delenv("Q4GSW_GEMM_KIND", raising=False)
+    monkeypatch.delenv("Q4GSW_GEMM_MSUB", raising=False)
+    inp = wl.random_inputs(100, 256, 256, 32, seed=5)
+    check_fwd(inp, 32)
+    route = q().q4gsw_last_route()
+    assert route.startswith("tcgen05_ts_gemm_fwd") and "tile=128x112x64" in route, route   # one 112-token tile
+    inp = wl.random_inputs(600, 256, 256, 32, seed=6)
+    check_bwd(inp, 32)
+    route = q().q4gsw_last_route()
+    assert route.startswith("tcgen05_gemm_bwd"), route   # above 512 tokens: shared-memory route
+
+
+def test_ss_variant_choice_is_automatic(monkeypatch):
+    monkeypatch.setenv("Q4GSW_GEMM_KIND", "ss")
     monkeypatch.delenv("Q4GSW_GEMM_MSUB", raising=False)
     inp = wl.random_inputs(100, 256, 256, 32, seed=5)
     check_fwd(inp, 32)
     assert "tile=128x" in q().q4gsw_last_route()   # fewer than 129 tokens: one accumulator
 
 
-def test_gemm_split_k_cluster_reduction(msub):
+def test_gemm_split_k_cluster_reduction(gemm_variant):
     # one output tile and a long contraction: the route splits K over a cluster
     inp = wl.integer_exact_inputs(100, 256, 4096, 64, seed=9)
     y, route = run_fwd(inp, 64)
