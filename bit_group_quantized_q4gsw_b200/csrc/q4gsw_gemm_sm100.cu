@@ -88,10 +88,9 @@ struct Args {
 
 constexpr int kMaxST = 5;
 struct SmemCtl {
-  uint64_t full[kMaxST];
-  uint64_t empty[kMaxST];
-  uint64_t wready[WST];
-  uint64_t wempty[WST];
+  uint64_t full[kMaxST];       // stage s loaded (TMA transaction bytes)
+  uint64_t consumed[kMaxST];   // the MMAs of the stage in slot s completed (one commit per stage)
+  uint64_t wready[WST];        // dequantised tile w written (all dequantisation warps)
   uint64_t accfull;
   uint64_t drain;
   uint32_t tmem_base;
@@ -143,11 +142,10 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(&ctl->full[i], 1);
-      mbar_init(&ctl->empty[i], 1);
+      mbar_init(&ctl->consumed[i], 1);
     }
     for (int i = 0; i < WST; ++i) {
       mbar_init(&ctl->wready[i], kDequantWarps);
-      mbar_init(&ctl->wempty[i], 1);
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
@@ -200,7 +198,7 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       int issued = pre;
       for (int it = pre; it < nit; ++it) {
         const int s = it % ST;
-        if (!mbar_wait(&ctl->empty[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
+        if (!mbar_wait(&ctl->consumed[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
         mbar_arrive_expect_tx(&ctl->full[s], A_STAGE + P_BYTES + args.sc_bytes);
         load_weights(it);
         load_act(it);
@@ -212,26 +210,31 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Between stages this thread only waits on wready (each dequantisation
+    // warp saw the stage's full barrier before arriving), tests the next
+    // stage's wready while the last MMAs of this stage are queued, and
+    // commits once: the tensor core holds little more than the MMA it runs.
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(BM, BN, BWD);
+      bool next_ready = false;
       for (int it = 0; it < nit; ++it) {
         const int s = it % ST, w = it % WST;
-        if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 2u)) break;
-        if (!mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
+        if (!next_ready && !mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
         tc_fence_after();
         const uint32_t a0 = sbase + OFF_A + s * A_STAGE, w0 = sbase + OFF_W + w * W_BYTES;
 #pragma unroll
         for (int ks = 0; ks < TK / 16; ++ks) {
           const uint64_t bd = BWD ? smem_desc_sw128(w0 + ks * 2048, 8192, 1024)
                                   : smem_desc_sw128(w0 + 32 * ks, 16, 1024);
+          if (ks == TK / 16 - 1)
+            next_ready = it + 1 < nit && mbar_test_wait(&ctl->wready[(it + 1) % WST], ((it + 1) / WST) & 1);
 #pragma unroll
           for (int ms = 0; ms < MSUB; ++ms) {
             const uint64_t ad = smem_desc_sw128(a0 + ms * A_BYTES + 32 * ks, 16, 1024);
             mma_f16_ss(tmem + ms * 256, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
           }
         }
-        mma_commit(&ctl->empty[s]);
-        mma_commit(&ctl->wempty[w]);
+        mma_commit(&ctl->consumed[s]);
       }
       mma_commit(&ctl->accfull);
       mma_commit(&ctl->drain);
@@ -277,7 +280,10 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
     for (int it = 0; it < nit; ++it) {
       const int s = it % ST, w = it % WST;
       if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
-      if (it >= WST && !mbar_wait(&ctl->wempty[w], ((it / WST) - 1) & 1, abort_flag, &g_device_error, 32u)) break;
+      // tile w is free once the MMAs of stage it - WST completed
+      if (it >= WST &&
+          !mbar_wait(&ctl->consumed[(it - WST) % ST], ((it - WST) / ST) & 1, abort_flag, &g_device_error, 32u))
+        break;
       const uint32_t pk = sbase + OFF_P + s * P_BYTES;
       const uint32_t sc = sbase + OFF_SC + s * SC_BYTES;
       const uint2 c0 = lds64(pk + pk_off0);
@@ -373,14 +379,20 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
           const int m = mb + row, n = n0 + 4 * chunk;
           if (m >= args.M || n >= args.out_cols) continue;
           const int off = row * 256 + 4 * (chunk ^ (row & 7));
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int qq = 0; qq < S; ++qq) {
-            const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + off);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
-          }
+          // all S loads in flight at once, then the sum in rank order
+          float4 part[8];
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq)
+            if (qq < S) part[qq] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + off);
+          float4 acc = part[0];
+#pragma unroll
+          for (int qq = 1; qq < 8; ++qq)
+            if (qq < S) {
+              acc.x += part[qq].x;
+              acc.y += part[qq].y;
+              acc.z += part[qq].z;
+              acc.w += part[qq].w;
+            }
           store4(m, n, acc);
         }
       }

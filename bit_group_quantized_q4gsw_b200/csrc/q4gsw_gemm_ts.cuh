@@ -68,13 +68,13 @@ struct Args {
   int stages_total;
   int sc_bytes;       // bytes of the scale box of one stage
   int bt;             // tokens per tile
+  int tma_out;        // outputs written by tensor store / reduce-add (map_y*), else by threads
 };
 
 struct Ctl {
-  uint64_t full[8];
-  uint64_t empty[8];
-  uint64_t wready[WST];
-  uint64_t wempty[WST];
+  uint64_t full[8];       // stage s loaded (TMA transaction bytes)
+  uint64_t consumed[8];   // the MMAs of the stage in slot s completed (one commit per stage)
+  uint64_t wready[WST];   // dequantised stage in TMEM slot w written (all dequantisation warps)
   uint64_t accfull;
   uint64_t drain;
   uint32_t tmem_base;
@@ -109,7 +109,9 @@ __device__ __forceinline__ uint32_t nibbles_minus8(uint32_t v) {
 template <bool BWD, int ST>
 __global__ void __launch_bounds__(kThreads, 1)
 q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
-                     const __grid_constant__ CUtensorMap map_sc, const Args args) {
+                     const __grid_constant__ CUtensorMap map_sc, const __grid_constant__ CUtensorMap map_y0,
+                     const __grid_constant__ CUtensorMap map_y1, const __grid_constant__ CUtensorMap map_y2,
+                     const Args args) {
   using namespace sm100;
   using SM = Smem<ST>;
   extern __shared__ uint8_t smem_raw[];
@@ -131,12 +133,9 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(&ctl->full[i], 1);
-      mbar_init(&ctl->empty[i], 1);
+      mbar_init(&ctl->consumed[i], 1);
     }
-    for (int i = 0; i < WST; ++i) {
-      mbar_init(&ctl->wready[i], kDequantWarps);
-      mbar_init(&ctl->wempty[i], 1);
-    }
+    for (int i = 0; i < WST; ++i) mbar_init(&ctl->wready[i], kDequantWarps);
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -188,7 +187,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       int issued = pre;
       for (int it = pre; it < nit; ++it) {
         const int s = it % ST;
-        if (!mbar_wait(&ctl->empty[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
+        if (!mbar_wait(&ctl->consumed[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
         mbar_arrive_expect_tx(&ctl->full[s], tx);
         load_weights(it);
         load_act(it);
@@ -200,21 +199,28 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The tensor core accepts little more than the MMA it is executing, so
+    // every cycle this thread spends between stages is a bubble: it waits on
+    // wready alone (each dequantisation warp saw the stage's full barrier
+    // before arriving, so wready covers the activation tile too), tests the
+    // next stage's barrier while the last MMA of this stage is queued, and
+    // commits once per stage.
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(BW, args.bt, false);
+      bool next_ready = false;
       for (int it = 0; it < nit; ++it) {
         const int s = it % ST, w = it % WST;
-        if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 2u)) break;
-        if (!mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
+        if (!next_ready && !mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
         tc_fence_after();
         const uint32_t x0 = sbase + SM::OFF_X + s * X_BYTES;
 #pragma unroll
         for (int ks = 0; ks < TK / 16; ++ks) {
+          if (ks == TK / 16 - 1)
+            next_ready = it + 1 < nit && mbar_test_wait(&ctl->wready[(it + 1) % WST], ((it + 1) / WST) & 1);
           const uint64_t bd = smem_desc_sw128(x0 + 32 * ks, 16, 1024);
           mma_f16_ts(tmem, tmem + ACC_COLS + w * A_COLS + 8 * ks, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
         }
-        mma_commit(&ctl->empty[s]);
-        mma_commit(&ctl->wempty[w]);
+        mma_commit(&ctl->consumed[s]);
       }
       mma_commit(&ctl->accfull);
       mma_commit(&ctl->drain);
@@ -254,7 +260,10 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     for (int it = 0; it < nit; ++it) {
       const int s = it % ST, w = it % WST;
       if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
-      if (it >= WST && !mbar_wait(&ctl->wempty[w], ((it / WST) - 1) & 1, abort_flag, &g_device_error, 32u)) break;
+      // TMEM slot w is free once the MMAs of stage it - WST completed
+      if (it >= WST &&
+          !mbar_wait(&ctl->consumed[(it - WST) % ST], ((it - WST) / ST) & 1, abort_flag, &g_device_error, 32u))
+        break;
       tc_fence_after();
       const uint32_t pk = sbase + SM::OFF_P + s * P_BYTES;
       const uint32_t sc = sbase + SM::OFF_SC + s * SC_BYTES;
@@ -289,11 +298,8 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
 
   // ---------------------------------------------------------------- epilogue
   // Warp w (2..17) reads TMEM lanes 32 (w % 4) .. +31 (weight rows) and the
-  // token columns [64 c, 64 c + 64) with c = (w - 2) / 4.  Without split-K
-  // each lane stores its feature of 32 tokens, so a warp store covers 128
-  // contiguous bytes of one output row.  With split-K the tile is parked in
-  // shared memory as [token][128 features] and the cluster sums the S partial
-  // tiles row by row.
+  // token columns [64 c, 64 c + 64) with c = (w - 2) / 4, and parks them in
+  // shared memory (the operand ring is idle by now) as [token][128 features].
   const bool epi = warp >= 2;
   griddep_wait();   // outputs may still be read by the previous kernel of the stream
   bool have_acc = false;
@@ -303,18 +309,10 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     if (have_acc) tc_fence_after();
   }
   const OutSplit& o = args.out;
-  float* stage_f32 = reinterpret_cast<float*>(smem);   // split-K staging [256 tokens][128 features]
+  float* stage_f32 = reinterpret_cast<float*>(smem);   // staging [256 tokens][128 features]
   if (epi && have_acc) {
     const int q = warp & 3, cb = (warp - 2) >> 2;
     const int r = 32 * q + lane;
-    const int f = f0 + r;
-    float* base = nullptr;
-    size_t ld = 0;
-    if (S == 1 && f < args.rows_out) {
-      if (f < o.n1) { base = o.y0 + f; ld = (size_t)o.n1; }
-      else if (f < o.n2) { base = o.y1 + (f - o.n1); ld = (size_t)(o.n2 - o.n1); }
-      else { base = o.y2 + (f - o.n2); ld = (size_t)(o.N - o.n2); }
-    }
 #pragma unroll 1
     for (int c32 = 0; c32 < 2; ++c32) {
       const int col = 64 * cb + 32 * c32;
@@ -322,48 +320,89 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, v);
       tmem_wait_ld();
-      if (S == 1) {
-        if (base) {
-          // tokens of this tile only: columns past bt hold no accumulator
-          const int mlim = min(args.M - (t0 + col), args.bt - col);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < mlim) base[(size_t)(t0 + col + j) * ld] = __uint_as_float(v[j]);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stage_f32[(col + j) * BW + r] = __uint_as_float(v[j]);
-      }
+      for (int j = 0; j < 32; ++j) stage_f32[(col + j) * BW + r] = __uint_as_float(v[j]);
     }
   }
-  if (S > 1) {
-    // every thread of every CTA of the cluster passes both barriers, aborted or not
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    const int rk = (int)cluster.block_rank();
-    const int row_b = rk * args.bt / S, row_e = (rk + 1) * args.bt / S;
-    if (!*abort_flag) {
-      for (int idx = threadIdx.x; idx < (row_e - row_b) * (BW / 4); idx += kThreads) {
-        const int row = row_b + idx / (BW / 4), c4 = idx % (BW / 4);
-        const int m = t0 + row, f = f0 + 4 * c4;
-        if (m >= args.M || f >= args.rows_out) continue;
-        const int offs = row * BW + 4 * c4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int qq = 0; qq < S; ++qq) {
-          const float4 vv = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + offs);
-          acc.x += vv.x;
-          acc.y += vv.y;
-          acc.z += vv.z;
-          acc.w += vv.w;
-        }
-        float* dst;
-        if (f < o.n1) dst = o.y0 + (size_t)m * o.n1 + f;
-        else if (f < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (f - o.n1);
-        else dst = o.y2 + (size_t)m * (o.N - o.n2) + (f - o.n2);
-        *reinterpret_cast<float4*>(dst) = acc;
+  if (args.tma_out) {
+    // Tensor store of the [bt][128] fp32 tile (rows past M and features past
+    // the output clipped by the map).  With split-K, rank 0 stores its partial
+    // and, once that store has completed, the other ranks add theirs at L2
+    // (tensor reduce-add), so no CTA reads another's shared memory and each
+    // leaves as soon as its tile has been read out of shared memory.  The
+    // order of the S-1 additions is not fixed.
+    const CUtensorMap* my = f0 < o.n1 ? &map_y0 : (f0 < o.n2 ? &map_y1 : &map_y2);
+    const int c0 = f0 < o.n1 ? f0 : (f0 < o.n2 ? f0 - o.n1 : f0 - o.n2);
+    fence_proxy_async_smem();
+    __syncthreads();
+    const bool ok = !*abort_flag;
+    if (S == 1) {
+      if (threadIdx.x == 0 && ok) {
+        tma_store_2d(my, stage_f32, c0, t0);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+    } else {
+      cg::cluster_group cluster = cg::this_cluster();
+      const int rk = (int)cluster.block_rank();
+      if (rk == 0 && threadIdx.x == 0 && ok) {
+        tma_store_2d(my, stage_f32, c0, t0);
+        bulk_commit();
+        bulk_wait_all();
+        fence_proxy_async_global();
+      }
+      cluster.sync();   // every thread of every CTA of the cluster, aborted or not
+      if (rk != 0 && threadIdx.x == 0 && ok) {
+        fence_proxy_async_global();
+        tma_reduce_add_2d(my, stage_f32, c0, t0);
+        bulk_commit();
+        bulk_wait_read_all();
       }
     }
-    cluster.sync();
+  } else {
+    // Copy-out: one warp writes 512 contiguous bytes (128 features of one
+    // token); with split-K, rank rk sums rows [rk bt / S, (rk + 1) bt / S) of
+    // the S partial tiles, loading all S before adding them in rank order.
+    // Every thread of every CTA of the cluster passes the barriers, aborted or not.
+    cg::cluster_group cluster = cg::this_cluster();
+    if (S > 1) cluster.sync();
+    else __syncthreads();
+    {
+      const int rk = S > 1 ? (int)cluster.block_rank() : 0;
+      const int row_b = rk * args.bt / S, row_e = (rk + 1) * args.bt / S;
+      if (!*abort_flag) {
+        for (int idx = threadIdx.x; idx < (row_e - row_b) * (BW / 4); idx += kThreads) {
+          const int row = row_b + idx / (BW / 4), c4 = idx % (BW / 4);
+          const int m = t0 + row, f = f0 + 4 * c4;
+          if (m >= args.M || f >= args.rows_out) continue;
+          const int offs = row * BW + 4 * c4;
+          float4 acc;
+          if (S == 1) {
+            acc = *reinterpret_cast<const float4*>(stage_f32 + offs);
+          } else {
+            float4 part[8];
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq)
+              if (qq < S) part[qq] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + offs);
+            acc = part[0];
+#pragma unroll
+            for (int qq = 1; qq < 8; ++qq)
+              if (qq < S) {
+                acc.x += part[qq].x;
+                acc.y += part[qq].y;
+                acc.z += part[qq].z;
+                acc.w += part[qq].w;
+              }
+          }
+          float* dst;
+          if (f < o.n1) dst = o.y0 + (size_t)m * o.n1 + f;
+          else if (f < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (f - o.n1);
+          else dst = o.y2 + (size_t)m * (o.N - o.n2) + (f - o.n2);
+          *reinterpret_cast<float4*>(dst) = acc;
+        }
+      }
+    }
+    if (S > 1) cluster.sync();
   }
   tc_fence_before();
   __syncthreads();
@@ -422,6 +461,29 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
   }
   if (!ok || a.sc_bytes > SC_BYTES) return cudaErrorInvalidValue;
 
+  // Output tensor maps [M][width] fp32, box [bt][128]: usable when every
+  // buffer starts 16-byte aligned and no 128-feature tile straddles two of
+  // them; otherwise the threads write the outputs.
+  CUtensorMap map_y[3];
+  {
+    const int nb[3] = {0, out.n1, out.n2};
+    const int ne[3] = {out.n1, out.n2, out.N};
+    float* const yb[3] = {out.y0, out.y1, out.y2};
+    bool tma_out = (out.n1 % BW == 0 || out.n1 == out.N) && (out.n2 % BW == 0 || out.n2 == out.N);
+    for (int i = 0; i < 3 && tma_out; ++i) {
+      const int width = ne[i] - nb[i];
+      if (width <= 0) {
+        map_y[i] = map_y[0];
+        continue;
+      }
+      tma_out = (reinterpret_cast<uintptr_t>(yb[i]) % 16 == 0) &&
+                make_map_2d(&map_y[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, yb[i], (uint64_t)width, M,
+                            (uint64_t)width * 4, BW, a.bt, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    a.tma_out = tma_out ? 1 : 0;
+    if (!tma_out) map_y[0] = map_y[1] = map_y[2] = map_act;   // never read
+  }
+
   auto kern = q4gsw_gemm_ts_kernel<BWD, ST>;
   constexpr int smem = Smem<ST>::BYTES;
   static bool attr_done[64] = {};
@@ -474,9 +536,9 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
   attr[0].val.clusterDim.z = best_S;
   cfg.gridDim = dim3(tiles_f, tiles_t, best_S);
   if (route)
-    snprintf(route, route_len, "tcgen05_ts_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d",
-             BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, WST, tiles_f, tiles_t, best_S);
-  return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, a);
+    snprintf(route, route_len, "tcgen05_ts_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d out=%s",
+             BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, WST, tiles_f, tiles_t, best_S, a.tma_out ? "tma" : "st");
+  return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, map_y[0], map_y[1], map_y[2], a);
 }
 
 }  // namespace q4gsw
