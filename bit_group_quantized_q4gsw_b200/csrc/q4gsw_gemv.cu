@@ -24,6 +24,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 
 #include "q4gsw_common.cuh"
 #include "q4gsw_internal.h"
@@ -432,8 +433,31 @@ static cudaError_t launch_cluster(Kern kernel, dim3 grid, int threads, int clust
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Route between the two forward GEMVs.  The TMA-ring kernel (64-row CTAs,
+// two per SM for up to 8 tokens) is taken for 9..16 tokens, and for up to 8
+// tokens when its CTAs spread evenly over the SMs (each SM's share within 15 %
+// of the busiest SM's); otherwise the register-fed kernel, whose 16-row CTAs
+// balance better, is faster (measured on B200: 14336x4096 at M=1, 224 CTAs on
+// 148 SMs, 13.4 vs 11.3 us).  Q4GSW_GEMV_KIND=reg or tma pins the route.
+static bool use_reg_gemv(int N, int K, int M) {
+  const char* e = getenv("Q4GSW_GEMV_KIND");
+  if (e && e[0] == 'r' && e[1] == 'e' && e[2] == 'g' && e[3] == 0) return true;
+  if (e && e[0] == 't' && e[1] == 'm' && e[2] == 'a' && e[3] == 0) return false;
+  if (M > 8) return false;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = (N + 63) / 64, stages = (K + 255) / 256;
+  int S = 2 * sms / tiles;
+  S = S < 1 ? 1 : (S > 8 ? 8 : S);
+  while (S > 1 && stages / S < 2) --S;
+  const double per_sm = (double)tiles * S / sms;
+  return per_sm / ceil(per_sm) < 0.85;
+}
+
 cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M,
                             OutSplit out, cudaStream_t stream, char* route, int route_len) {
+  if (!use_reg_gemv(N, K, M)) return launch_gemv_tma_fwd(packed, N, K, gs, x, M, out, stream, route, route_len);
   const int tiles = (N + 15) / 16;
   const int zs = (M + 15) / 16;
   const int NT = (M <= 8) ? 1 : 2;

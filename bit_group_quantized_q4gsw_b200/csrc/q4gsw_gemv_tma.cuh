@@ -1,0 +1,373 @@
+// q4gsw_gemv_tma.cuh - forward GEMV route for small token counts (M <= 16 per
+// z-slice) that streams the packed weight through a TMA ring (sm_100a).
+// Included once, by q4gsw_gemm_sm100.cu, which owns the device error word and
+// the tensor-map helpers.
+//
+//   y[m, n] = sum_k x[m, k] (code[n, k] - 8) s[k / gs, n]
+// ("[ExecuTorch][Vulkan] Add et_vk.linear_q4gsw_backward kernel (4-bit
+// input-grad)", PR description; this is the forward it mirrors.)
+//
+// At M <= 16 the layer is a weight stream: every code byte is read once and
+// used for at most 16 tokens, so the kernel lives or dies by the bytes it keeps
+// in flight.  One producer thread per CTA keeps ST stages of 256 contraction
+// columns in flight with TMA (codes of 32 nibble pairs, their scale rows, the
+// activation columns); sixteen consumer warps (four row groups of 8 pairs x
+// the four 64-column blocks of a stage) turn each stage into mma.sync m16n8k16
+// steps (A = 16 weight rows, B = 8 tokens), with the codes entering the MMA as
+// exact integers code - 8 and the fp16 scale applied to the fp32 partial sum
+// of each group, as in the register-fed GEMV.  The four block slices are summed
+// in shared memory, split-K CTAs of a cluster through distributed shared
+// memory, both in a fixed order.
+#pragma once
+
+namespace q4gsw {
+namespace gv {
+
+constexpr int kRowGroups = 4;                         // 8 nibble pairs (16 rows) each
+constexpr int kBlockSlices = 4;                       // 64-column block of the stage
+constexpr int kConsumerWarps = kRowGroups * kBlockSlices;
+constexpr int kThreads = 32 * (1 + kConsumerWarps);   // warp 0 produces
+constexpr int RP = 8 * kRowGroups;                    // nibble pairs per CTA (64 output rows)
+constexpr int SK = 256;                               // contraction columns per stage
+constexpr int CODE_BYTES = RP * SK;                   // two [32 pairs][128 B] boxes, 8 KB
+constexpr int SC_BYTES = 16 * 128;                    // scale rows of a stage (gs 16: 16 rows of 64 n)
+constexpr int CTL_BYTES = 256;
+
+template <int NT>
+struct Cfg {
+  static constexpr int MB = 8 * NT;                   // token rows of the activation boxes
+  static constexpr int XBOX = MB * 128 < 1024 ? 1024 : MB * 128;   // one [MB][64] box, 1 KB aligned
+  static constexpr int X_BYTES = 4 * XBOX;
+  static constexpr int STAGE = CODE_BYTES + SC_BYTES + X_BYTES;
+  // one 8-token tile: two CTAs per SM (registers capped at 60); two tiles:
+  // one CTA per SM with a deeper ring
+  static constexpr int kCtasPerSm = NT == 1 ? 2 : 1;
+  static constexpr int ST = NT == 1 ? 6 : 10;
+  static constexpr int OFF_CTL = ST * STAGE;
+  static constexpr int OFF_RED = OFF_CTL + CTL_BYTES;   // [slice][16 tokens][64 rows] fp32 partial tiles
+  static constexpr int BYTES = OFF_RED + kBlockSlices * 16 * 64 * 4 + 1024;
+  static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
+  static_assert(ST <= 12, "barrier arrays");
+  static_assert(BYTES <= (kCtasPerSm == 2 ? 116 * 1024 : 226 * 1024), "CTAs per SM");
+};
+
+struct Ctl {
+  uint64_t full[12];
+  uint64_t empty[12];
+  int abort;
+};
+static_assert(sizeof(Ctl) <= CTL_BYTES, "control block");
+
+// MMA row g of row group w reads pair row 8 w + perm(g): the two pairs a
+// quarter of the warp reads together then differ in bit 2, so under the
+// 128-byte swizzle their 16-byte code chunks fall on distinct banks.
+__device__ __forceinline__ int pair_of(int w, int g) { return 8 * w + ((g & 1) << 2) + (g >> 1); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// grid = (ceil(N / 64) row tiles, S contraction splits, ceil(M / 16) token
+// slices), cluster = (1, S, 1).  SPG = 16-column steps per scale group
+// (1: gs 16, 2: gs 32, 4: gs >= 64).
+template <int NT, int SPG>
+__global__ void __launch_bounds__(kThreads, Cfg<NT>::kCtasPerSm)
+gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
+                    const __grid_constant__ CUtensorMap map_x, OutSplit out, int M, int N, int K, int gs,
+                    int stages_total) {
+  using namespace sm100;
+  using C = Cfg<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);   // [slice][token][64 rows]
+  volatile int* abort_flag = &ctl->abort;
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, split = blockIdx.y, S = gridDim.y;
+  const int tok0 = blockIdx.z * 16;
+  const int Mz = min(16, M - tok0);
+  const int n0 = tile * 64;
+  const int st_begin = (int)((long long)split * stages_total / S);
+  const int st_end = (int)((long long)(split + 1) * stages_total / S);
+  const int nit = st_end - st_begin;
+  const int gsl = __ffs(gs) - 1;
+
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::ST; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], kConsumerWarps);
+    }
+    ctl->abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&map_pk);
+    prefetch_tmap(&map_sc);
+    prefetch_tmap(&map_x);
+  }
+  __syncthreads();
+
+  // scale rows per stage: (SK / gs) for gs <= SK, else 1
+  const int sc_rows = gs < SK ? SK / gs : 1;
+  const uint32_t tx = CODE_BYTES + sc_rows * 128 + 4 * C::MB * 128;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      auto load_weights = [&](int it) {
+        const int s = it % C::ST;
+        const int kc = (st_begin + it) * SK;
+        uint8_t* st = smem + s * C::STAGE;
+        tma_load_2d(st, &map_pk, &ctl->full[s], kc, n0 / 2);
+        tma_load_2d(st + CODE_BYTES / 2, &map_pk, &ctl->full[s], kc + 128, n0 / 2);
+        tma_load_2d(st + CODE_BYTES, &map_sc, &ctl->full[s], n0, kc >> gsl);
+      };
+      auto load_x = [&](int it) {
+        const int s = it % C::ST;
+        const int kc = (st_begin + it) * SK;
+        uint8_t* xs = smem + s * C::STAGE + CODE_BYTES + SC_BYTES;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(xs + b * C::XBOX, &map_x, &ctl->full[s], kc + 64 * b, tok0);
+      };
+      // the packed weight is constant: its first stages are requested before
+      // waiting for the kernel that produces x
+      const int pre = nit < C::ST ? nit : C::ST;
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&ctl->full[it], tx);
+        load_weights(it);
+      }
+      griddep_wait();
+      for (int it = 0; it < pre; ++it) load_x(it);
+      int issued = pre;
+      for (int it = pre; it < nit; ++it) {
+        const int s = it % C::ST;
+        if (!mbar_wait(&ctl->empty[s], ((it / C::ST) - 1) & 1, abort_flag, &g_device_error, 64u)) break;
+        mbar_arrive_expect_tx(&ctl->full[s], tx);
+        load_weights(it);
+        load_x(it);
+        issued = it + 1;
+      }
+      for (int it = (issued > C::ST ? issued - C::ST : 0); it < issued; ++it)
+        mbar_wait_teardown(&ctl->full[it % C::ST], (it / C::ST) & 1);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    griddep_wait();   // outputs of this kernel may still be read by the previous one
+    const int cw = warp - 1, w = cw & (kRowGroups - 1), bs = cw >> 2, g = lane >> 2, t = lane & 3;
+    const int r = pair_of(w, g);   // pair row in the CTA: rows n0 + 2r (even), n0 + 2r + 1 (odd)
+    // per-thread shared-memory offsets inside a stage: 16-byte code chunk t of
+    // block bs (128-byte swizzle inside the [32 pairs][128 B] box bs / 2)
+    const uint32_t code_off = (bs >> 1) * (CODE_BYTES / 2) + r * 128 + 16 * ((4 * (bs & 1) + t) ^ (r & 7));
+    uint32_t x_off[NT][4];  // token 8 j + g, columns 16 i + 4 t .. + 3 of the [MB][64] box bs
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row = 8 * j + g;
+        x_off[j][i] = CODE_BYTES + SC_BYTES + bs * C::XBOX + row * 128 + 16 * ((2 * i + (t >> 1)) ^ (row & 7)) +
+                      8 * (t & 1);
+      }
+    // scale words of block bs: row (64 bs + 16 SPG q) >> gsl of the stage's box
+    // (stages start on multiples of 256 columns), half2 of pair r
+    uint32_t sc_off[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = 64 * bs + (SPG == 4 ? 0 : 16 * SPG * q);
+      sc_off[q] = CODE_BYTES + (uint32_t)(gs < SK ? (col >> gsl) : 0) * 128 + 4 * r;
+    }
+
+    float acc[NT][4], part[2][NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[j][c] = part[0][j][c] = part[1][j][c] = 0.f;
+    auto flush = [&](uint32_t s_word) {
+      const __half2 s2 = u32_as_h2(s_word);
+      const float se = __low2float(s2), so = __high2float(s2);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        acc[j][0] = fmaf(part[0][j][0] + part[1][j][0], se, acc[j][0]);
+        acc[j][1] = fmaf(part[0][j][1] + part[1][j][1], se, acc[j][1]);
+        acc[j][2] = fmaf(part[0][j][2] + part[1][j][2], so, acc[j][2]);
+        acc[j][3] = fmaf(part[0][j][3] + part[1][j][3], so, acc[j][3]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) part[0][j][c] = part[1][j][c] = 0.f;
+      }
+    };
+
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % C::ST;
+      if (!mbar_wait(&ctl->full[s], (it / C::ST) & 1, abort_flag, &g_device_error, 128u)) break;
+      const uint32_t st = sbase + s * C::STAGE;
+      const uint4 wv = lds128(st + code_off);
+      const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+      uint2 xv[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[j][i] = lds64(st + x_off[j][i]);
+      uint32_t sw[4];
+#pragma unroll
+      for (int q = 0; q < (SPG == 4 ? 1 : 4 / SPG); ++q) sw[q] = lds32(st + sc_off[q]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const RowPairs rp = codes_minus8_rows(words[i]);
+        const uint32_t a[4] = {h2_as_u32(rp.ev01), h2_as_u32(rp.od01), h2_as_u32(rp.ev23), h2_as_u32(rp.od23)};
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          const uint32_t bf[2] = {xv[j][i].x, xv[j][i].y};
+          mma_16816(part[i & 1][j], a, bf);
+        }
+        if (SPG == 1) flush(sw[i]);
+        if (SPG == 2 && (i & 1)) flush(sw[i >> 1]);
+      }
+      if (SPG == 4) {
+        // this warp's next block (one stage later) starts another group, or
+        // the split ends here
+        const int k0 = (st_begin + it) * SK + 64 * bs;
+        if (((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1) flush(sw[0]);
+      }
+    }
+    // D fragment: rows g (even n of pair r) and g + 8 (odd n), tokens 2t, 2t+1 of tile j
+    float* rs = red + bs * 16 * 64;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      rs[(8 * j + 2 * t) * 64 + 2 * r] = acc[j][0];
+      rs[(8 * j + 2 * t + 1) * 64 + 2 * r] = acc[j][1];
+      rs[(8 * j + 2 * t) * 64 + 2 * r + 1] = acc[j][2];
+      rs[(8 * j + 2 * t + 1) * 64 + 2 * r + 1] = acc[j][3];
+    }
+  }
+  // the four block slices, summed in order into slice 0
+  __syncthreads();
+  for (int e = threadIdx.x; e < Mz * 64; e += kThreads)
+    red[e] = ((red[e] + red[16 * 64 + e]) + red[2 * 16 * 64 + e]) + red[3 * 16 * 64 + e];
+
+  // Rank rk of the cluster sums tokens [rk Mz / S, (rk + 1) Mz / S) of the S
+  // partial tiles in rank order and stores them (64 features per token).
+  cg::cluster_group cluster = cg::this_cluster();
+  if (S > 1) cluster.sync();
+  else __syncthreads();
+  if (!*abort_flag) {
+    const int rk = S > 1 ? (int)cluster.block_rank() : 0;
+    const int tb = rk * Mz / S, te = (rk + 1) * Mz / S;
+    for (int e = threadIdx.x; e < (te - tb) * 64; e += kThreads) {
+      const int tok = tb + (e >> 6), nl = e & 63;
+      const int n = n0 + nl;
+      if (n >= N) continue;
+      float v = 0.f;
+      for (int q = 0; q < S; ++q) v += (q == rk ? red : cluster.map_shared_rank(red, q))[tok * 64 + nl];
+      const size_t m = (size_t)(tok0 + tok);
+      if (n < out.n1) out.y0[m * out.n1 + n] = v;
+      else if (n < out.n2) out.y1[m * (out.n2 - out.n1) + (n - out.n1)] = v;
+      else out.y2[m * (out.N - out.n2) + (n - out.n2)] = v;
+    }
+  }
+  if (S > 1) cluster.sync();
+}
+
+}  // namespace gv
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+template <int NT, int SPG>
+static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUtensorMap& map_sc,
+                                           const CUtensorMap& map_x, OutSplit out, int M, int N, int K, int gs,
+                                           int stages_total, dim3 grid, cudaStream_t stream) {
+  using C = gv::Cfg<NT>;
+  auto kern = gv::gemv_fwd_tma_kernel<NT, SPG>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int d = (dev >= 0 && dev < 64) ? dev : 0;
+  if (!attr_done[d]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+    if (e != cudaSuccess) return e;
+    if (grid.y > 8) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    attr_done[d] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(gv::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = grid.y;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, map_x, out, M, N, K, gs, stages_total);
+}
+
+cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
+                                cudaStream_t stream, char* route, int route_len) {
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  const Layout L = layout_of(N, K, gs);
+  const int G = K / gs;
+  const int NT = (M <= 8) ? 1 : 2;
+  const int zs = (M + 15) / 16;
+  const int tiles = (N + 63) / 64;
+  const int stages_total = (K + gv::SK - 1) / gv::SK;
+  // fill the resident CTA slots in one wave, at least two stages per split,
+  // clusters of at most 8
+  int sms = 148;
+  {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int slots = sms * (NT == 1 ? gv::Cfg<1>::kCtasPerSm : gv::Cfg<2>::kCtasPerSm);
+  int S = slots / (tiles * zs);
+  S = S < 1 ? 1 : (S > 8 ? 8 : S);
+  while (S > 1 && stages_total / S < 2) --S;
+  const int sc_rows = gs < gv::SK ? gv::SK / gs : 1;
+  CUtensorMap map_pk, map_sc, map_x;
+  const bool ok =
+      make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, gv::RP, CU_TENSOR_MAP_SWIZZLE_128B) &&
+      make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pk + L.scales_offset, N, G, (uint64_t)N * 2, 64, sc_rows,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, (uint64_t)K * 2, 64, 8 * NT,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  const int spg = gs == 16 ? 1 : gs == 32 ? 2 : 4;
+  const dim3 grid(tiles, S, zs);
+  cudaError_t e;
+  if (NT == 1)
+    e = spg == 1 ? launch_gemv_tma_variant<1, 1>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
+      : spg == 2 ? launch_gemv_tma_variant<1, 2>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
+                 : launch_gemv_tma_variant<1, 4>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream);
+  else
+    e = spg == 1 ? launch_gemv_tma_variant<2, 1>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
+      : spg == 2 ? launch_gemv_tma_variant<2, 2>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
+                 : launch_gemv_tma_variant<2, 4>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream);
+  if (route)
+    snprintf(route, route_len, "gemv_tma_fwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S,
+             zs, stages_total);
+  return e;
+}
+
+}  // namespace q4gsw
