@@ -484,6 +484,11 @@ cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint
 
 cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M,
                             float* d_x, cudaStream_t stream, char* route, int route_len) {
+  {
+    const char* e = getenv("Q4GSW_GEMV_KIND");
+    const bool reg = e && e[0] == 'r' && e[1] == 'e' && e[2] == 'g' && e[3] == 0;
+    if (!reg) return launch_gemv_tma_bwd(packed, N, K, gs, d_out, M, d_x, stream, route, route_len);
+  }
   const int tiles = (K + 127) / 128;
   const int zs = (M + 15) / 16;
   const int NT = (M <= 8) ? 1 : 2;

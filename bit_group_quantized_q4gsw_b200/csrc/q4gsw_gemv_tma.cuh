@@ -1,5 +1,6 @@
-// q4gsw_gemv_tma.cuh - forward GEMV route for small token counts (M <= 16 per
-// z-slice) that streams the packed weight through a TMA ring (sm_100a).
+// q4gsw_gemv_tma.cuh - GEMV routes for small token counts (M <= 16 per
+// z-slice) that stream the packed weight through a TMA ring (sm_100a):
+// forward and input gradient.
 // Included once, by q4gsw_gemm_sm100.cu, which owns the device error word and
 // the tensor-map helpers.
 //
@@ -282,6 +283,237 @@ gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_con
   if (S > 1) cluster.sync();
 }
 
+
+// ---------------------------------------------------------------------------
+// Input gradient: d_x[m, k] = sum_n d_out[m, n] (code[n, k] - 8) s[k / gs, n]
+// ---------------------------------------------------------------------------
+// MMA roles as in the register-fed kernel: A = weight^T tile (16 output
+// columns k x 16 contraction rows n = 8 nibble pairs; a register holds the
+// (even n, odd n) half2 of one byte, scaled per element), B = d_out^T (16 n x
+// 8 tokens).  A CTA owns 128 output columns (two 64-byte blocks) and streams
+// stages of 64 nibble pairs (128 contraction rows): codes [64 pairs][128 B]
+// (128-byte swizzle), d_out [MB tokens][2 x 64 n] and the scale rows of the
+// CTA's column groups for those 128 n.  Consumer warp c takes the 8 pairs
+// 8c .. 8c + 7 of every stage; lane (g, t) reads 16 bytes at chunk g & 3 of
+// block g >> 2 in pair rows 8c + t and 8c + t + 4, i.e. columns
+// 64 (g >> 2) + 16 i + 4 (g & 3) + e; MMA q = 2 i + h maps A row g to e = 2h
+// and row g + 8 to e = 2h + 1.
+constexpr int kBwdConsumers = 8;
+constexpr int kBwdThreads = 32 * (1 + kBwdConsumers);
+constexpr int BWD_CODE_BYTES = 64 * 128;   // 64 pairs x 128 columns
+constexpr int BWD_SC_BYTES = 8 * 256;      // up to 8 scale rows of 128 n
+
+template <int NT>
+struct BwdCfg {
+  static constexpr int MB = 8 * NT;
+  static constexpr int DBOX = MB * 128 < 1024 ? 1024 : MB * 128;   // one [MB][64 n] box
+  static constexpr int STAGE = BWD_CODE_BYTES + BWD_SC_BYTES + 2 * DBOX;
+  static constexpr int ST = NT == 1 ? 8 : 7;
+  static constexpr int OFF_CTL = ST * STAGE;
+  static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
+  static constexpr int RED_FLOATS = kBwdConsumers * MB * 128;   // warp partials, reuse the ring
+  static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
+  static_assert(RED_FLOATS * 4 + MB * 128 * 4 <= OFF_CTL, "reduction fits in the ring");
+  static_assert(BYTES <= 113 * 1024, "two CTAs per SM");
+};
+
+template <int NT, int SPB>  // SPB scale groups per 64-column block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
+__global__ void __launch_bounds__(kBwdThreads, 2)
+gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
+                    const __grid_constant__ CUtensorMap map_d, float* __restrict__ dx, int M, int N, int K,
+                    int gs, int stages_total) {
+  using namespace sm100;
+  using C = BwdCfg<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
+  volatile int* abort_flag = &ctl->abort;
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.y, S = gridDim.y;
+  const int tok0 = blockIdx.z * 16;
+  const int Mz = min(16, M - tok0);
+  const int kbase = 128 * blockIdx.x;
+  const int st_begin = (int)((long long)split * stages_total / S);
+  const int st_end = (int)((long long)(split + 1) * stages_total / S);
+  const int nit = st_end - st_begin;
+  const int gsl = __ffs(gs) - 1;
+  const int sc_rows = gs < 128 ? 128 / gs : 1;
+
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::ST; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], kBwdConsumers);
+    }
+    ctl->abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&map_pk);
+    prefetch_tmap(&map_sc);
+    prefetch_tmap(&map_d);
+  }
+  __syncthreads();
+  const uint32_t tx = BWD_CODE_BYTES + sc_rows * 256 + 2 * C::MB * 128;
+
+  float acc[NT][8][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[j][q][c] = 0.f;
+  const int g = lane >> 2, t = lane & 3;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      auto load_weights = [&](int it) {
+        const int s = it % C::ST;
+        const int n0 = (st_begin + it) * 128;
+        uint8_t* st = smem + s * C::STAGE;
+        tma_load_2d(st, &map_pk, &ctl->full[s], kbase, n0 / 2);
+        tma_load_2d(st + BWD_CODE_BYTES, &map_sc, &ctl->full[s], n0, kbase >> gsl);
+      };
+      auto load_d = [&](int it) {
+        const int s = it % C::ST;
+        const int n0 = (st_begin + it) * 128;
+        uint8_t* ds = smem + s * C::STAGE + BWD_CODE_BYTES + BWD_SC_BYTES;
+        tma_load_2d(ds, &map_d, &ctl->full[s], n0, tok0);
+        tma_load_2d(ds + C::DBOX, &map_d, &ctl->full[s], n0 + 64, tok0);
+      };
+      const int pre = nit < C::ST ? nit : C::ST;
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&ctl->full[it], tx);
+        load_weights(it);
+      }
+      griddep_wait();   // d_out may come from the previous kernel of the stream
+      for (int it = 0; it < pre; ++it) load_d(it);
+      int issued = pre;
+      for (int it = pre; it < nit; ++it) {
+        const int s = it % C::ST;
+        if (!mbar_wait(&ctl->empty[s], ((it / C::ST) - 1) & 1, abort_flag, &g_device_error, 64u)) break;
+        mbar_arrive_expect_tx(&ctl->full[s], tx);
+        load_weights(it);
+        load_d(it);
+        issued = it + 1;
+      }
+      for (int it = (issued > C::ST ? issued - C::ST : 0); it < issued; ++it)
+        mbar_wait_teardown(&ctl->full[it % C::ST], (it / C::ST) & 1);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    griddep_wait();   // outputs may still be read by the previous kernel
+    const int c = warp - 1;
+    const int rowA = 8 * c + t, rowB = rowA + 4;   // pair rows of the stage
+    const int J = g >> 2;                          // 64-column block of this lane
+    const uint32_t offA = rowA * 128 + 16 * ((4 * J + (g & 3)) ^ (rowA & 7));
+    const uint32_t offB = rowB * 128 + 16 * ((4 * J + (g & 3)) ^ (rowB & 7));
+    // d_out words (n = 2 rowA, 2 rowA + 1) and (2 rowB, 2 rowB + 1) of token 8 j + g
+    uint32_t dA[NT], dB[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int row = 8 * j + g;
+      const int nA = 2 * rowA, nB = 2 * rowB;      // 0..127 within the stage
+      dA[j] = BWD_CODE_BYTES + BWD_SC_BYTES + (nA >> 6) * C::DBOX + row * 128 +
+              16 * ((((nA & 63) * 2) >> 4) ^ (row & 7)) + (((nA & 63) * 2) & 15);
+      dB[j] = BWD_CODE_BYTES + BWD_SC_BYTES + (nB >> 6) * C::DBOX + row * 128 +
+              16 * ((((nB & 63) * 2) >> 4) ^ (row & 7)) + (((nB & 63) * 2) & 15);
+    }
+    // scale half2 of pairs rowA / rowB in the row of each column group
+    uint32_t scA[SPB], scB[SPB];
+#pragma unroll
+    for (int q = 0; q < SPB; ++q) {
+      const int col = 64 * J + 16 * (q * (4 / SPB)) + 4 * (g & 3);
+      const int r = ((kbase + col) >> gsl) - (kbase >> gsl);
+      scA[q] = BWD_CODE_BYTES + r * 256 + 4 * rowA;
+      scB[q] = BWD_CODE_BYTES + r * 256 + 4 * rowB;
+    }
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % C::ST;
+      if (!mbar_wait(&ctl->full[s], (it / C::ST) & 1, abort_flag, &g_device_error, 128u)) break;
+      const uint32_t st = sbase + s * C::STAGE;
+      const uint4 va = lds128(st + offA), vb = lds128(st + offB);
+      uint32_t bfr[NT][2];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        bfr[j][0] = lds32(st + dA[j]);
+        bfr[j][1] = lds32(st + dB[j]);
+      }
+      uint32_t sa[SPB], sb[SPB];
+#pragma unroll
+      for (int q = 0; q < SPB; ++q) {
+        sa[q] = lds32(st + scA[q]);
+        sb[q] = lds32(st + scB[q]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
+      const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+      const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = i / (4 / SPB);
+        const __half2 hsa = u32_as_h2(sa[q]), hsb = u32_as_h2(sb[q]);
+        const ColPairs ca = codes_minus8_cols(wa[i]);
+        const ColPairs cb = codes_minus8_cols(wb[i]);
+        const __half2 la[4] = {ca.c0, ca.c1, ca.c2, ca.c3};
+        const __half2 lb[4] = {cb.c0, cb.c1, cb.c2, cb.c3};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t af[4] = {h2_as_u32(__hmul2(la[2 * h], hsa)), h2_as_u32(__hmul2(la[2 * h + 1], hsa)),
+                                  h2_as_u32(__hmul2(lb[2 * h], hsb)), h2_as_u32(__hmul2(lb[2 * h + 1], hsb))};
+#pragma unroll
+          for (int j = 0; j < NT; ++j) mma_16816(acc[j][2 * i + h], af, bfr[j]);
+        }
+      }
+    }
+  }
+
+  // Warp partials (into the idle ring), summed over the warps in order, then
+  // over the cluster in rank order.
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(smem);                 // [consumer][MB tokens][128 columns]
+  float* cta_part = red + C::RED_FLOATS;                       // [MB tokens][128 columns]
+  if (warp > 0) {
+    float* mine = red + (warp - 1) * (C::MB * 128);
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int i = q >> 1, h = q & 1;
+        const int kl = 64 * (g >> 2) + 16 * i + 4 * (g & 3) + 2 * h;
+        const int tk = 8 * j + 2 * t;
+        mine[tk * 128 + kl] = acc[j][q][0];
+        mine[(tk + 1) * 128 + kl] = acc[j][q][1];
+        mine[tk * 128 + kl + 1] = acc[j][q][2];
+        mine[(tk + 1) * 128 + kl + 1] = acc[j][q][3];
+      }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < Mz * 128; idx += kBwdThreads) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kBwdConsumers; ++w) v += red[w * (C::MB * 128) + idx];
+    cta_part[idx] = v;
+  }
+  cg::cluster_group cluster = cg::this_cluster();
+  if (S > 1) cluster.sync();
+  else __syncthreads();
+  if (!*abort_flag) {
+    const int rk = S > 1 ? (int)cluster.block_rank() : 0;
+    const int tb = rk * Mz / S, te = (rk + 1) * Mz / S;
+    const int kw = min(128, K - kbase);
+    for (int e = tb * 128 + threadIdx.x; e < te * 128; e += kBwdThreads) {
+      const int tok = e >> 7, kl = e & 127;
+      if (kl >= kw) continue;
+      float v = 0.f;
+      for (int q = 0; q < S; ++q) v += (q == rk ? cta_part : cluster.map_shared_rank(cta_part, q))[e];
+      dx[(size_t)(tok0 + tok) * K + kbase + kl] = v;
+    }
+  }
+  if (S > 1) cluster.sync();
+}
+
 }  // namespace gv
 
 // ---------------------------------------------------------------------------
@@ -366,6 +598,70 @@ cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, const 
                  : launch_gemv_tma_variant<2, 4>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream);
   if (route)
     snprintf(route, route_len, "gemv_tma_fwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S,
+             zs, stages_total);
+  return e;
+}
+
+cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
+                                cudaStream_t stream, char* route, int route_len) {
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  const Layout L = layout_of(N, K, gs);
+  const int G = K / gs;
+  const int NT = (M <= 8) ? 1 : 2;
+  const int zs = (M + 15) / 16;
+  const int tiles = (K + 127) / 128;
+  const int stages_total = (N + 127) / 128;
+  int sms = 148;
+  {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  // fill the two resident CTA slots per SM, at least two stages per split
+  int S = 2 * sms / (tiles * zs);
+  S = S < 1 ? 1 : (S > 8 ? 8 : S);
+  while (S > 1 && stages_total / S < 2) --S;
+  const int sc_rows = gs < 128 ? 128 / gs : 1;
+  CUtensorMap map_pk, map_sc, map_d;
+  const bool ok =
+      make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+      make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pk + L.scales_offset, N, G, (uint64_t)N * 2, 128,
+                  sc_rows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_map_2d(&map_d, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d_out, N, M, (uint64_t)N * 2, 64, 8 * NT,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  const int spb = gs >= 64 ? 1 : gs == 32 ? 2 : 4;
+  const dim3 grid(tiles, S, zs);
+  auto launch = [&](auto kern, int smem) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(gv::kBwdThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = S;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, map_d, d_x, M, N, K, gs, stages_total);
+  };
+  cudaError_t e;
+  if (NT == 1)
+    e = spb == 1 ? launch(gv::gemv_bwd_tma_kernel<1, 1>, gv::BwdCfg<1>::BYTES)
+      : spb == 2 ? launch(gv::gemv_bwd_tma_kernel<1, 2>, gv::BwdCfg<1>::BYTES)
+                 : launch(gv::gemv_bwd_tma_kernel<1, 4>, gv::BwdCfg<1>::BYTES);
+  else
+    e = spb == 1 ? launch(gv::gemv_bwd_tma_kernel<2, 1>, gv::BwdCfg<2>::BYTES)
+      : spb == 2 ? launch(gv::gemv_bwd_tma_kernel<2, 2>, gv::BwdCfg<2>::BYTES)
+                 : launch(gv::gemv_bwd_tma_kernel<2, 4>, gv::BwdCfg<2>::BYTES);
+  if (route)
+    snprintf(route, route_len, "gemv_tma_bwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S,
              zs, stages_total);
   return e;
 }

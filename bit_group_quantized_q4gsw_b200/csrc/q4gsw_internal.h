@@ -36,6 +36,8 @@ cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint
 // per z-slice).
 cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
                                 cudaStream_t stream, char* route, int route_len);
+cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
+                                cudaStream_t stream, char* route, int route_len);
 
 // tcgen05 GEMM routes (any M >= 1; used above the GEMV range).
 cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,

@@ -216,15 +216,21 @@ def gemv_variant(request, monkeypatch):
 
 @pytest.mark.parametrize("M,N,K,gs", [(1, 64, 128, 32), (3, 136, 320, 16), (8, 1032, 576, 64), (9, 72, 256, 128),
                                       (16, 264, 1344, 32), (5, 8, 64, 64), (2, 4096, 2048, 256)])
-def test_gemv_forward_routes(M, N, K, gs, gemv_variant):
+def test_gemv_routes(M, N, K, gs, gemv_variant):
     inp = wl.random_inputs(M, N, K, gs, seed=3 * M + N + K)
     check_fwd(inp, gs)
     route = q().q4gsw_last_route()
     assert route.startswith("gemv_tma_fwd" if gemv_variant == "tma" else "gemv_fwd"), route
+    check_bwd(inp, gs)
+    route = q().q4gsw_last_route()
+    assert route.startswith("gemv_tma_bwd" if gemv_variant == "tma" else "gemv_bwd"), route
     inp = wl.integer_exact_inputs(M, N, K, gs, seed=M + 1)
     y, _ = run_fwd(inp, gs)
     ref, _ = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), gs)
     assert np.array_equal(y.astype(np.float64), ref)
+    dx, _ = run_bwd(inp, gs)
+    ref, _ = o.linear_bwd_input(bits(inp.d_out), inp.codes, bits(inp.scales), gs)
+    assert np.array_equal(dx.astype(np.float64), ref)
 
 
 def test_non_default_stream():
