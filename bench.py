@@ -49,7 +49,7 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
 # dram__bytes_write.sum; profiles/gemm_*.md), with the hash of the kernel
 # sources they were taken on: reported only while the sources still match.
-NCU_TRAFFIC = {"sources_sha": "aac3f012669ed01e", "bytes_per_launch": {'up_fwd': 11561216, 'up_bwd': 17852672, 'down_fwd': 17852416, 'down_bwd': 11560960, 'qkv_fwd': 5662976}}
+NCU_TRAFFIC = {"sources_sha": "06952cb3aa239747", "bytes_per_launch": {'up_fwd': 11560960, 'up_bwd': 17852416, 'down_fwd': 17852672, 'down_bwd': 11560960, 'qkv_fwd': 5662720}}
 
 
 def sources_sha() -> str:
