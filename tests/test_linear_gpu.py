@@ -215,7 +215,8 @@ def gemv_variant(request, monkeypatch):
 
 
 @pytest.mark.parametrize("M,N,K,gs", [(1, 64, 128, 32), (3, 136, 320, 16), (8, 1032, 576, 64), (9, 72, 256, 128),
-                                      (16, 264, 1344, 32), (5, 8, 64, 64), (2, 4096, 2048, 256)])
+                                      (16, 264, 1344, 32), (5, 8, 64, 64), (2, 4096, 2048, 256),
+                                      (1, 128, 2048, 512), (12, 200, 4096, 1024), (7, 392, 3008, 64)])
 def test_gemv_routes(M, N, K, gs, gemv_variant):
     inp = wl.random_inputs(M, N, K, gs, seed=3 * M + N + K)
     check_fwd(inp, gs)
