@@ -431,43 +431,77 @@ def run_gpu(args, rank, world, local_rank):
         src = inputs[name].d_out if kind == "bwd" else inputs[name].x
         host_in[name] = torch.from_numpy(src).pin_memory()
     host_out = {name: [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in gs.outs[name]] for name, _, _ in ops}
-    dev_in = {name: torch.empty(host_in[name].shape, dtype=torch.float16, device=device) for name, _, _ in ops}
+    # Three streams, device inputs and outputs double-buffered: the copy-in of
+    # step i+1 and the copy-out of step i-1 overlap the launches of step i.
+    # Every step still copies all of its inputs in and all of its outputs out.
+    dev_in = [{name: torch.empty(host_in[name].shape, dtype=torch.float16, device=device) for name, _, _ in ops}
+              for _ in range(2)]
+    dev_out = [gs.outs, {name: [torch.empty_like(t) for t in v] for name, v in gs.outs.items()}]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for v in host_out.values() for t in v)
     e2e_steps = max(1, min(args.steps, 50))
+    s_comp = torch.cuda.current_stream(device)
+    s_h2d = torch.cuda.Stream(device)
+    s_d2h = torch.cuda.Stream(device)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_copied = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):
+        comp_done[b].record(s_comp)
+        out_copied[b].record(s_comp)
 
-    def e2e_step(c):
-        for name, kind, sh in ops:
-            dev_in[name].copy_(host_in[name], non_blocking=True)
-        for name, kind, sh in ops:
-            pk = gs.packed[sh.name][c]
-            o = gs.outs[name]
-            if kind == "qkv":
-                Nq, Nk, Nv = sh.splits
-                q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, dev_in[name], outs=o)
-            elif kind == "fwd":
-                q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, dev_in[name], y=o[0])
-            else:
-                q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, dev_in[name], d_x=o[0])
-        for name, _, _ in ops:
-            for hb, db in zip(host_out[name], gs.outs[name]):
-                hb.copy_(db, non_blocking=True)
+    def e2e_step(i, c):
+        b = i & 1
+        s_h2d.wait_event(comp_done[b])          # step i-2 no longer reads dev_in[b]
+        with torch.cuda.stream(s_h2d):
+            for name, _, _ in ops:
+                dev_in[b][name].copy_(host_in[name], non_blocking=True)
+            in_ready[b].record(s_h2d)
+        s_comp.wait_event(in_ready[b])
+        s_comp.wait_event(out_copied[b])        # step i-2's outputs have reached the host
+        with torch.cuda.stream(s_comp):
+            for name, kind, sh in ops:
+                pk = gs.packed[sh.name][c]
+                o = dev_out[b][name]
+                xin = dev_in[b][name]
+                if kind == "qkv":
+                    Nq, Nk, Nv = sh.splits
+                    q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, xin, outs=o)
+                elif kind == "fwd":
+                    q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, xin, y=o[0])
+                else:
+                    q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, xin, d_x=o[0])
+            comp_done[b].record(s_comp)
+        s_d2h.wait_event(comp_done[b])
+        with torch.cuda.stream(s_d2h):
+            for name, _, _ in ops:
+                for hb, db in zip(host_out[name], dev_out[b][name]):
+                    hb.copy_(db, non_blocking=True)
+            out_copied[b].record(s_d2h)
 
     for i in range(min(args.warmup, 3)):
-        e2e_step(i % copies)
+        e2e_step(i, i % copies)
     torch.cuda.synchronize(device)
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
+    start = torch.cuda.Event()
+    e0.record(s_comp)
+    start.record(s_comp)
+    s_h2d.wait_event(start)
+    s_d2h.wait_event(start)
     for i in range(e2e_steps):
-        e2e_step(i % copies)
-    e1.record()
+        e2e_step(i, i % copies)
+    s_comp.wait_event(out_copied[0])
+    s_comp.wait_event(out_copied[1])
+    e1.record(s_comp)
     torch.cuda.synchronize(device)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     e2e = {"value": job_throughput(world, flops_step, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+           "overlap": "copy-in of step i+1 and copy-out of step i-1 run on their own streams beside the "
+                      "launches of step i (device buffers double-buffered)"}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
