@@ -49,7 +49,7 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
 # dram__bytes_write.sum; profiles/gemm_*.md), with the hash of the kernel
 # sources they were taken on: reported only while the sources still match.
-NCU_TRAFFIC = {"sources_sha": "06952cb3aa239747", "bytes_per_launch": {'up_fwd': 11560960, 'up_bwd': 17852416, 'down_fwd': 17852672, 'down_bwd': 11560960, 'qkv_fwd': 5662720}}
+NCU_TRAFFIC = {"sources_sha": "ed63c1fc9c001ed9", "bytes_per_launch": {'up_fwd': 11561472, 'up_bwd': 17852672, 'down_fwd': 17852928, 'down_bwd': 11561216, 'qkv_fwd': 5662976}}
 
 
 def sources_sha() -> str:
@@ -79,12 +79,18 @@ def step_ops():
 
 def op_flops(kind, sh, M=None):
     M = sh.M if M is None else M
+    if kind == "emb":
+        return float(M * sh.K)          # one multiply per gathered element
     return 2.0 * M * sh.N * sh.K
 
 
 def op_bytes(kind, sh, M=None):
     """Algorithmic bytes: packed codes + scales once, activations in, fp32 out."""
     M = sh.M if M is None else M
+    if kind == "emb":
+        # per gathered row: its nibble-pair row (K bytes, the row shares them
+        # with its pair), its K/gs fp16 scales, K fp32 outputs; the 4-byte id
+        return M * (sh.K + 2 * (sh.K // sh.group_size) + 4 * sh.K + 4)
     w = sh.N * sh.K // 2 + 2 * (sh.K // sh.group_size) * sh.N
     if kind == "bwd":
         return w + 2 * M * sh.N + 4 * M * sh.K
@@ -529,7 +535,7 @@ def run_sweep(args):
     import bit_group_quantized_q4gsw_b200 as q
     device = torch.device("cuda", 0)
     peaks = measured_peaks()
-    shapes = wl.tiny() + wl.decode() + wl.qkv() + wl.adapter() + wl.sweep()
+    shapes = wl.tiny() + wl.decode() + wl.qkv() + wl.adapter() + wl.sweep() + wl.embedding()
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     if args.only:
         import re
@@ -554,6 +560,10 @@ def run_sweep(args):
             elif kind == "fwd":
                 y = torch.empty((sh.M, sh.N), dtype=torch.float32, device=device)
                 fn = lambda pk: q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a, y=y)
+            elif kind == "emb":
+                ids = torch.from_numpy(wl.embedding_indices(sh)).to(device)
+                y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
+                fn = lambda pk: q.q4gsw_embedding(pk, sh.N, sh.K, sh.group_size, ids, out=y)
             else:
                 y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
                 fn = lambda pk: q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a, d_x=y)
@@ -620,6 +630,8 @@ def run_case(args):
             q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, a)
         elif kind == "fwd":
             q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a)
+        elif kind == "emb":
+            q.q4gsw_embedding(pk, sh.N, sh.K, sh.group_size, torch.from_numpy(wl.embedding_indices(sh, M)).to(device))
         else:
             q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a)
     torch.cuda.synchronize()

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libq4gsw.so")
 Q4GSW_OK = 0
 STATUS_NAMES = {0: "Q4GSW_OK", 1: "Q4GSW_ERR_NULL", 2: "Q4GSW_ERR_SHAPE", 3: "Q4GSW_ERR_ALIGN",
                 4: "Q4GSW_ERR_UNSUPPORTED", 5: "Q4GSW_ERR_CODE_RANGE", 6: "Q4GSW_ERR_CUDA",
-                7: "Q4GSW_ERR_SIZE", 8: "Q4GSW_ERR_TIMEOUT"}
+                7: "Q4GSW_ERR_SIZE", 8: "Q4GSW_ERR_TIMEOUT", 9: "Q4GSW_ERR_INDEX"}
 
 # (name, restype, argtypes) of every function declared in include/q4gsw.h
 _VP, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -32,6 +32,7 @@ SIGNATURES = [
     ("q4gsw_linear_fwd", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
     ("q4gsw_linear_bwd_input", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
     ("q4gsw_qkv_fwd", _I, [_VP, _I, _I, _I, _I, _I, _VP, _I, _VP, _VP, _VP, _VP]),
+    ("q4gsw_embedding", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
     ("q4gsw_device_error_check", _I, [_VP]),
     ("q4gsw_unpack", _I, [_VP, _I, _I, _I, _VP, _VP]),
     ("q4gsw_dequant", _I, [_VP, _I, _I, _I, _VP, _VP, _VP]),
@@ -166,8 +167,22 @@ def q4gsw_qkv_fwd(packed_qkv: torch.Tensor, Nq: int, Nk: int, Nv: int, K: int, g
     return yq, yk, yv
 
 
+def q4gsw_embedding(packed: torch.Tensor, N: int, K: int, group_size: int, indices: torch.Tensor,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """out[T, K] = dequant(W)[indices] in fp32 (indices int32 [T] on the device, each in [0, N))."""
+    T = indices.shape[0]
+    if out is None:
+        out = torch.empty((T, K), dtype=torch.float32, device=indices.device)
+    st = library().q4gsw_embedding(_dev(packed, torch.uint8, "packed"), N, K, group_size,
+                                   _dev(indices, torch.int32, "indices", 1), T,
+                                   _dev(out, torch.float32, "out", 2), _stream(indices))
+    _check("q4gsw_embedding", st)
+    return out
+
+
 def q4gsw_device_error_check(device=None) -> None:
-    """Raise Q4gswError(Q4GSW_ERR_TIMEOUT) if a kernel wait ran out since the last check."""
+    """Raise Q4gswError if a kernel wait ran out (Q4GSW_ERR_TIMEOUT) or an embedding
+    index was out of range (Q4GSW_ERR_INDEX) since the last check."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     st = library().q4gsw_device_error_check(torch.cuda.current_stream(dev).cuda_stream)
     _check("q4gsw_device_error_check", st)

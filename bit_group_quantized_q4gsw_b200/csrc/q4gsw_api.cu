@@ -72,6 +72,7 @@ const char* q4gsw_status_str(q4gsw_status s) {
     case Q4GSW_ERR_CUDA: return "CUDA runtime error";
     case Q4GSW_ERR_SIZE: return "buffer too small";
     case Q4GSW_ERR_TIMEOUT: return "a kernel wait ran out (results of the calls since the last check are invalid)";
+    case Q4GSW_ERR_INDEX: return "an embedding index was outside [0, N) (its row was written as zeros)";
   }
   return "unknown status";
 }
@@ -152,7 +153,23 @@ q4gsw_status q4gsw_device_error_check(q4gsw_stream_t stream) {
   unsigned int v = 0;
   q4gsw_status st = from_cuda(read_and_clear_device_error(stream, &v));
   if (st != Q4GSW_OK) return st;
-  return v ? Q4GSW_ERR_TIMEOUT : Q4GSW_OK;
+  if (v & ~0x100u) return Q4GSW_ERR_TIMEOUT;   // bit 8: embedding index range, every other bit: a wait ran out
+  return v ? Q4GSW_ERR_INDEX : Q4GSW_OK;
+}
+
+q4gsw_status q4gsw_embedding(const void* packed, int N, int K, int group_size, const int32_t* indices, int T,
+                             float* out, q4gsw_stream_t stream) {
+  if (T < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (T == 0) {
+    set_route("empty");
+    return Q4GSW_OK;
+  }
+  if (!packed || !indices || !out) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(out) || (reinterpret_cast<uintptr_t>(indices) & 3u)) return Q4GSW_ERR_ALIGN;
+  set_route("embedding_gather launches=1");
+  return from_cuda(launch_embedding(packed, N, K, group_size, indices, T, out, stream));
 }
 
 q4gsw_status q4gsw_unpack(const void* packed, int N, int K, int group_size, uint8_t* codes,

@@ -590,6 +590,7 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
 
 }  // namespace q4gsw
 
+#include "q4gsw_embedding.cuh"
 #include "q4gsw_gemm_ts.cuh"
 #include "q4gsw_gemv_tma.cuh"
 

@@ -45,8 +45,13 @@ cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, const uint
 cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
                             cudaStream_t stream, char* route, int route_len);
 
+// Embedding rows out[t] = dequant(W)[indices[t]] (fp32); an index outside
+// [0, N) gives a zero row and sets kIndexErrorBit in the device error word.
+cudaError_t launch_embedding(const void* packed, int N, int K, int gs, const int32_t* indices, int T, float* out,
+                             cudaStream_t stream);
+
 // Reads (and clears when set) the device word in which kernels record waits
-// that ran out; synchronises `stream`.
+// that ran out (and embedding indices out of range); synchronises `stream`.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int* host_value);
 
 }  // namespace q4gsw

@@ -80,8 +80,22 @@ def sweep():
     return out
 
 
+def embedding():
+    """Embedding gathers from a 1B-class table (vocabulary 32000 x 2048 features,
+    gs 32): one decode token, a 512-token prompt and a 16384-token batch.  The
+    token ids come from ``embedding_indices``."""
+    return [Shape(f"embedding_T{T}_V32000_D2048", T, 32000, 2048, 32, seed=600 + i, directions=("emb",))
+            for i, T in enumerate((1, 512, 16384))]
+
+
+def embedding_indices(shape: Shape, T: int | None = None) -> np.ndarray:
+    """Seeded token ids, int32 [T], uniform over the table's N rows (repeats allowed)."""
+    T = shape.M if T is None else T
+    return np.random.default_rng(shape.seed + 10_000).integers(0, shape.N, T, dtype=np.int32)
+
+
 def all_shapes():
-    return tiny() + decode() + qkv() + adapter() + sweep()
+    return tiny() + decode() + qkv() + adapter() + sweep() + embedding()
 
 
 def by_name(name: str) -> Shape:

@@ -78,7 +78,8 @@ typedef enum {
   Q4GSW_ERR_CODE_RANGE = 5,   /* q4gsw_prepack saw a code > 15 */
   Q4GSW_ERR_CUDA = 6,         /* the CUDA runtime reported an error */
   Q4GSW_ERR_SIZE = 7,         /* a byte count passed in is too small */
-  Q4GSW_ERR_TIMEOUT = 8       /* a kernel's bounded wait ran out (q4gsw_device_error_check) */
+  Q4GSW_ERR_TIMEOUT = 8,      /* a kernel's bounded wait ran out (q4gsw_device_error_check) */
+  Q4GSW_ERR_INDEX = 9         /* q4gsw_embedding saw an index outside [0, N) (q4gsw_device_error_check) */
 } q4gsw_status;
 
 /* Version of the packed-weight byte layout written by q4gsw_prepack. */
@@ -116,8 +117,10 @@ Q4GSW_API q4gsw_status q4gsw_prepack(const uint8_t *codes, const uint16_t *scale
  * Forward: y[m,n] = sum_k x[m,k] * w[n,k], fp32 accumulation.
  *   packed  a blob from q4gsw_prepack for the same (N, K, gs)
  *   x       fp16 [M, K];   y  fp32 [M, N] (overwritten)
- * Route: M <= 16 a tensor-core GEMV over the streamed packed weight; larger M
- * a tcgen05 GEMM that dequantises into shared memory (q4gsw_last_route()).
+ * Route (q4gsw_last_route()): M <= 16 a tensor-core GEMV over the streamed
+ * packed weight; 16 < M <= 512 a tcgen05 GEMM whose weight tile is
+ * dequantised into tensor memory; larger M a tcgen05 GEMM that dequantises
+ * into shared memory.
  */
 Q4GSW_API q4gsw_status q4gsw_linear_fwd(const void *packed, int N, int K, int group_size,
                               const uint16_t *x, int M, float *y,
@@ -146,12 +149,31 @@ Q4GSW_API q4gsw_status q4gsw_qkv_fwd(const void *packed_qkv, int Nq, int Nk, int
                            q4gsw_stream_t stream);
 
 /*
+ * Embedding rows gathered from a packed q4gsw weight used as a table of N
+ * rows of K features ("[ExecuTorch][WebGPU] Replace broad QKV fusion with
+ * BK64 kernel", description of #21483: the Q4 embedding reads the linear
+ * weight's nibble layout, is_linear_weight):
+ *   out[t, k] = (code[idx[t], k] - 8) * s[k / gs, idx[t]]   for t < T, k < K,
+ * each element the exact fp32 product (as q4gsw_dequant's w32).
+ *   packed   a blob from q4gsw_prepack for (N, K, gs)
+ *   indices  int32 [T] on the device, each in [0, N)
+ *   out      fp32 [T, K] (overwritten)
+ * T = 0 enqueues nothing.  An index outside [0, N) cannot be seen on the host:
+ * its row is written as zeros and q4gsw_device_error_check then returns
+ * Q4GSW_ERR_INDEX.
+ */
+Q4GSW_API q4gsw_status q4gsw_embedding(const void *packed, int N, int K, int group_size,
+                             const int32_t *indices, int T, float *out,
+                             q4gsw_stream_t stream);
+
+/*
  * Kernel health check.  Every wait inside this library's kernels is bounded
  * (about one second); a wait that runs out makes its kernel stop early and
  * record the event in a device-side status word instead of hanging.  This call
  * waits for `stream`, reads that word for the current device and clears it:
  * Q4GSW_ERR_TIMEOUT means the outputs of the calls since the previous check are
- * not valid.  Returns Q4GSW_OK otherwise.
+ * not valid; Q4GSW_ERR_INDEX that an embedding index was out of range (a
+ * timeout takes precedence).  Returns Q4GSW_OK otherwise.
  */
 Q4GSW_API q4gsw_status q4gsw_device_error_check(q4gsw_stream_t stream);
 

@@ -303,6 +303,28 @@ def dequant_w16_bits_fast(codes: np.ndarray, scale_bits: np.ndarray, group_size:
 # ----------------------------------------------------------------------------
 # The three products.  Accumulation is in float64 on exact float32 weights.
 # ----------------------------------------------------------------------------
+def embedding(codes: np.ndarray, scale_bits: np.ndarray, group_size: int, indices) -> np.ndarray:
+    """Rows of the dequantised weight gathered by index, exact float32 [T, K].
+
+    The Q4 embedding reads the linear weight's nibble layout ("[ExecuTorch][WebGPU]
+    Replace broad QKV fusion with BK64 kernel", description of #21483:
+    is_linear_weight); each element is the dequantisation of "[ExecuTorch][Vulkan]
+    Add et_vk.linear_q4gsw_backward kernel (4-bit input-grad)", PR description:
+        out[t, k] = (code[idx[t], k] - 8) * s[k // gs, idx[t]].
+    An index outside [0, N) raises IndexError.
+    """
+    codes = np.asarray(codes)
+    idx = np.asarray(indices, dtype=np.int64).reshape(-1)
+    N, K = codes.shape
+    if idx.size and (idx.min() < 0 or idx.max() >= N):
+        raise IndexError("embedding index outside [0, N)")
+    c = codes[idx, :].astype(np.int64)                    # [T, K]
+    s = fp16_bits_to_float(scale_bits)                    # [G, N]
+    g_of_k = np.arange(K) // group_size
+    s_tk = s[g_of_k, :][:, idx].T                         # s[k // gs, idx[t]] -> [T, K]
+    return ((c - ZERO_POINT).astype(np.float64) * s_tk).astype(np.float32)
+
+
 def linear_fwd(x_bits: np.ndarray, codes: np.ndarray, scale_bits: np.ndarray, group_size: int):
     """y[m, n] = sum_k x[m, k] * w[n, k]; returns (y, bound) with bound = sum_k |x||w|.
 

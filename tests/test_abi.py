@@ -21,7 +21,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = b.library()
     names = declared_functions()
-    assert len(names) == 11
+    assert len(names) == 12
     assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
     for n in names:
         assert hasattr(lib, n), n
@@ -82,3 +82,19 @@ def test_status_strings_and_version():
     for s in range(9):
         assert b.q4gsw_status_str(s)
     assert b.q4gsw_status_str(99) == "unknown status"
+
+
+def test_embedding_arguments_are_checked_on_the_host():
+    lib = b.library()
+    fake = 0x100000
+    assert lib.q4gsw_embedding(fake, 62, 128, 32, fake, 4, fake, None) == 2        # N % 4
+    assert lib.q4gsw_embedding(fake, 64, 96, 32, fake, 4, fake, None) == 3         # K % 64
+    assert lib.q4gsw_embedding(fake, 64, 128, 48, fake, 4, fake, None) == 4        # group size
+    assert lib.q4gsw_embedding(fake, 64, 128, 32, fake, -1, fake, None) == 2       # T < 0
+    assert lib.q4gsw_embedding(None, 64, 128, 32, None, 0, None, None) == 0        # T = 0: nothing to do
+    assert b.q4gsw_last_route() == "empty"
+    assert lib.q4gsw_embedding(None, 64, 128, 32, fake, 4, fake, None) == 1
+    assert lib.q4gsw_embedding(fake, 64, 128, 32, None, 4, fake, None) == 1
+    assert lib.q4gsw_embedding(fake, 64, 128, 32, fake + 2, 4, fake, None) == 3    # indices 4-byte aligned
+    assert lib.q4gsw_embedding(fake, 64, 128, 32, fake, 4, fake + 4, None) == 3    # out 16-byte aligned
+    assert b.q4gsw_status_str(9).startswith("an embedding index")

@@ -364,3 +364,63 @@ def test_pins_catch_planted_mistakes():
 
     for bad in (wrong_zero_point, wrong_group_index, transposed_scale, sign_flip, swapped_nibbles):
         assert not _pins_pass(bad), bad.__name__
+
+
+# ----------------------------------------------------------------------------- embedding rows
+def _embedding_fixture():
+    """N=4 rows (2 nibble pairs), K=64, gs=32: hand-chosen codes and scales."""
+    codes = np.full((4, 64), 8, dtype=np.uint8)
+    codes[0, :4] = [15, 0, 8, 7]
+    codes[1, :4] = [1, 2, 3, 4]
+    codes[2, :] = 0
+    codes[3, :] = 15
+    scales = np.array([[0.5, -0.25, 2.0, 1.0], [0.125, 4.0, -1.0, 0.0625]], dtype=np.float16)
+    return codes, scales.view(np.uint16)
+
+
+def test_embedding_hand_worked_rows():
+    codes, sb = _embedding_fixture()
+    out = o.embedding(codes, sb, 32, [3, 0, 2, 3, 1])
+    assert out.shape == (5, 64) and out.dtype == np.float32
+    # row 3: code 15 -> 7 x 1.0 in group 0, 7 x 0.0625 in group 1
+    assert (out[0, :32] == 7.0).all() and (out[0, 32:] == 0.4375).all()
+    assert np.array_equal(out[3], out[0])
+    # row 0: (15-8) 0.5, (0-8) 0.5, (8-8) 0.5, (7-8) 0.5, then zero point
+    assert out[1, :4].tolist() == [3.5, -4.0, 0.0, -0.5]
+    assert (out[1, 4:] == 0.0).all()
+    # row 2: code 0 -> -8 x 2.0, -8 x -1.0
+    assert (out[2, :32] == -16.0).all() and (out[2, 32:] == 8.0).all()
+    # row 1: (1..4 - 8) x -0.25, then 0 x -0.25 = -0.0 (IEEE) and 0 x 4.0 = +0.0
+    assert out[4, :4].tolist() == [1.75, 1.5, 1.25, 1.0]
+    assert np.signbit(out[4, 4:32]).all() and not np.signbit(out[4, 32:]).any()
+
+
+def test_embedding_rejects_indices_out_of_range_and_allows_empty():
+    codes, sb = _embedding_fixture()
+    with pytest.raises(IndexError):
+        o.embedding(codes, sb, 32, [4])
+    with pytest.raises(IndexError):
+        o.embedding(codes, sb, 32, [-1])
+    assert o.embedding(codes, sb, 32, []).shape == (0, 64)
+
+
+def test_embedding_is_a_row_selection_of_the_dequantised_weight():
+    rng = np.random.default_rng(7)
+    codes = rng.integers(0, 16, size=(24, 192), dtype=np.uint8)
+    sb = rng.uniform(-2, 2, size=(12, 24)).astype(np.float16).view(np.uint16)
+    idx = rng.integers(0, 24, size=40)
+    assert np.array_equal(o.embedding(codes, sb, 16, idx), o.dequant_w32(codes, sb, 16)[idx])
+
+
+def test_embedding_planted_mistakes_fail_the_fixture():
+    codes, sb = _embedding_fixture()
+    idx = np.array([3, 0, 2, 3, 1])
+    good = o.embedding(codes, sb, 32, idx)
+    s = o.fp16_bits_to_float(sb)
+    g = np.arange(64) // 32
+    # scale taken from the token position instead of the gathered row
+    wrong_col = ((codes[idx].astype(np.int64) - 8) * s[g][:, np.arange(5) % 4].T).astype(np.float32)
+    assert not np.array_equal(wrong_col, good)
+    # odd rows read from the low nibble of the pair (rows 2p and 2p+1 swapped)
+    swapped = o.embedding(codes, sb, 32, idx ^ 1)
+    assert not np.array_equal(swapped, good)
