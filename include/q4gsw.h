@@ -100,7 +100,7 @@ Q4GSW_API size_t q4gsw_packed_bytes(int N, int K, int group_size);
 
 /*
  * One-time packer ([P2] "Key changes": the prepack shared by forward and
- * backward; [P3]: "packing the constant weights and scales once").
+ * backward; [P3]: the constant weights and scales are packed once).
  *   codes   uint8 [N, K], one code per byte, each in 0..15
  *   scales  fp16  [K/gs, N]
  *   packed  output, packed_bytes >= q4gsw_packed_bytes(N, K, gs)
