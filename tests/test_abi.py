@@ -98,3 +98,22 @@ def test_embedding_arguments_are_checked_on_the_host():
     assert lib.q4gsw_embedding(fake, 64, 128, 32, fake + 2, 4, fake, None) == 3    # indices 4-byte aligned
     assert lib.q4gsw_embedding(fake, 64, 128, 32, fake, 4, fake + 4, None) == 3    # out 16-byte aligned
     assert b.q4gsw_status_str(9).startswith("an embedding index")
+
+
+def test_every_workload_shape_is_accepted_by_the_library():
+    from bit_group_quantized_q4gsw_b200 import workloads as wl
+    for sh in wl.all_shapes():
+        assert b.q4gsw_packed_bytes(sh.N, sh.K, sh.group_size) == \
+            o.packed_layout(sh.N, sh.K, sh.group_size)["total_bytes"] > 0, sh.name
+        if sh.splits:
+            assert sum(sh.splits) == sh.N and all(s % 8 == 0 for s in sh.splits), sh.name
+
+
+def test_embedding_token_ids_are_seeded_and_in_range():
+    import numpy as np
+    from bit_group_quantized_q4gsw_b200 import workloads as wl
+    for sh in wl.embedding():
+        ids = wl.embedding_indices(sh)
+        assert ids.dtype == np.int32 and ids.shape == (sh.M,)
+        assert ids.min() >= 0 and ids.max() < sh.N
+        assert np.array_equal(ids, wl.embedding_indices(sh))
