@@ -47,8 +47,8 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
             "+ down and up input grads; M=512 tokens, group_size 32")
 
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
-# dram__bytes_write.sum; profiles/gemm_*.md), with the hash of the kernel
-# sources they were taken on: reported only while the sources still match.
+# dram__bytes_write.sum), with the hash of the kernel sources they were taken
+# on: reported only while the sources still match, null otherwise.
 NCU_TRAFFIC = {"sources_sha": "ed63c1fc9c001ed9", "bytes_per_launch": {'up_fwd': 11561472, 'up_bwd': 17852672, 'down_fwd': 17852928, 'down_bwd': 11561216, 'qkv_fwd': 5662976}}
 
 
@@ -198,32 +198,54 @@ def host_inputs():
     return out
 
 
-def cpu_baseline(inputs, budget_s: float = 12.0):
-    t, _ = oracle_sample_step(inputs, 64)            # probe
-    frac = 64 if t > budget_s / 4 else max(1, int(64 * t / (budget_s / 4)))
-    frac = max(1, frac)
+ORACLE_BUDGET_S = 150.0   # bound on the oracle's whole timed run (warm-up included)
+
+
+def oracle_sample_fraction(inputs, runs: int) -> int:
+    """The one sample rule of both oracle legs: the first 1/frac of each op's
+    output features, frac the smallest power of two >= 16 for which `runs`
+    sample steps fit in ORACLE_BUDGET_S on this host."""
+    t, _ = oracle_sample_step(inputs, 64)
+    t16 = 4.0 * t                    # cost grows with the sampled features
+    frac = 16
+    while frac < 4096 and runs * t16 * 16 / frac > ORACLE_BUDGET_S:
+        frac *= 2
+    return frac
+
+
+def oracle_sample_text(frac: int, flops: float) -> str:
+    return (f"all 5 ops of the step, all 512 tokens, first 1/{frac} of each op's output features "
+            f"({flops / 1e9:.3f} GFLOP per sample step)")
+
+
+def cpu_baseline(inputs, runs: int = 10):
+    frac = oracle_sample_fraction(inputs, runs)
     times, flops = [], 0.0
-    t_end = time.perf_counter() + budget_s
-    while time.perf_counter() < t_end or not times:
+    for _ in range(runs):
         dt, flops = oracle_sample_step(inputs, frac)
         times.append(dt)
     value = flops / statistics.median(times) / 1e12
     return {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"all 5 ops of the step, all 512 tokens, first 1/{frac} of each op's output features; "
-                      f"{len(times)} repetitions, median"}
+            "sample": oracle_sample_text(frac, flops) + f"; {runs} sample steps, median"}
+
+
+def step_config(world: int) -> dict:
+    """The workload description both arms print (identical keys and values)."""
+    ops = step_ops()
+    set_bytes = sum(weight_bytes(sh) for sh in {sh.name: sh for _, _, sh in ops}.values())
+    act_bytes = sum(2 * sh.M * (sh.N if k == "bwd" else sh.K) for _, k, sh in ops)
+    copies = max(2, math.ceil(2.0 * L2_BYTES / (set_bytes + act_bytes)))
+    return {"workload": WORKLOAD, "global_batch": 512 * world, "seq_len": 512,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": f"rotating {copies} copies of weights+activations "
+                  f"({copies * (set_bytes + act_bytes) / 1e6:.0f} MB) > 126 MB L2"}, copies
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
     inputs = host_inputs()
-    t, _ = oracle_sample_step(inputs, 64)
-    total_budget = 150.0
-    per_step = max(0.05, total_budget / max(1, args.steps + args.warmup))
-    frac = 64
-    while frac < 4096 and t > per_step:
-        frac *= 2
-        t /= 2
+    frac = oracle_sample_fraction(inputs, args.steps + args.warmup)
     for _ in range(args.warmup):
         oracle_sample_step(inputs, frac)
     times, flops = [], 0.0
@@ -232,14 +254,13 @@ def run_reference(args, rank, world):
         times.append(dt)
     ms = 1e3 * sum(times) / len(times)
     value = flops / (ms / 1e3) / 1e12
-    sample = (f"all 5 ops, 512 tokens, first 1/{frac} of each op's output features ({flops / 1e9:.3f} GFLOP per step)")
+    config, _ = step_config(world)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "global_batch": 512, "seq_len": 512, "parallelism": "replicas"},
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": oracle_sample_text(frac, flops) + f"; {args.steps} timed steps, mean"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -351,9 +372,8 @@ def run_gpu(args, rank, world, local_rank):
     peaks = measured_peaks()
     inputs = host_inputs()
     ops = step_ops()
-    set_bytes = sum(weight_bytes(sh) for sh in {sh.name: sh for _, _, sh in ops}.values())
-    act_bytes = sum(inputs[n].x.nbytes if k != "bwd" else inputs[n].d_out.nbytes for n, k, _ in ops)
-    copies = args.copies or max(2, math.ceil(2.0 * L2_BYTES / (set_bytes + act_bytes)))
+    config, copies = step_config(world)
+    copies = args.copies or copies
     gs = GpuStep(inputs, copies, device)
     per_call = gs.launches_per_call()
     launches_per_step = sum(n for n, _ in per_call.values())
@@ -512,16 +532,15 @@ def run_gpu(args, rank, world, local_rank):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16 inputs, f32 accumulate", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "global_batch": 512 * world, "seq_len": 512,
-                       "parallelism": f"replicas{world}" if world > 1 else "single",
-                       "l2": f"rotating {copies} copies of weights+activations "
-                             f"({copies * (set_bytes + act_bytes) / 1e6:.0f} MB) > 126 MB L2"},
+            "config": config,
             "weight_gbs": world * wbytes_step / (ms_step / 1e3) / 1e9,
             "roofline": roof, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e,
             "ops_ms_sampled": {k: round(v, 5) for k, v in op_ms.items()},
             "ops_tflops": {n: op_flops(k, sh) / (op_ms[n] / 1e3) / 1e12 for n, k, sh in ops},
             "routes": {k: v[1] for k, v in per_call.items()}}
+    if not args.no_shapes:
+        line["shapes"] = shape_legs(device, peaks, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inputs)
     if rank == 0:
@@ -529,7 +548,120 @@ def run_gpu(args, rank, world, local_rank):
     return 0
 
 
-# ----------------------------------------------------------------------------- per-shape sweep
+# ----------------------------------------------------------------------------- per-shape timing
+def time_shape(q, sh, kind, device, flush, peaks):
+    """One operation of one configuration shape: mean time per launch over a
+    CUDA graph of back-to-back launches whose packed weights rotate through
+    copies totalling > 3x the L2, plus one launch timed alone after an L2 flush.
+    Returns the JSON record with both rooflines."""
+    import torch
+    inp = wl.make_inputs(sh)
+    codes = torch.from_numpy(inp.codes).to(device)
+    scales = torch.from_numpy(inp.scales).to(device)
+    first = q.q4gsw_prepack(codes, scales, sh.group_size)
+    del codes, scales
+    wb = weight_bytes(sh)
+    R = max(2, math.ceil(3 * L2_BYTES / wb))
+    packs = [first] + [first.clone() for _ in range(R - 1)]
+    src = inp.d_out if kind == "bwd" else inp.x
+    a = torch.from_numpy(src).to(device)
+    if kind == "qkv":
+        Nq, Nk, Nv = sh.splits
+        outs = tuple(torch.empty((sh.M, n), dtype=torch.float32, device=device) for n in (Nq, Nk, Nv))
+        fn = lambda pk: q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, a, outs=outs)
+    elif kind == "fwd":
+        y = torch.empty((sh.M, sh.N), dtype=torch.float32, device=device)
+        fn = lambda pk: q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a, y=y)
+    elif kind == "emb":
+        ids = torch.from_numpy(wl.embedding_indices(sh)).to(device)
+        y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
+        fn = lambda pk: q.q4gsw_embedding(pk, sh.N, sh.K, sh.group_size, ids, out=y)
+    else:
+        y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
+        fn = lambda pk: q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a, d_x=y)
+    for i in range(5):
+        fn(packs[i % R])
+    torch.cuda.synchronize()
+    iters = max(R, 50)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(iters):
+            fn(packs[i % R])
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / (reps * iters) / 1e3
+    # one launch after an L2 flush (a 256 MB write), timed alone: the launch is
+    # enqueued while the flush still runs, so host launch latency stays
+    # outside the events
+    singles = []
+    for r in range(3):
+        torch.cuda.synchronize()
+        flush.fill_(r)
+        e0.record()
+        fn(packs[r % R])
+        e1.record()
+        torch.cuda.synchronize()
+        singles.append(e0.elapsed_time(e1) * 1e3)
+    t1 = sorted(singles)[1]
+    route = q.q4gsw_last_route()
+    del g, packs, first
+    fl = op_flops(kind, sh)
+    by = op_bytes(kind, sh)
+    rec = {"shape": sh.name, "dir": kind, "M": sh.M, "N": sh.N, "K": sh.K, "gs": sh.group_size,
+           "us": t * 1e6, "tflops": fl / t / 1e12, "gbs": by / t / 1e9, "weight_gbs": wb / t / 1e9,
+           "frac_tc": fl / t / 1e12 / peaks["tflops"], "frac_hbm_measured": by / t / 1e9 / peaks["hbm_gbs"],
+           "frac_hbm_8tbs": by / t / 8e12, "us_single_cold": t1, "route": route, "copies": R,
+           "timing": f"CUDA graph of {iters} back-to-back launches over {R} rotating weight copies "
+                     f"(> 3x L2), {reps} replays; us_single_cold: one launch after a 256 MB L2 flush"}
+    ridge = peaks["tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if kind != "emb" and fl / by >= ridge:
+        rec["roofline"] = {"bound": "tensor", "achieved": fl / t / 1e12, "peak": peaks["tflops"], "unit": "TFLOP/s",
+                           "frac": fl / t / 1e12 / peaks["tflops"], "traffic": None,
+                           "peak_kind": f"bf16 dense burst ({peaks['source']})"}
+    else:
+        rec["roofline"] = {"bound": "hbm", "achieved": by / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": by / t / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                           "peak_kind": f"HBM copy ({peaks['source']})"}
+    return rec
+
+
+# The configuration shapes timed beside the step: the memory-bound half of the
+# metric (decode M=1; the sweep's M=1 and M=16 on both 8B-class matrices) and
+# the largest compute-bound shapes (the sweep's M=4096).
+SHAPE_LEGS = [("decode_N2048_K2048", "fwd"), ("decode_N8192_K2048", "fwd"), ("decode_N2048_K8192", "fwd"),
+              ("sweep_M1_N14336_K4096", "fwd"), ("sweep_M1_N14336_K4096", "bwd"),
+              ("sweep_M1_N4096_K14336", "fwd"), ("sweep_M1_N4096_K14336", "bwd"),
+              ("sweep_M16_N14336_K4096", "fwd"), ("sweep_M16_N14336_K4096", "bwd"),
+              ("sweep_M16_N4096_K14336", "fwd"), ("sweep_M16_N4096_K14336", "bwd"),
+              ("sweep_M4096_N14336_K4096", "fwd"), ("sweep_M4096_N14336_K4096", "bwd"),
+              ("sweep_M4096_N4096_K14336", "fwd"), ("sweep_M4096_N4096_K14336", "bwd")]
+
+
+def shape_legs(device, peaks, world):
+    import torch
+    import bit_group_quantized_q4gsw_b200 as q
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    out = []
+    for name, kind in SHAPE_LEGS:
+        barrier(world)
+        rec = time_shape(q, wl.by_name(name), kind, device, flush, peaks)
+        # whole-job figures: every rank runs the same shape (replicas)
+        t_max = max_over_ranks(rec["us"], world)
+        rec["us_max_over_ranks"] = t_max
+        out.append(rec)
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_sweep(args):
     import torch
     import bit_group_quantized_q4gsw_b200 as q
@@ -541,72 +673,9 @@ def run_sweep(args):
         import re
         shapes = [s for s in shapes if re.search(args.only, s.name)]
     for sh in shapes:
-        inp = wl.make_inputs(sh)
-        codes = torch.from_numpy(inp.codes).to(device)
-        scales = torch.from_numpy(inp.scales).to(device)
-        first = q.q4gsw_prepack(codes, scales, sh.group_size)
-        del codes, scales
-        wb = weight_bytes(sh)
-        R = max(2, math.ceil(3 * L2_BYTES / wb))
-        packs = [first] + [first.clone() for _ in range(R - 1)]
         kinds = ["qkv"] if sh.splits else list(sh.directions)
         for kind in kinds:
-            src = inp.d_out if kind == "bwd" else inp.x
-            a = torch.from_numpy(src).to(device)
-            if kind == "qkv":
-                Nq, Nk, Nv = sh.splits
-                outs = tuple(torch.empty((sh.M, n), dtype=torch.float32, device=device) for n in (Nq, Nk, Nv))
-                fn = lambda pk: q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, a, outs=outs)
-            elif kind == "fwd":
-                y = torch.empty((sh.M, sh.N), dtype=torch.float32, device=device)
-                fn = lambda pk: q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a, y=y)
-            elif kind == "emb":
-                ids = torch.from_numpy(wl.embedding_indices(sh)).to(device)
-                y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
-                fn = lambda pk: q.q4gsw_embedding(pk, sh.N, sh.K, sh.group_size, ids, out=y)
-            else:
-                y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
-                fn = lambda pk: q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a, d_x=y)
-            for i in range(5):
-                fn(packs[i % R])
-            torch.cuda.synchronize()
-            iters = max(R, 50)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for i in range(iters):
-                    fn(packs[i % R])
-            g.replay()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = 3
-            e0.record()
-            for _ in range(reps):
-                g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            t = e0.elapsed_time(e1) / (reps * iters) / 1e3
-            # one launch after an L2 flush (a 256 MB write), timed alone: the
-            # launch is enqueued while the flush still runs, so host launch
-            # latency stays outside the events
-            singles = []
-            for r in range(3):
-                torch.cuda.synchronize()
-                flush.fill_(r)
-                e0.record()
-                fn(packs[r % R])
-                e1.record()
-                torch.cuda.synchronize()
-                singles.append(e0.elapsed_time(e1) * 1e3)
-            t1 = sorted(singles)[1]
-            fl = op_flops(kind, sh)
-            by = op_bytes(kind, sh)
-            print(json.dumps({"shape": sh.name, "dir": kind, "M": sh.M, "N": sh.N, "K": sh.K, "gs": sh.group_size,
-                              "us": t * 1e6, "tflops": fl / t / 1e12, "gbs": by / t / 1e9,
-                              "weight_gbs": wb / t / 1e9, "frac_tc": fl / t / 1e12 / peaks["tflops"],
-                              "frac_hbm_measured": by / t / 1e9 / peaks["hbm_gbs"], "frac_hbm_8tbs": by / t / 8e12,
-                              "us_single_cold": t1, "route": q.q4gsw_last_route(), "copies": R}), flush=True)
-            del g
-        del packs, first
+            print(json.dumps(time_shape(q, sh, kind, device, flush, peaks)), flush=True)
         torch.cuda.empty_cache()
     return 0
 
@@ -650,6 +719,7 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--only", default="")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-shapes", action="store_true", help="skip the per-shape legs beside the step")
     ap.add_argument("--case", default="", help="SHAPE:DIR, e.g. adapter_up_M512:fwd (profiling launches)")
     ap.add_argument("--case-m", type=int, default=0)
     ap.add_argument("--iters", type=int, default=3)

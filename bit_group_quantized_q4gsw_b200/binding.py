@@ -36,6 +36,8 @@ SIGNATURES = [
     ("q4gsw_device_error_check", _I, [_VP]),
     ("q4gsw_unpack", _I, [_VP, _I, _I, _I, _VP, _VP]),
     ("q4gsw_dequant", _I, [_VP, _I, _I, _I, _VP, _VP, _VP]),
+    ("q4gsw_debug_pin_routes", _I, [_I, _I]),
+    ("q4gsw_debug_wait_timeout", _I, [ctypes.c_uint, _VP]),
     ("q4gsw_last_route", ctypes.c_char_p, []),
     ("q4gsw_status_str", ctypes.c_char_p, [_I]),
 ]
@@ -186,6 +188,23 @@ def q4gsw_device_error_check(device=None) -> None:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     st = library().q4gsw_device_error_check(torch.cuda.current_stream(dev).cuda_stream)
     _check("q4gsw_device_error_check", st)
+
+
+GEMV_ROUTES = {"auto": 0, "reg": 1, "tma": 2}
+GEMM_ROUTES = {"auto": 0, "ts": 1, "ss": 2, "ss1": 3, "ss2": 4}
+
+
+def q4gsw_debug_pin_routes(gemv: str = "auto", gemm: str = "auto") -> None:
+    """Pin the kernel routes of this thread's later calls (debug export; see include/q4gsw.h)."""
+    st = library().q4gsw_debug_pin_routes(GEMV_ROUTES[gemv], GEMM_ROUTES[gemm])
+    _check("q4gsw_debug_pin_routes", st)
+
+
+def q4gsw_debug_wait_timeout(limit_us: int, device=None) -> None:
+    """Enqueue the bounded-wait probe: one wait that runs out after limit_us microseconds."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = library().q4gsw_debug_wait_timeout(limit_us, torch.cuda.current_stream(dev).cuda_stream)
+    _check("q4gsw_debug_wait_timeout", st)
 
 
 def q4gsw_unpack(packed: torch.Tensor, N: int, K: int, group_size: int) -> torch.Tensor:

@@ -18,6 +18,32 @@
 #include "q4gsw_common.cuh"
 #include "q4gsw_internal.h"
 
+namespace q4gsw {
+
+RoutePins& route_pins() {
+  thread_local RoutePins pins;
+  return pins;
+}
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  return dev;
+}
+
+int sm_count(int dev) {
+  static std::atomic<int> cached[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) dev = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+}  // namespace q4gsw
+
 using namespace q4gsw;
 
 namespace {
@@ -170,6 +196,19 @@ q4gsw_status q4gsw_embedding(const void* packed, int N, int K, int group_size, c
   if (!aligned16(packed) || !aligned16(out) || (reinterpret_cast<uintptr_t>(indices) & 3u)) return Q4GSW_ERR_ALIGN;
   set_route("embedding_gather launches=1");
   return from_cuda(launch_embedding(packed, N, K, group_size, indices, T, out, stream));
+}
+
+q4gsw_status q4gsw_debug_pin_routes(int gemv, int gemm) {
+  if (gemv < kGemvAuto || gemv > kGemvTma || gemm < kGemmAuto || gemm > kGemmSs2) return Q4GSW_ERR_SHAPE;
+  route_pins().gemv = gemv;
+  route_pins().gemm = gemm;
+  return Q4GSW_OK;
+}
+
+q4gsw_status q4gsw_debug_wait_timeout(unsigned int limit_us, q4gsw_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000u) return Q4GSW_ERR_SHAPE;
+  set_route("wait_probe launches=1");
+  return from_cuda(launch_wait_probe(limit_us, stream));
 }
 
 q4gsw_status q4gsw_unpack(const void* packed, int N, int K, int group_size, uint8_t* codes,

@@ -21,8 +21,10 @@ namespace q4gsw {
 constexpr unsigned int kIndexErrorBit = 0x100u;   // device error word: embedding index out of range
 constexpr int kEmbThreads = 128;
 
+namespace emb {
+
 __global__ void __launch_bounds__(kEmbThreads)
-embedding_kernel(const uint8_t* __restrict__ packed, const int32_t* __restrict__ indices, float* __restrict__ out,
+q4gsw_embedding_kernel(const uint8_t* __restrict__ packed, const int32_t* __restrict__ indices, float* __restrict__ out,
                  int N, int K, int gs, int T) {
   const Layout L = layout_of(N, K, gs);
   const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
@@ -58,12 +60,14 @@ embedding_kernel(const uint8_t* __restrict__ packed, const int32_t* __restrict__
   }
 }
 
+}  // namespace emb
+
 cudaError_t launch_embedding(const void* packed, int N, int K, int gs, const int32_t* indices, int T, float* out,
                              cudaStream_t stream) {
   const int chunks = K / 16;
   const dim3 grid((chunks + kEmbThreads - 1) / kEmbThreads, T < 65535 ? T : 65535);
-  embedding_kernel<<<grid, kEmbThreads, 0, stream>>>(static_cast<const uint8_t*>(packed), indices, out, N, K, gs,
-                                                     T);
+  emb::q4gsw_embedding_kernel<<<grid, kEmbThreads, 0, stream>>>(static_cast<const uint8_t*>(packed), indices, out, N,
+                                                                K, gs, T);
   return cudaGetLastError();
 }
 

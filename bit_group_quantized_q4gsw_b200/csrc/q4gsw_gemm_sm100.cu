@@ -42,8 +42,13 @@ namespace cg = cooperative_groups;
 
 namespace q4gsw {
 
-// OR of the codes of waits that timed out (read and cleared by the host).
+// OR of the codes of waits that timed out and of out-of-range embedding
+// indices: one word per device, shared by every stream and host thread (read
+// and cleared by q4gsw_device_error_check).
 __device__ unsigned int g_device_error = 0;
+// Values swapped out of g_device_error, one slot per concurrent check.
+constexpr int kErrorSlots = 64;
+__device__ unsigned int g_error_snapshot[kErrorSlots];
 
 namespace gemm {
 
@@ -413,15 +418,18 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 lookup_encode_fn() {
+  cudaDriverEntryPointQueryResult q;
+  void* p = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  return nullptr;
+}
+
+// The driver's tensor-map encoder, looked up once (thread-safe static init).
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = lookup_encode_fn();
   return fn;
 }
 
@@ -456,15 +464,15 @@ static cudaError_t gemm_variant(const CUtensorMap& map_act, const CUtensorMap& m
   using namespace gemm;
   auto kern = q4gsw_gemm_kernel<BWD, ST, SCB, MSUB>;
   constexpr int smem = Smem<ST, SCB, MSUB>::BYTES;
-  static bool attr_done[64] = {};
-  static int max_clusters[64][9] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int d = (dev >= 0 && dev < 64) ? dev : 0;
-  if (!attr_done[d]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static PerDeviceOnce attr_once;
+  static std::atomic<int> max_clusters[kMaxDevices][9];
+  const int dev = current_device();
+  const int d = (dev >= 0 && dev < kMaxDevices) ? dev : 0;
+  {
+    cudaError_t e = once_per_device(attr_once, dev, [&] {
+      return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
     if (e != cudaSuccess) return e;
-    attr_done[d] = true;
   }
   const int tiles_m = (a.M + BM * MSUB - 1) / (BM * MSUB);
   cudaLaunchConfig_t cfg = {};
@@ -486,14 +494,13 @@ static cudaError_t gemm_variant(const CUtensorMap& map_act, const CUtensorMap& m
   double best_cost = 1e30;
   for (int S = 1; S <= 8; ++S) {
     if (S > 1 && a.stages_total / S < 4) break;
-    if (!max_clusters[d][S]) {
+    int n = max_clusters[d][S].load(std::memory_order_relaxed);
+    if (n == 0) {   // not measured yet on this device (concurrent callers store the same value)
       attr[0].val.clusterDim.z = S;
       cfg.gridDim = dim3(tiles_n, tiles_m, S);
-      int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = -1;
-      max_clusters[d][S] = n;
+      max_clusters[d][S].store(n, std::memory_order_relaxed);
     }
-    const int n = max_clusters[d][S];
     if (n < 1) continue;
     const double waves = ceil((double)tiles / n);
     const double cost = waves * ((double)a.stages_total / S * t + (S > 1 ? 8.0 : 2.0) * MSUB);
@@ -510,11 +517,11 @@ static cudaError_t gemm_variant(const CUtensorMap& map_act, const CUtensorMap& m
   return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, a);
 }
 
-// Q4GSW_GEMM_MSUB=1 or 2 pins the number of 128-token accumulators per CTA
-// (for tuning and tests); unset or 0 lets the cost model choose.
+// Number of 128-token accumulators per CTA pinned by q4gsw_debug_pin_routes
+// (1 or 2), or 0: the cost model chooses.
 static int forced_msub() {
-  const char* e = getenv("Q4GSW_GEMM_MSUB");
-  return (e && (e[0] == '1' || e[0] == '2') && e[1] == 0) ? e[0] - '0' : 0;
+  const int g = route_pins().gemm;
+  return g == kGemmSs1 ? 1 : g == kGemmSs2 ? 2 : 0;
 }
 
 template <bool BWD>
@@ -600,11 +607,11 @@ namespace q4gsw {
 // in tensor memory (its shared-memory traffic is lowest); above, the
 // shared-memory route with two 128-token accumulators per CTA re-reads each
 // activation tile half as often from L2 and wins (measured on B200 at 1024 and
-// 4096 tokens).  Q4GSW_GEMM_KIND=ss or ts pins the route (tests and tuning).
+// 4096 tokens).  q4gsw_debug_pin_routes can pin either route.
 static bool use_ss_route(int M) {
-  const char* e = getenv("Q4GSW_GEMM_KIND");
-  if (e && e[0] == 's' && e[1] == 's' && e[2] == 0) return true;
-  if (e && e[0] == 't' && e[1] == 's' && e[2] == 0) return false;
+  const int g = route_pins().gemm;
+  if (g == kGemmTs) return false;
+  if (g == kGemmSs || g == kGemmSs1 || g == kGemmSs2) return true;
   return M > 512;
 }
 
@@ -621,19 +628,42 @@ cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint
   return launch_gemm_ts_impl<true>(packed, N, K, gs, d_out, M, single_output(d_x, K), stream, route, route_len);
 }
 
-cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int* host_value) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbolAsync(host_value, g_device_error, sizeof(unsigned int), 0,
-                                            cudaMemcpyDeviceToHost, stream);
-  if (e != cudaSuccess) return e;
-  e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return e;
-  if (*host_value) {
-    e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, stream);
-    if (e != cudaSuccess) return e;
-    e = cudaStreamSynchronize(stream);
+__global__ void q4gsw_error_exchange_kernel(unsigned int slot) {
+  g_error_snapshot[slot] = atomicExch(&g_device_error, 0u);
+}
+
+// A wait on a barrier that nothing completes, bounded by limit_ns: the
+// failure path of every kernel's waits, run on purpose and without a fault.
+__global__ void q4gsw_wait_probe_kernel(unsigned long long limit_ns) {
+  using namespace sm100;
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
   }
-  return e;
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, &g_device_error, 0x200u, limit_ns);
+}
+
+cudaError_t launch_wait_probe(unsigned int limit_us, cudaStream_t stream) {
+  q4gsw_wait_probe_kernel<<<1, 32, 0, stream>>>(1000ull * limit_us);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int* host_value) {
+  // The swap is one atomic on the device, so a bit that a kernel on another
+  // stream sets after it stays in the word for the next check.
+  static std::atomic<unsigned int> next_slot{0};
+  const unsigned int slot = next_slot.fetch_add(1, std::memory_order_relaxed) % kErrorSlots;
+  q4gsw_error_exchange_kernel<<<1, 1, 0, stream>>>(slot);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbolAsync(host_value, g_error_snapshot, sizeof(unsigned int), slot * sizeof(unsigned int),
+                                cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(stream);
 }
 
 }  // namespace q4gsw

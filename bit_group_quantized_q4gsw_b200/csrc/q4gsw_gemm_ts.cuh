@@ -486,15 +486,15 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
 
   auto kern = q4gsw_gemm_ts_kernel<BWD, ST>;
   constexpr int smem = Smem<ST>::BYTES;
-  static bool attr_done[64] = {};
-  static int max_clusters[64][9] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int d = (dev >= 0 && dev < 64) ? dev : 0;
-  if (!attr_done[d]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static PerDeviceOnce attr_once;
+  static std::atomic<int> max_clusters[kMaxDevices][9];
+  const int dev = current_device();
+  const int d = (dev >= 0 && dev < kMaxDevices) ? dev : 0;
+  {
+    cudaError_t e = once_per_device(attr_once, dev, [&] {
+      return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
     if (e != cudaSuccess) return e;
-    attr_done[d] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -517,14 +517,13 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
   double best_cost = 1e30;
   for (int S = 1; S <= 8; ++S) {
     if (S > 1 && a.stages_total / S < 4) break;
-    if (!max_clusters[d][S]) {
+    int n = max_clusters[d][S].load(std::memory_order_relaxed);
+    if (n == 0) {   // not measured yet on this device (concurrent callers store the same value)
       attr[0].val.clusterDim.z = S;
       cfg.gridDim = dim3(tiles_f, tiles_t, S);
-      int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = -1;
-      max_clusters[d][S] = n;
+      max_clusters[d][S].store(n, std::memory_order_relaxed);
     }
-    const int n = max_clusters[d][S];
     if (n < 1) continue;
     const double waves = ceil((double)tiles / n);
     const double cost = waves * ((double)a.stages_total / S + (S > 1 ? 8.0 : 2.0));

@@ -24,7 +24,6 @@
 
 #include <cmath>
 #include <cstdio>
-#include <cstdlib>
 
 #include "q4gsw_common.cuh"
 #include "q4gsw_internal.h"
@@ -32,6 +31,7 @@
 namespace cg = cooperative_groups;
 
 namespace q4gsw {
+namespace rg {
 
 constexpr int kGemvWarps = 4;
 constexpr int kGemvThreads = 32 * kGemvWarps;
@@ -46,7 +46,7 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // SPG = 16-column steps per scale group (1: gs 16, 2: gs 32, 4: gs >= 64).
 template <int NT, int SPG>
 __global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 7 : 4)
-gemv_fwd_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x, OutSplit out, int M, int N,
+q4gsw_gemv_fwd_reg_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x, OutSplit out, int M, int N,
                 int K, int gs) {
   __shared__ float red[kGemvWarps][16][16];  // [warp][token][row]
   __shared__ float cta_part[16][16];         // [token][row]
@@ -225,7 +225,7 @@ constexpr int kBwdWarps = 8;
 constexpr int kBwdThreads = 32 * kBwdWarps;
 
 template <int NT, int SPB>  // NT 8-token tiles; SPB scale groups per block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
-__global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __restrict__ packed,
+__global__ void __launch_bounds__(kBwdThreads) q4gsw_gemv_bwd_reg_kernel(const uint8_t* __restrict__ packed,
                                                                const __half* __restrict__ dout,
                                                                float* __restrict__ dx,
                                                                int M, int N, int K, int gs) {
@@ -375,26 +375,21 @@ __global__ void __launch_bounds__(kBwdThreads) gemv_bwd_kernel(const uint8_t* __
   if (S > 1) cluster.sync();
 }
 
+}  // namespace rg
+
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
-static int sm_count() {
-  static int cached = 0;
-  if (!cached) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached = n > 0 ? n : 148;
-  }
-  return cached;
-}
-
+using rg::kGemvWarps;
+using rg::kGemvThreads;
+using rg::kBwdWarps;
+using rg::kBwdThreads;
 // Contraction splits S (the cluster size), from measurements on B200 over the
 // decode, MLP and 8B-layer shapes: the forward wants about six CTAs per SM and
 // no split that leaves a large weight's warps with fewer than 8 blocks; the
 // input gradient, whose output tile is narrow, wants about 320 CTAs.
 static int fwd_splits(long long tiles, int blocks_per_tile, size_t weight_bytes) {
-  int S = (int)lround(6.0 * sm_count() / (double)tiles);
+  int S = (int)lround(6.0 * sm_count(current_device()) / (double)tiles);
   S = S < 1 ? 1 : S > 8 ? 8 : S;
   // a large weight keeps at least 8 blocks (a few pipeline turns) per warp
   const int min_blocks = weight_bytes >= ((size_t)16 << 20) ? 8 : 1;
@@ -438,15 +433,13 @@ static cudaError_t launch_cluster(Kern kernel, dim3 grid, int threads, int clust
 // tokens when its CTAs spread evenly over the SMs (each SM's share within 15 %
 // of the busiest SM's); otherwise the register-fed kernel, whose 16-row CTAs
 // balance better, is faster (measured on B200: 14336x4096 at M=1, 224 CTAs on
-// 148 SMs, 13.4 vs 11.3 us).  Q4GSW_GEMV_KIND=reg or tma pins the route.
+// 148 SMs, 13.4 vs 11.3 us).  q4gsw_debug_pin_routes can pin either kernel.
 static bool use_reg_gemv(int N, int K, int M) {
-  const char* e = getenv("Q4GSW_GEMV_KIND");
-  if (e && e[0] == 'r' && e[1] == 'e' && e[2] == 'g' && e[3] == 0) return true;
-  if (e && e[0] == 't' && e[1] == 'm' && e[2] == 'a' && e[3] == 0) return false;
+  const int pin = route_pins().gemv;
+  if (pin == kGemvReg) return true;
+  if (pin == kGemvTma) return false;
   if (M > 8) return false;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count(current_device());
   const int tiles = (N + 63) / 64, stages = (K + 255) / 256;
   int S = 2 * sms / tiles;
   S = S < 1 ? 1 : (S > 8 ? 8 : S);
@@ -469,7 +462,7 @@ cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint
 #define Q4_FWD(NT_, SPG_)                                                                                       \
   do {                                                                                                          \
     S = fwd_splits((long long)tiles * zs, K / 64, (size_t)N * K / 2);                                        \
-    err = launch_cluster(gemv_fwd_kernel<NT_, SPG_>, dim3(tiles, S, zs), kGemvThreads, S, 0, stream, pk, xh, out, \
+    err = launch_cluster(rg::q4gsw_gemv_fwd_reg_kernel<NT_, SPG_>, dim3(tiles, S, zs), kGemvThreads, S, 0, stream, pk, xh, out, \
                          M, N, K, gs);                                                                          \
   } while (0)
   if (NT == 1) {
@@ -484,11 +477,8 @@ cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint
 
 cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M,
                             float* d_x, cudaStream_t stream, char* route, int route_len) {
-  {
-    const char* e = getenv("Q4GSW_GEMV_KIND");
-    const bool reg = e && e[0] == 'r' && e[1] == 'e' && e[2] == 'g' && e[3] == 0;
-    if (!reg) return launch_gemv_tma_bwd(packed, N, K, gs, d_out, M, d_x, stream, route, route_len);
-  }
+  // the TMA-ring input gradient is the default; the register-fed one runs only when pinned
+  if (route_pins().gemv != kGemvReg) return launch_gemv_tma_bwd(packed, N, K, gs, d_out, M, d_x, stream, route, route_len);
   const int tiles = (K + 127) / 128;
   const int zs = (M + 15) / 16;
   const int NT = (M <= 8) ? 1 : 2;
@@ -500,10 +490,10 @@ cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint
   cudaError_t err;
 #define Q4_BWD(NT_, SPB_)                                                                                         \
   do {                                                                                                            \
-    err = cudaFuncSetAttribute(gemv_bwd_kernel<NT_, SPB_>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    err = cudaFuncSetAttribute(rg::q4gsw_gemv_bwd_reg_kernel<NT_, SPB_>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (err == cudaSuccess) {                                                                                     \
       S = bwd_splits((long long)tiles * zs, (N + 15) / 16, kBwdWarps);                                           \
-      err = launch_cluster(gemv_bwd_kernel<NT_, SPB_>, dim3(tiles, S, zs), kBwdThreads, S, smem, stream, pk, dh,  \
+      err = launch_cluster(rg::q4gsw_gemv_bwd_reg_kernel<NT_, SPB_>, dim3(tiles, S, zs), kBwdThreads, S, smem, stream, pk, dh,  \
                            d_x, M, N, K, gs);                                                                     \
     }                                                                                                             \
   } while (0)

@@ -86,7 +86,7 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 // (1: gs 16, 2: gs 32, 4: gs >= 64).
 template <int NT, int SPG>
 __global__ void __launch_bounds__(kThreads, Cfg<NT>::kCtasPerSm)
-gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
+q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
                     const __grid_constant__ CUtensorMap map_x, OutSplit out, int M, int N, int K, int gs,
                     int stages_total) {
   using namespace sm100;
@@ -319,7 +319,7 @@ struct BwdCfg {
 
 template <int NT, int SPB>  // SPB scale groups per 64-column block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
 __global__ void __launch_bounds__(kBwdThreads, 2)
-gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
+q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
                     const __grid_constant__ CUtensorMap map_d, float* __restrict__ dx, int M, int N, int K,
                     int gs, int stages_total) {
   using namespace sm100;
@@ -524,19 +524,13 @@ static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUte
                                            const CUtensorMap& map_x, OutSplit out, int M, int N, int K, int gs,
                                            int stages_total, dim3 grid, cudaStream_t stream) {
   using C = gv::Cfg<NT>;
-  auto kern = gv::gemv_fwd_tma_kernel<NT, SPG>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int d = (dev >= 0 && dev < 64) ? dev : 0;
-  if (!attr_done[d]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+  auto kern = gv::q4gsw_gemv_fwd_tma_kernel<NT, SPG>;
+  static PerDeviceOnce attr_once;
+  {
+    cudaError_t e = once_per_device(attr_once, current_device(), [&] {
+      return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+    });
     if (e != cudaSuccess) return e;
-    if (grid.y > 8) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-    }
-    attr_done[d] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -566,12 +560,7 @@ cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, const 
   const int stages_total = (K + gv::SK - 1) / gv::SK;
   // fill the resident CTA slots in one wave, at least two stages per split,
   // clusters of at most 8
-  int sms = 148;
-  {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
+  const int sms = sm_count(current_device());
   const int slots = sms * (NT == 1 ? gv::Cfg<1>::kCtasPerSm : gv::Cfg<2>::kCtasPerSm);
   int S = slots / (tiles * zs);
   S = S < 1 ? 1 : (S > 8 ? 8 : S);
@@ -611,12 +600,7 @@ cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const 
   const int zs = (M + 15) / 16;
   const int tiles = (K + 127) / 128;
   const int stages_total = (N + 127) / 128;
-  int sms = 148;
-  {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
+  const int sms = sm_count(current_device());
   // fill the two resident CTA slots per SM, at least two stages per split
   int S = 2 * sms / (tiles * zs);
   S = S < 1 ? 1 : (S > 8 ? 8 : S);
@@ -653,13 +637,13 @@ cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const 
   };
   cudaError_t e;
   if (NT == 1)
-    e = spb == 1 ? launch(gv::gemv_bwd_tma_kernel<1, 1>, gv::BwdCfg<1>::BYTES)
-      : spb == 2 ? launch(gv::gemv_bwd_tma_kernel<1, 2>, gv::BwdCfg<1>::BYTES)
-                 : launch(gv::gemv_bwd_tma_kernel<1, 4>, gv::BwdCfg<1>::BYTES);
+    e = spb == 1 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<1, 1>, gv::BwdCfg<1>::BYTES)
+      : spb == 2 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<1, 2>, gv::BwdCfg<1>::BYTES)
+                 : launch(gv::q4gsw_gemv_bwd_tma_kernel<1, 4>, gv::BwdCfg<1>::BYTES);
   else
-    e = spb == 1 ? launch(gv::gemv_bwd_tma_kernel<2, 1>, gv::BwdCfg<2>::BYTES)
-      : spb == 2 ? launch(gv::gemv_bwd_tma_kernel<2, 2>, gv::BwdCfg<2>::BYTES)
-                 : launch(gv::gemv_bwd_tma_kernel<2, 4>, gv::BwdCfg<2>::BYTES);
+    e = spb == 1 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<2, 1>, gv::BwdCfg<2>::BYTES)
+      : spb == 2 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<2, 2>, gv::BwdCfg<2>::BYTES)
+                 : launch(gv::q4gsw_gemv_bwd_tma_kernel<2, 4>, gv::BwdCfg<2>::BYTES);
   if (route)
     snprintf(route, route_len, "gemv_tma_bwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S,
              zs, stages_total);

@@ -2,10 +2,41 @@
 // library.  Not part of the C ABI.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 namespace q4gsw {
+
+// Route pins of the calling host thread (set by q4gsw_debug_pin_routes; 0
+// everywhere means the launchers choose).  Thread-local, like the route string.
+enum GemvPin { kGemvAuto = 0, kGemvReg = 1, kGemvTma = 2 };
+enum GemmPin { kGemmAuto = 0, kGemmTs = 1, kGemmSs = 2, kGemmSs1 = 3, kGemmSs2 = 4 };
+struct RoutePins {
+  int gemv = kGemvAuto;
+  int gemm = kGemmAuto;
+};
+RoutePins& route_pins();
+
+// One-time set-up per device (cudaFuncSetAttribute of one kernel variant),
+// safe when several host threads make their first call at the same time: the
+// first caller runs `fn`, the others wait for it and then see its result.
+constexpr int kMaxDevices = 64;
+struct PerDeviceOnce {
+  std::once_flag flag[kMaxDevices];
+  std::atomic<int> err[kMaxDevices];
+};
+template <typename F>
+inline cudaError_t once_per_device(PerDeviceOnce& o, int dev, F&& fn) {
+  if (dev < 0 || dev >= kMaxDevices) return fn();   // not cached
+  std::call_once(o.flag[dev], [&] { o.err[dev].store(static_cast<int>(fn())); });
+  return static_cast<cudaError_t>(o.err[dev].load());
+}
+
+// Device the calling thread is bound to (cudaGetDevice), and its SM count.
+int current_device();
+int sm_count(int dev);
 
 cudaError_t launch_prepack(const uint8_t* codes, const uint16_t* scales, int N, int K, int gs,
                            void* packed, cudaStream_t stream, uint32_t* host_flag);
@@ -50,8 +81,13 @@ cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint
 cudaError_t launch_embedding(const void* packed, int N, int K, int gs, const int32_t* indices, int T, float* out,
                              cudaStream_t stream);
 
-// Reads (and clears when set) the device word in which kernels record waits
-// that ran out (and embedding indices out of range); synchronises `stream`.
+// One thread block that waits on a barrier nothing completes until its
+// bounded wait (limit_us microseconds) runs out and records a time-out.
+cudaError_t launch_wait_probe(unsigned int limit_us, cudaStream_t stream);
+
+// Swaps the device word in which kernels record waits that ran out (and
+// embedding indices out of range) with 0 in one atomic operation, ordered on
+// `stream`, and returns the old value; synchronises `stream`.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int* host_value);
 
 }  // namespace q4gsw

@@ -13,11 +13,12 @@
 #include "q4gsw_internal.h"
 
 namespace q4gsw {
+namespace pk {
 
 // One thread per 16-byte output chunk of the codes region: pair p, 64-byte
 // block b, quarter t of the block.  The chunk holds word slots 4t .. 4t+3, i.e.
 // columns 64b + 16 i + 4 t + e for i, e in 0..3.
-__global__ void prepack_codes_kernel(const uint8_t* __restrict__ codes, uint8_t* __restrict__ packed,
+__global__ void q4gsw_prepack_codes_kernel(const uint8_t* __restrict__ codes, uint8_t* __restrict__ packed,
                                      int N, int K, uint32_t* __restrict__ range_flag) {
   const int blocks_per_row = K / 64;
   const long long chunks = (long long)(N / 2) * blocks_per_row * 4;
@@ -46,7 +47,7 @@ __global__ void prepack_codes_kernel(const uint8_t* __restrict__ codes, uint8_t*
 
 // Scales copy, zero padding and trailer words 0..4 (word 5, the range flag, is
 // zeroed by the host before this runs and only ever OR-ed).
-__global__ void prepack_tail_kernel(const uint16_t* __restrict__ scales, uint8_t* __restrict__ packed,
+__global__ void q4gsw_prepack_tail_kernel(const uint16_t* __restrict__ scales, uint8_t* __restrict__ packed,
                                     int N, int K, int gs) {
   const Layout L = layout_of(N, K, gs);
   const size_t tid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
@@ -67,7 +68,7 @@ __global__ void prepack_tail_kernel(const uint16_t* __restrict__ scales, uint8_t
   }
 }
 
-__global__ void unpack_kernel(const uint8_t* __restrict__ packed, uint8_t* __restrict__ codes, int N, int K) {
+__global__ void q4gsw_unpack_kernel(const uint8_t* __restrict__ packed, uint8_t* __restrict__ codes, int N, int K) {
   const int blocks_per_row = K / 64;
   const long long chunks = (long long)(N / 2) * blocks_per_row * 4;
   for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < chunks;
@@ -92,7 +93,7 @@ __global__ void unpack_kernel(const uint8_t* __restrict__ packed, uint8_t* __res
 // The dequantised weight, produced with the same conversions the GEMM
 // kernels use: w16 = fp16((code - 8)) * scale rounded once (HMUL2), and the
 // exact fp32 product w32.
-__global__ void dequant_kernel(const uint8_t* __restrict__ packed, float* __restrict__ w32,
+__global__ void q4gsw_dequant_kernel(const uint8_t* __restrict__ packed, float* __restrict__ w32,
                                uint16_t* __restrict__ w16, int N, int K, int gs) {
   const Layout L = layout_of(N, K, gs);
   const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
@@ -133,6 +134,8 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ packed, float* __rest
   }
 }
 
+}  // namespace pk
+
 static int grid_for(long long work, int threads) {
   long long g = (work + threads - 1) / threads;
   if (g > 148LL * 16) g = 148LL * 16;
@@ -148,8 +151,8 @@ cudaError_t launch_prepack(const uint8_t* codes, const uint16_t* scales, int N, 
   cudaError_t err = cudaMemsetAsync(out + L.trailer_offset, 0, kTrailerBytes, stream);
   if (err != cudaSuccess) return err;
   const long long chunks = (long long)(N / 2) * (K / 64) * 4;
-  prepack_codes_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(codes, out, N, K, flag);
-  prepack_tail_kernel<<<grid_for((long long)(L.scales_bytes / 16) + 256, 256), 256, 0, stream>>>(scales, out, N, K, gs);
+  pk::q4gsw_prepack_codes_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(codes, out, N, K, flag);
+  pk::q4gsw_prepack_tail_kernel<<<grid_for((long long)(L.scales_bytes / 16) + 256, 256), 256, 0, stream>>>(scales, out, N, K, gs);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   err = cudaMemcpyAsync(host_flag, flag, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream);
@@ -159,14 +162,14 @@ cudaError_t launch_prepack(const uint8_t* codes, const uint16_t* scales, int N, 
 
 cudaError_t launch_unpack(const void* packed, int N, int K, uint8_t* codes, cudaStream_t stream) {
   const long long chunks = (long long)(N / 2) * (K / 64) * 4;
-  unpack_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(static_cast<const uint8_t*>(packed), codes, N, K);
+  pk::q4gsw_unpack_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(static_cast<const uint8_t*>(packed), codes, N, K);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequant(const void* packed, int N, int K, int gs, float* w32, uint16_t* w16,
                            cudaStream_t stream) {
   const long long chunks = (long long)(N / 2) * (K / 64) * 4;
-  dequant_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(static_cast<const uint8_t*>(packed), w32, w16, N, K, gs);
+  pk::q4gsw_dequant_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(static_cast<const uint8_t*>(packed), w32, w16, N, K, gs);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,8 @@
 // q4gsw_sm100.cuh - thin inline-PTX wrappers for the Blackwell (sm_100a)
 // features the GEMM route uses: mbarriers, TMA tensor loads, tensor memory
 // (tcgen05.alloc / ld / dealloc), tcgen05.mma with shared-memory descriptors.
-// Every wait is bounded: past kWaitCycles the waiter raises the CTA's abort
-// flag and the library's device error word, and returns false.
+// Every wait is bounded: past kWaitNs of wall-clock time the waiter raises the
+// CTA's abort flag and the library's device error word, and returns false.
 #pragma once
 
 #include <cuda.h>
@@ -11,8 +11,15 @@
 namespace q4gsw {
 namespace sm100 {
 
-// ~1 s at 2 GHz: far above any legitimate wait of this library's kernels.
-constexpr long long kWaitCycles = 2000000000LL;
+// Wall-clock bound of every wait (nanoseconds of %globaltimer): far above any
+// legitimate wait of this library's kernels, and independent of the SM clock.
+constexpr unsigned long long kWaitNs = 1000000000ull;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -62,12 +69,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with parity `parity` of `bar` to complete.  Returns false
-// (after raising the abort flags) if it does not within kWaitCycles, or if
+// (after raising the abort flags) if it does not within `limit_ns`, or if
 // another thread of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* error_word, unsigned int code) {
+                                          unsigned int* error_word, unsigned int code,
+                                          unsigned long long limit_ns = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
+  const unsigned long long t0 = global_ns();
   while (true) {
     // try_wait suspends the thread for a while inside the hardware before it
     // reports "not yet", so the abort and clock checks run only every 8 tries
@@ -75,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int r = 0; r < 8; ++r)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(error_word, code);
       return false;
@@ -85,9 +93,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Bounded wait used during teardown: does not look at the abort flag.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
+  const unsigned long long t0 = global_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (global_ns() - t0 > kWaitNs) return false;
   }
   return true;
 }

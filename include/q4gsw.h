@@ -26,8 +26,11 @@
  * Conventions for every entry point
  *   - Every pointer argument is a DEVICE pointer on the current CUDA device,
  *     except where stated.  The caller allocates and owns every buffer; the
- *     library allocates no device memory and keeps no state besides a
- *     thread-local route string.
+ *     library allocates no device memory.  Its state: per host thread, the
+ *     route string (q4gsw_last_route) and the debug route pins
+ *     (q4gsw_debug_pin_routes); per device, one status word shared by every
+ *     stream and thread (see q4gsw_device_error_check) and caches of kernel
+ *     attributes and occupancy, filled on first use.
  *   - Dense operands are contiguous row-major.  fp16 values are passed as
  *     uint16_t bit patterns; outputs are fp32.
  *   - Device pointers must be 16-byte aligned (Q4GSW_ERR_ALIGN otherwise).
@@ -37,7 +40,8 @@
  *     error nothing is enqueued and outputs are untouched.  A launch failure
  *     reported by the CUDA runtime returns Q4GSW_ERR_CUDA.
  *   - No CPU fallback exists: every result is computed by this library's
- *     CUDA kernels.  Calls are thread-safe and re-entrant.
+ *     CUDA kernels.  Calls may be made from several host threads at once
+ *     (first-use caches are filled under std::call_once or atomics).
  *   - The compute calls launch with programmatic dependent launch: a call may
  *     start while the previous kernel on `stream` is still finishing.  It waits
  *     for that kernel before reading activations or writing outputs, but the
@@ -168,12 +172,16 @@ Q4GSW_API q4gsw_status q4gsw_embedding(const void *packed, int N, int K, int gro
 
 /*
  * Kernel health check.  Every wait inside this library's kernels is bounded
- * (about one second); a wait that runs out makes its kernel stop early and
- * record the event in a device-side status word instead of hanging.  This call
- * waits for `stream`, reads that word for the current device and clears it:
- * Q4GSW_ERR_TIMEOUT means the outputs of the calls since the previous check are
- * not valid; Q4GSW_ERR_INDEX that an embedding index was out of range (a
- * timeout takes precedence).  Returns Q4GSW_OK otherwise.
+ * (one second of wall-clock time); a wait that runs out makes its kernel stop
+ * early, leaving its outputs partly or wholly unwritten, and record the event
+ * in the device's status word instead of hanging.  The word is one per device,
+ * shared by every stream and host thread.  This call swaps it with zero in one
+ * atomic operation, ordered after the work already enqueued on `stream`, then
+ * waits for `stream`: events recorded later (by kernels of other streams) stay
+ * in the word for the next check.  Q4GSW_ERR_TIMEOUT means the outputs of the
+ * calls on this device since the previous check cannot be trusted;
+ * Q4GSW_ERR_INDEX that an embedding index was out of range (a timeout takes
+ * precedence).  Returns Q4GSW_OK otherwise.
  */
 Q4GSW_API q4gsw_status q4gsw_device_error_check(q4gsw_stream_t stream);
 
@@ -189,6 +197,30 @@ Q4GSW_API q4gsw_status q4gsw_unpack(const void *packed, int N, int K, int group_
  */
 Q4GSW_API q4gsw_status q4gsw_dequant(const void *packed, int N, int K, int group_size,
                            float *w32, uint16_t *w16, q4gsw_stream_t stream);
+
+/*
+ * Debug export (tests and tuning): pins the kernel route of the calls this
+ * host thread makes from now on.
+ *   gemv  calls with M <= 16:  0 automatic, 1 register-fed GEMV, 2 TMA-ring GEMV
+ *         (the input gradient has no TMA-ring/register choice other than these two)
+ *   gemm  calls with M > 16:   0 automatic, 1 tensor-memory GEMM, 2 shared-memory
+ *         GEMM (accumulators per CTA chosen), 3 shared-memory GEMM with one
+ *         128-token accumulator, 4 with two
+ * Every pinned route computes the same function (within the output bound).
+ * Values outside these ranges return Q4GSW_ERR_SHAPE and change nothing.
+ */
+Q4GSW_API q4gsw_status q4gsw_debug_pin_routes(int gemv, int gemm);
+
+/*
+ * Debug export (test of the failure path, no fault involved): enqueues one
+ * thread block whose single waiting thread waits, through the same bounded wait
+ * the compute kernels use, on a barrier that nothing completes.  After
+ * limit_us microseconds (1 .. 1000000) the wait gives up, records a time-out
+ * in the device status word and the kernel returns, so the following
+ * q4gsw_device_error_check returns Q4GSW_ERR_TIMEOUT.  Other limits return
+ * Q4GSW_ERR_SHAPE.
+ */
+Q4GSW_API q4gsw_status q4gsw_debug_wait_timeout(unsigned int limit_us, q4gsw_stream_t stream);
 
 /* Thread-local description of the kernel route the last call on this thread
  * enqueued (for example "gemv_fwd nt=1 splitk=8"); never NULL. */

@@ -21,7 +21,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = b.library()
     names = declared_functions()
-    assert len(names) == 12
+    assert len(names) == 14
     assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
     for n in names:
         assert hasattr(lib, n), n
@@ -117,3 +117,28 @@ def test_embedding_token_ids_are_seeded_and_in_range():
         assert ids.dtype == np.int32 and ids.shape == (sh.M,)
         assert ids.min() >= 0 and ids.max() < sh.N
         assert np.array_equal(ids, wl.embedding_indices(sh))
+
+
+def test_debug_route_pins_are_checked_and_thread_local():
+    import threading
+    lib = b.library()
+    assert lib.q4gsw_debug_pin_routes(3, 0) == 2          # gemv pin out of range
+    assert lib.q4gsw_debug_pin_routes(0, 5) == 2          # gemm pin out of range
+    assert lib.q4gsw_debug_pin_routes(-1, 0) == 2
+    for gemv in range(3):
+        for gemm in range(5):
+            assert lib.q4gsw_debug_pin_routes(gemv, gemm) == 0
+    seen = []
+    # a pin set on another thread does not leak into this one, nor the reverse:
+    # the other thread's status on a valid pin is OK whatever this thread pinned
+    t = threading.Thread(target=lambda: seen.append(lib.q4gsw_debug_pin_routes(1, 1)))
+    t.start()
+    t.join()
+    assert seen == [0]
+    assert lib.q4gsw_debug_pin_routes(0, 0) == 0
+
+
+def test_wait_probe_limit_is_checked_on_the_host():
+    lib = b.library()
+    assert lib.q4gsw_debug_wait_timeout(0, None) == 2
+    assert lib.q4gsw_debug_wait_timeout(1000001, None) == 2

@@ -208,10 +208,11 @@ def test_odd_weight_shapes(N, K, gs):
 
 
 @pytest.fixture(params=["tma", "reg"])
-def gemv_variant(request, monkeypatch):
-    """Pins the forward GEMV: TMA-ring weight stream or register-fed."""
-    monkeypatch.setenv("Q4GSW_GEMV_KIND", request.param)
-    return request.param
+def gemv_variant(request):
+    """Pins the GEMV: TMA-ring weight stream or register-fed (q4gsw_debug_pin_routes)."""
+    q().q4gsw_debug_pin_routes(gemv=request.param)
+    yield request.param
+    q().q4gsw_debug_pin_routes()
 
 
 @pytest.mark.parametrize("M,N,K,gs", [(1, 64, 128, 32), (3, 136, 320, 16), (8, 1032, 576, 64), (9, 72, 256, 128),
@@ -250,14 +251,12 @@ def test_non_default_stream():
 
 # ----------------------------------------------------------------------------- tcgen05 GEMM routes
 @pytest.fixture(params=["ts", "ss1", "ss2"])
-def gemm_variant(request, monkeypatch):
+def gemm_variant(request):
     """Pins the GEMM route: weight tile in tensor memory (ts, the default), or
     dequantised into shared memory with one or two 128-token accumulators."""
-    v = request.param
-    monkeypatch.setenv("Q4GSW_GEMM_KIND", v[:2])
-    if v.startswith("ss"):
-        monkeypatch.setenv("Q4GSW_GEMM_MSUB", v[2])
-    return v
+    q().q4gsw_debug_pin_routes(gemm=request.param)
+    yield request.param
+    q().q4gsw_debug_pin_routes()
 
 
 def _route_ok(route, direction, variant):
@@ -279,9 +278,8 @@ def test_gemm_route_tails(M, N, K, gs, gemm_variant):
     assert _route_ok(route, "bwd", gemm_variant), route
 
 
-def test_gemm_default_routes(monkeypatch):
-    monkeypatch.delenv("Q4GSW_GEMM_KIND", raising=False)
-    monkeypatch.delenv("Q4GSW_GEMM_MSUB", raising=False)
+def test_gemm_default_routes():
+    q().q4gsw_debug_pin_routes()
     inp = wl.random_inputs(100, 256, 256, 32, seed=5)
     check_fwd(inp, 32)
     route = q().q4gsw_last_route()
@@ -292,12 +290,14 @@ def test_gemm_default_routes(monkeypatch):
     assert route.startswith("tcgen05_gemm_bwd"), route   # above 512 tokens: shared-memory route
 
 
-def test_ss_variant_choice_is_automatic(monkeypatch):
-    monkeypatch.setenv("Q4GSW_GEMM_KIND", "ss")
-    monkeypatch.delenv("Q4GSW_GEMM_MSUB", raising=False)
-    inp = wl.random_inputs(100, 256, 256, 32, seed=5)
-    check_fwd(inp, 32)
-    assert "tile=128x" in q().q4gsw_last_route()   # fewer than 129 tokens: one accumulator
+def test_ss_variant_choice_is_automatic():
+    q().q4gsw_debug_pin_routes(gemm="ss")
+    try:
+        inp = wl.random_inputs(100, 256, 256, 32, seed=5)
+        check_fwd(inp, 32)
+        assert "tile=128x" in q().q4gsw_last_route()   # fewer than 129 tokens: one accumulator
+    finally:
+        q().q4gsw_debug_pin_routes()
 
 
 def test_gemm_split_k_cluster_reduction(gemm_variant):
