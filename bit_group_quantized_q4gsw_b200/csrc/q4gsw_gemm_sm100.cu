@@ -378,7 +378,7 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       cluster.sync();
       const int r = (int)cluster.block_rank();
       const int row_b = r * BM / S, row_e = (r + 1) * BM / S;
-      if (!*abort_flag) {
+      if (!cluster_any_abort(cluster, &ctl->abort, S)) {
         for (int idx = threadIdx.x; idx < (row_e - row_b) * 64; idx += kThreads) {
           const int row = row_b + (idx >> 6), chunk = idx & 63;
           const int m = mb + row, n = n0 + 4 * chunk;

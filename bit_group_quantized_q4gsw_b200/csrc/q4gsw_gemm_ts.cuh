@@ -370,7 +370,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     {
       const int rk = S > 1 ? (int)cluster.block_rank() : 0;
       const int row_b = rk * args.bt / S, row_e = (rk + 1) * args.bt / S;
-      if (!*abort_flag) {
+      if (!(S > 1 ? cluster_any_abort(cluster, &ctl->abort, S) : *abort_flag)) {
         for (int idx = threadIdx.x; idx < (row_e - row_b) * (BW / 4); idx += kThreads) {
           const int row = row_b + idx / (BW / 4), c4 = idx % (BW / 4);
           const int m = t0 + row, f = f0 + 4 * c4;

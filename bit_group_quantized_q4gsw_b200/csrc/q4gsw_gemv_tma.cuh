@@ -265,7 +265,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   cg::cluster_group cluster = cg::this_cluster();
   if (S > 1) cluster.sync();
   else __syncthreads();
-  if (!*abort_flag) {
+  if (!(S > 1 ? cluster_any_abort(cluster, &ctl->abort, S) : *abort_flag)) {
     const int rk = S > 1 ? (int)cluster.block_rank() : 0;
     const int tb = rk * Mz / S, te = (rk + 1) * Mz / S;
     for (int e = threadIdx.x; e < (te - tb) * 64; e += kThreads) {
@@ -499,7 +499,7 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   cg::cluster_group cluster = cg::this_cluster();
   if (S > 1) cluster.sync();
   else __syncthreads();
-  if (!*abort_flag) {
+  if (!(S > 1 ? cluster_any_abort(cluster, &ctl->abort, S) : *abort_flag)) {
     const int rk = S > 1 ? (int)cluster.block_rank() : 0;
     const int tb = rk * Mz / S, te = (rk + 1) * Mz / S;
     const int kw = min(128, K - kbase);

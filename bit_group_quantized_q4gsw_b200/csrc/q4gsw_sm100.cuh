@@ -1,25 +1,23 @@
 // q4gsw_sm100.cuh - thin inline-PTX wrappers for the Blackwell (sm_100a)
 // features the GEMM route uses: mbarriers, TMA tensor loads, tensor memory
 // (tcgen05.alloc / ld / dealloc), tcgen05.mma with shared-memory descriptors.
-// Every wait is bounded: past kWaitNs of wall-clock time the waiter raises the
-// CTA's abort flag and the library's device error word, and returns false.
+// Every wait is bounded (kWaitNs): past it the waiter raises the CTA's abort
+// flag and the library's device error word, and returns false.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cstdint>
 
 namespace q4gsw {
 namespace sm100 {
 
-// Wall-clock bound of every wait (nanoseconds of %globaltimer): far above any
-// legitimate wait of this library's kernels, and independent of the SM clock.
+// Bound of every wait, in nanoseconds: far above any legitimate wait of this
+// library's kernels.  It is counted in SM cycles (clock64, monotonic on its
+// SM) at 2 cycles per nanosecond; the SM clock never exceeds 2 GHz on B200, so
+// the wall-clock time before a wait gives up is at least the bound.
 constexpr unsigned long long kWaitNs = 1000000000ull;
-
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
+constexpr long long kCyclesPerNs = 2;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -75,7 +73,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           unsigned int* error_word, unsigned int code,
                                           unsigned long long limit_ns = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
+  const long long limit = (long long)limit_ns * kCyclesPerNs;
+  const long long t0 = clock64();
   while (true) {
     // try_wait suspends the thread for a while inside the hardware before it
     // reports "not yet", so the abort and clock checks run only every 8 tries
@@ -83,7 +82,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int r = 0; r < 8; ++r)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > limit_ns) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       atomicOr(error_word, code);
       return false;
@@ -93,11 +92,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Bounded wait used during teardown: does not look at the abort flag.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = global_ns();
+  const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitNs) return false;
+    if (clock64() - t0 > (long long)kWaitNs * kCyclesPerNs) return false;
   }
   return true;
+}
+
+// Called between two cluster barriers (every CTA's main loop is over): true if
+// the wait of any CTA of the cluster ran out, so that no CTA stores sums that
+// include another CTA's unfinished partial tile.
+__device__ __forceinline__ bool cluster_any_abort(cooperative_groups::cluster_group& cluster, int* abort_flag,
+                                                  int S) {
+  int any = 0;
+  for (int q = 0; q < S; ++q) any |= *static_cast<volatile int*>(cluster.map_shared_rank(abort_flag, q));
+  return any != 0;
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {

@@ -24,16 +24,18 @@ def run_fwd(inp, gs):
     blob = pack_on_gpu(inp, gs)
     N, K = inp.codes.shape
     y = q().q4gsw_linear_fwd(blob, N, K, gs, cuda(inp.x))
-    torch.cuda.synchronize()
-    return y.cpu().numpy(), q().q4gsw_last_route()
+    route = q().q4gsw_last_route()
+    q().q4gsw_device_error_check()   # a wait that ran out is reported as such, not as a wrong number
+    return y.cpu().numpy(), route
 
 
 def run_bwd(inp, gs):
     blob = pack_on_gpu(inp, gs)
     N, K = inp.codes.shape
     dx = q().q4gsw_linear_bwd_input(blob, N, K, gs, cuda(inp.d_out))
-    torch.cuda.synchronize()
-    return dx.cpu().numpy(), q().q4gsw_last_route()
+    route = q().q4gsw_last_route()
+    q().q4gsw_device_error_check()
+    return dx.cpu().numpy(), route
 
 
 def check_fwd(inp, gs, rows=None):

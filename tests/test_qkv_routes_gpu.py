@@ -31,8 +31,9 @@ def run_qkv(inp, splits, gs):
     Nq, Nk, Nv = splits
     blob = pack_on_gpu(inp, gs)
     outs = q().q4gsw_qkv_fwd(blob, Nq, Nk, Nv, inp.codes.shape[1], gs, cuda(inp.x))
-    torch.cuda.synchronize()
-    return [t.cpu().numpy() for t in outs], q().q4gsw_last_route()
+    route = q().q4gsw_last_route()
+    q().q4gsw_device_error_check()
+    return [t.cpu().numpy() for t in outs], route
 
 
 def check_route(M, split_name, gemv="auto", gemm="auto", route_prefix=""):
