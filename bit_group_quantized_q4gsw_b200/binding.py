@@ -36,6 +36,13 @@ SIGNATURES = [
     ("q4gsw_device_error_check", _I, [_VP]),
     ("q4gsw_unpack", _I, [_VP, _I, _I, _I, _VP, _VP]),
     ("q4gsw_dequant", _I, [_VP, _I, _I, _I, _VP, _VP, _VP]),
+    ("q4gsw_packed_bytes_f32s", _SZ, [_I, _I, _I]),
+    ("q4gsw_prepack_f32s", _I, [_VP, _VP, _I, _I, _I, _VP, _SZ, _VP]),
+    ("q4gsw_linear_fwd_f32s", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
+    ("q4gsw_linear_bwd_input_f32s", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
+    ("q4gsw_qkv_fwd_f32s", _I, [_VP, _I, _I, _I, _I, _I, _VP, _I, _VP, _VP, _VP, _VP]),
+    ("q4gsw_embedding_f32s", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
+    ("q4gsw_dequant_f32s", _I, [_VP, _I, _I, _I, _VP, _VP, _VP]),
     ("q4gsw_debug_pin_routes", _I, [_I, _I]),
     ("q4gsw_debug_wait_timeout", _I, [ctypes.c_uint, _VP]),
     ("q4gsw_last_route", ctypes.c_char_p, []),
@@ -118,67 +125,84 @@ def q4gsw_status_str(status: int) -> str:
 
 def q4gsw_prepack(codes: torch.Tensor, scales: torch.Tensor, group_size: int,
                   packed: torch.Tensor | None = None) -> torch.Tensor:
-    """codes uint8 [N, K] (0..15), scales fp16 [K/gs, N] -> packed uint8 blob."""
+    """codes uint8 [N, K] (0..15), scales fp16 [K/gs, N] -> packed uint8 blob.
+
+    fp32 scales select the fp32-scale packer (layout version 2, q4gsw_prepack_f32s);
+    its blob goes to the *_f32s compute functions."""
     lib = library()
     N, K = codes.shape
-    nbytes = lib.q4gsw_packed_bytes(N, K, group_size)
+    f32s = scales.dtype == torch.float32
+    nbytes = (lib.q4gsw_packed_bytes_f32s if f32s else lib.q4gsw_packed_bytes)(N, K, group_size)
     if packed is None:
         packed = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=codes.device)
-    st = lib.q4gsw_prepack(_dev(codes, torch.uint8, "codes", 2), _dev(scales, torch.float16, "scales", 2),
-                           N, K, group_size, _dev(packed, torch.uint8, "packed"), packed.numel(), _stream(codes))
-    _check("q4gsw_prepack", st)
+    fn, name = (lib.q4gsw_prepack_f32s, "q4gsw_prepack_f32s") if f32s else (lib.q4gsw_prepack, "q4gsw_prepack")
+    st = fn(_dev(codes, torch.uint8, "codes", 2), _dev(scales, torch.float32 if f32s else torch.float16, "scales", 2),
+            N, K, group_size, _dev(packed, torch.uint8, "packed"), packed.numel(), _stream(codes))
+    _check(name, st)
     return packed
 
 
+def q4gsw_prepack_f32s(codes: torch.Tensor, scales: torch.Tensor, group_size: int,
+                       packed: torch.Tensor | None = None) -> torch.Tensor:
+    """codes uint8 [N, K] (0..15), scales fp32 [K/gs, N] -> layout-version-2 blob."""
+    if scales.dtype != torch.float32:
+        raise TypeError("q4gsw_prepack_f32s takes fp32 scales")
+    return q4gsw_prepack(codes, scales, group_size, packed)
+
+
 def q4gsw_linear_fwd(packed: torch.Tensor, N: int, K: int, group_size: int, x: torch.Tensor,
-                     y: torch.Tensor | None = None) -> torch.Tensor:
-    """y[M, N] = x[M, K] @ dequant(W)[N, K]^T in fp32."""
+                     y: torch.Tensor | None = None, f32s: bool = False) -> torch.Tensor:
+    """y[M, N] = x[M, K] @ dequant(W)[N, K]^T in fp32 (f32s: a layout-version-2 blob)."""
     M = x.shape[0]
     if y is None:
         y = torch.empty((M, N), dtype=torch.float32, device=x.device)
-    st = library().q4gsw_linear_fwd(_dev(packed, torch.uint8, "packed"), N, K, group_size,
-                                    _dev(x, torch.float16, "x", 2), M, _dev(y, torch.float32, "y", 2), _stream(x))
-    _check("q4gsw_linear_fwd", st)
+    name = "q4gsw_linear_fwd_f32s" if f32s else "q4gsw_linear_fwd"
+    st = getattr(library(), name)(_dev(packed, torch.uint8, "packed"), N, K, group_size,
+                                  _dev(x, torch.float16, "x", 2), M, _dev(y, torch.float32, "y", 2), _stream(x))
+    _check(name, st)
     return y
 
 
 def q4gsw_linear_bwd_input(packed: torch.Tensor, N: int, K: int, group_size: int, d_out: torch.Tensor,
-                           d_x: torch.Tensor | None = None) -> torch.Tensor:
-    """d_x[M, K] = d_out[M, N] @ dequant(W)[N, K] in fp32."""
+                           d_x: torch.Tensor | None = None, f32s: bool = False) -> torch.Tensor:
+    """d_x[M, K] = d_out[M, N] @ dequant(W)[N, K] in fp32 (f32s: a layout-version-2 blob)."""
     M = d_out.shape[0]
     if d_x is None:
         d_x = torch.empty((M, K), dtype=torch.float32, device=d_out.device)
-    st = library().q4gsw_linear_bwd_input(_dev(packed, torch.uint8, "packed"), N, K, group_size,
-                                          _dev(d_out, torch.float16, "d_out", 2), M,
-                                          _dev(d_x, torch.float32, "d_x", 2), _stream(d_out))
-    _check("q4gsw_linear_bwd_input", st)
+    name = "q4gsw_linear_bwd_input_f32s" if f32s else "q4gsw_linear_bwd_input"
+    st = getattr(library(), name)(_dev(packed, torch.uint8, "packed"), N, K, group_size,
+                                  _dev(d_out, torch.float16, "d_out", 2), M,
+                                  _dev(d_x, torch.float32, "d_x", 2), _stream(d_out))
+    _check(name, st)
     return d_x
 
 
 def q4gsw_qkv_fwd(packed_qkv: torch.Tensor, Nq: int, Nk: int, Nv: int, K: int, group_size: int,
-                  x: torch.Tensor, outs=None):
+                  x: torch.Tensor, outs=None, f32s: bool = False):
     """Three projections of x from one packed [Nq+Nk+Nv, K] weight -> (y_q, y_k, y_v)."""
     M = x.shape[0]
     if outs is None:
         outs = tuple(torch.empty((M, n), dtype=torch.float32, device=x.device) for n in (Nq, Nk, Nv))
     yq, yk, yv = outs
-    st = library().q4gsw_qkv_fwd(_dev(packed_qkv, torch.uint8, "packed_qkv"), Nq, Nk, Nv, K, group_size,
-                                 _dev(x, torch.float16, "x", 2), M, _dev(yq, torch.float32, "y_q", 2),
-                                 _dev(yk, torch.float32, "y_k", 2), _dev(yv, torch.float32, "y_v", 2), _stream(x))
-    _check("q4gsw_qkv_fwd", st)
+    name = "q4gsw_qkv_fwd_f32s" if f32s else "q4gsw_qkv_fwd"
+    st = getattr(library(), name)(_dev(packed_qkv, torch.uint8, "packed_qkv"), Nq, Nk, Nv, K, group_size,
+                                  _dev(x, torch.float16, "x", 2), M, _dev(yq, torch.float32, "y_q", 2),
+                                  _dev(yk, torch.float32, "y_k", 2), _dev(yv, torch.float32, "y_v", 2), _stream(x))
+    _check(name, st)
     return yq, yk, yv
 
 
 def q4gsw_embedding(packed: torch.Tensor, N: int, K: int, group_size: int, indices: torch.Tensor,
-                    out: torch.Tensor | None = None) -> torch.Tensor:
+                    out: torch.Tensor | None = None, f32s: bool = False) -> torch.Tensor:
     """out[T, K] = dequant(W)[indices] in fp32 (indices int32 [T] on the device, each in [0, N))."""
     T = indices.shape[0]
     if out is None:
         out = torch.empty((T, K), dtype=torch.float32, device=indices.device)
-    st = library().q4gsw_embedding(_dev(packed, torch.uint8, "packed"), N, K, group_size,
-                                   _dev(indices, torch.int32, "indices", 1), T,
-                                   _dev(out, torch.float32, "out", 2), _stream(indices))
-    _check("q4gsw_embedding", st)
+    name = "q4gsw_embedding_f32s" if f32s else "q4gsw_embedding"
+    st = getattr(library(), name)(_dev(packed, torch.uint8, "packed"), N, K, group_size,
+                                  _dev(indices, torch.int32, "indices", 1), T,
+                                  _dev(out, torch.float32, "out", 2), _stream(indices))
+    _check(name, st)
     return out
 
 
@@ -216,12 +240,13 @@ def q4gsw_unpack(packed: torch.Tensor, N: int, K: int, group_size: int) -> torch
 
 
 def q4gsw_dequant(packed: torch.Tensor, N: int, K: int, group_size: int, want_w32: bool = True,
-                  want_w16: bool = True):
-    """(w32 fp32 [N, K] exact, w16 fp16 [N, K] tensor-core operand); either may be None."""
+                  want_w16: bool = True, f32s: bool = False):
+    """(w32 fp32 [N, K], w16 fp16 [N, K] tensor-core operand); either may be None."""
     w32 = torch.empty((N, K), dtype=torch.float32, device=packed.device) if want_w32 else None
     w16 = torch.empty((N, K), dtype=torch.float16, device=packed.device) if want_w16 else None
-    st = library().q4gsw_dequant(_dev(packed, torch.uint8, "packed"), N, K, group_size,
-                                 None if w32 is None else w32.data_ptr(),
-                                 None if w16 is None else w16.data_ptr(), _stream(packed))
-    _check("q4gsw_dequant", st)
+    name = "q4gsw_dequant_f32s" if f32s else "q4gsw_dequant"
+    st = getattr(library(), name)(_dev(packed, torch.uint8, "packed"), N, K, group_size,
+                                  None if w32 is None else w32.data_ptr(),
+                                  None if w16 is None else w16.data_ptr(), _stream(packed))
+    _check(name, st)
     return w32, w16

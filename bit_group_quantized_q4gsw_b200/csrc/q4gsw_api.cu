@@ -76,6 +76,107 @@ constexpr int kGemvMaxM = 16;
 
 }  // namespace
 
+namespace {
+
+q4gsw_status prepack_impl(const uint8_t* codes, const void* scales, int N, int K, int group_size, bool f32s,
+                          void* packed, size_t packed_bytes, q4gsw_stream_t stream) {
+  if (!codes || !scales || !packed) return Q4GSW_ERR_NULL;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(packed)) return Q4GSW_ERR_ALIGN;
+  if (packed_bytes < layout_of(N, K, group_size, f32s ? 4 : 2).total_bytes) return Q4GSW_ERR_SIZE;
+  uint32_t flag = 0;
+  set_route(f32s ? "prepack_f32s" : "prepack");
+  st = from_cuda(launch_prepack(codes, scales, N, K, group_size, f32s, packed, stream, &flag));
+  if (st != Q4GSW_OK) return st;
+  return flag ? Q4GSW_ERR_CODE_RANGE : Q4GSW_OK;
+}
+
+q4gsw_status linear_fwd_impl(const void* packed, int N, int K, int group_size, bool f32s, const uint16_t* x, int M,
+                             float* y, q4gsw_stream_t stream) {
+  if (M < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed || !x || !y) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y)) return Q4GSW_ERR_ALIGN;
+  char route[160];
+  cudaError_t e = M <= kGemvMaxM
+                      ? launch_gemv_fwd(packed, N, K, group_size, f32s, x, M, single_output(y, N), stream, route,
+                                        sizeof(route))
+                      : launch_gemm_fwd(packed, N, K, group_size, f32s, x, M, single_output(y, N), stream, route,
+                                        sizeof(route));
+  set_route(route);
+  return from_cuda(e);
+}
+
+q4gsw_status linear_bwd_impl(const void* packed, int N, int K, int group_size, bool f32s, const uint16_t* d_out, int M,
+                             float* d_x, q4gsw_stream_t stream) {
+  if (M < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed || !d_out || !d_x) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(d_out) || !aligned16(d_x)) return Q4GSW_ERR_ALIGN;
+  char route[160];
+  cudaError_t e = M <= kGemvMaxM
+                      ? launch_gemv_bwd(packed, N, K, group_size, f32s, d_out, M, d_x, stream, route, sizeof(route))
+                      : launch_gemm_bwd(packed, N, K, group_size, f32s, d_out, M, d_x, stream, route, sizeof(route));
+  set_route(route);
+  return from_cuda(e);
+}
+
+q4gsw_status qkv_fwd_impl(const void* packed_qkv, int Nq, int Nk, int Nv, int K, int group_size, bool f32s,
+                          const uint16_t* x, int M, float* y_q, float* y_k, float* y_v, q4gsw_stream_t stream) {
+  if (M < 0 || Nq <= 0 || Nk <= 0 || Nv <= 0) return Q4GSW_ERR_SHAPE;
+  if ((long long)Nq + Nk + Nv > 0x7fffffffLL) return Q4GSW_ERR_SHAPE;
+  const int N = Nq + Nk + Nv;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (Nq % 4 || Nk % 4 || Nv % 4) return Q4GSW_ERR_SHAPE;
+  if (Nq % 8 || Nk % 8 || Nv % 8) return Q4GSW_ERR_ALIGN;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed_qkv || !x || !y_q || !y_k || !y_v) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed_qkv) || !aligned16(x) || !aligned16(y_q) || !aligned16(y_k) || !aligned16(y_v))
+    return Q4GSW_ERR_ALIGN;
+  OutSplit out{y_q, y_k, y_v, Nq, Nq + Nk, N};
+  char route[120];
+  cudaError_t e = M <= kGemvMaxM
+                      ? launch_gemv_fwd(packed_qkv, N, K, group_size, f32s, x, M, out, stream, route, sizeof(route))
+                      : launch_gemm_fwd(packed_qkv, N, K, group_size, f32s, x, M, out, stream, route, sizeof(route));
+  char full[160];
+  snprintf(full, sizeof(full), "qkv %s", route);
+  set_route(full);
+  return from_cuda(e);
+}
+
+q4gsw_status embedding_impl(const void* packed, int N, int K, int group_size, bool f32s, const int32_t* indices, int T,
+                            float* out, q4gsw_stream_t stream) {
+  if (T < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (T == 0) {
+    set_route("empty");
+    return Q4GSW_OK;
+  }
+  if (!packed || !indices || !out) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(out) || (reinterpret_cast<uintptr_t>(indices) & 3u)) return Q4GSW_ERR_ALIGN;
+  set_route("embedding_gather launches=1");
+  return from_cuda(launch_embedding(packed, N, K, group_size, f32s, indices, T, out, stream));
+}
+
+q4gsw_status dequant_impl(const void* packed, int N, int K, int group_size, bool f32s, float* w32, uint16_t* w16,
+                          q4gsw_stream_t stream) {
+  if (!packed || (!w32 && !w16)) return Q4GSW_ERR_NULL;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (!aligned16(packed) || (w32 && !aligned16(w32)) || (w16 && !aligned16(w16))) return Q4GSW_ERR_ALIGN;
+  set_route("dequant");
+  return from_cuda(launch_dequant(packed, N, K, group_size, f32s, w32, w16, stream));
+}
+
+}  // namespace
+
 extern "C" {
 
 int q4gsw_layout_version(void) { return kLayoutVersion; }
@@ -83,6 +184,11 @@ int q4gsw_layout_version(void) { return kLayoutVersion; }
 size_t q4gsw_packed_bytes(int N, int K, int group_size) {
   if (check_weight_shape(N, K, group_size) != Q4GSW_OK) return 0;
   return layout_of(N, K, group_size).total_bytes;
+}
+
+size_t q4gsw_packed_bytes_f32s(int N, int K, int group_size) {
+  if (check_weight_shape(N, K, group_size) != Q4GSW_OK) return 0;
+  return layout_of(N, K, group_size, 4).total_bytes;
 }
 
 const char* q4gsw_last_route(void) { return g_route; }
@@ -105,74 +211,44 @@ const char* q4gsw_status_str(q4gsw_status s) {
 
 q4gsw_status q4gsw_prepack(const uint8_t* codes, const uint16_t* scales, int N, int K, int group_size,
                            void* packed, size_t packed_bytes, q4gsw_stream_t stream) {
-  if (!codes || !scales || !packed) return Q4GSW_ERR_NULL;
-  q4gsw_status st = check_weight_shape(N, K, group_size);
-  if (st != Q4GSW_OK) return st;
-  if (!aligned16(codes) || !aligned16(scales) || !aligned16(packed)) return Q4GSW_ERR_ALIGN;
-  if (packed_bytes < layout_of(N, K, group_size).total_bytes) return Q4GSW_ERR_SIZE;
-  uint32_t flag = 0;
-  set_route("prepack");
-  st = from_cuda(launch_prepack(codes, scales, N, K, group_size, packed, stream, &flag));
-  if (st != Q4GSW_OK) return st;
-  return flag ? Q4GSW_ERR_CODE_RANGE : Q4GSW_OK;
+  return prepack_impl(codes, scales, N, K, group_size, false, packed, packed_bytes, stream);
+}
+
+q4gsw_status q4gsw_prepack_f32s(const uint8_t* codes, const float* scales, int N, int K, int group_size,
+                                void* packed, size_t packed_bytes, q4gsw_stream_t stream) {
+  return prepack_impl(codes, scales, N, K, group_size, true, packed, packed_bytes, stream);
 }
 
 q4gsw_status q4gsw_linear_fwd(const void* packed, int N, int K, int group_size, const uint16_t* x, int M,
                               float* y, q4gsw_stream_t stream) {
-  if (M < 0) return Q4GSW_ERR_SHAPE;
-  q4gsw_status st = check_weight_shape(N, K, group_size);
-  if (st != Q4GSW_OK) return st;
-  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
-  if (!packed || !x || !y) return Q4GSW_ERR_NULL;
-  if (!aligned16(packed) || !aligned16(x) || !aligned16(y)) return Q4GSW_ERR_ALIGN;
-  char route[160];
-  cudaError_t e = M <= kGemvMaxM
-                      ? launch_gemv_fwd(packed, N, K, group_size, x, M, single_output(y, N), stream, route,
-                                        sizeof(route))
-                      : launch_gemm_fwd(packed, N, K, group_size, x, M, single_output(y, N), stream, route,
-                                        sizeof(route));
-  set_route(route);
-  return from_cuda(e);
+  return linear_fwd_impl(packed, N, K, group_size, false, x, M, y, stream);
+}
+
+q4gsw_status q4gsw_linear_fwd_f32s(const void* packed, int N, int K, int group_size, const uint16_t* x, int M,
+                                   float* y, q4gsw_stream_t stream) {
+  return linear_fwd_impl(packed, N, K, group_size, true, x, M, y, stream);
 }
 
 q4gsw_status q4gsw_linear_bwd_input(const void* packed, int N, int K, int group_size, const uint16_t* d_out,
                                     int M, float* d_x, q4gsw_stream_t stream) {
-  if (M < 0) return Q4GSW_ERR_SHAPE;
-  q4gsw_status st = check_weight_shape(N, K, group_size);
-  if (st != Q4GSW_OK) return st;
-  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
-  if (!packed || !d_out || !d_x) return Q4GSW_ERR_NULL;
-  if (!aligned16(packed) || !aligned16(d_out) || !aligned16(d_x)) return Q4GSW_ERR_ALIGN;
-  char route[160];
-  cudaError_t e = M <= kGemvMaxM
-                      ? launch_gemv_bwd(packed, N, K, group_size, d_out, M, d_x, stream, route, sizeof(route))
-                      : launch_gemm_bwd(packed, N, K, group_size, d_out, M, d_x, stream, route, sizeof(route));
-  set_route(route);
-  return from_cuda(e);
+  return linear_bwd_impl(packed, N, K, group_size, false, d_out, M, d_x, stream);
+}
+
+q4gsw_status q4gsw_linear_bwd_input_f32s(const void* packed, int N, int K, int group_size, const uint16_t* d_out,
+                                         int M, float* d_x, q4gsw_stream_t stream) {
+  return linear_bwd_impl(packed, N, K, group_size, true, d_out, M, d_x, stream);
 }
 
 q4gsw_status q4gsw_qkv_fwd(const void* packed_qkv, int Nq, int Nk, int Nv, int K, int group_size,
                            const uint16_t* x, int M, float* y_q, float* y_k, float* y_v,
                            q4gsw_stream_t stream) {
-  if (M < 0 || Nq <= 0 || Nk <= 0 || Nv <= 0) return Q4GSW_ERR_SHAPE;
-  if ((long long)Nq + Nk + Nv > 0x7fffffffLL) return Q4GSW_ERR_SHAPE;
-  const int N = Nq + Nk + Nv;
-  q4gsw_status st = check_weight_shape(N, K, group_size);
-  if (st != Q4GSW_OK) return st;
-  if (Nq % 4 || Nk % 4 || Nv % 4) return Q4GSW_ERR_SHAPE;
-  if (Nq % 8 || Nk % 8 || Nv % 8) return Q4GSW_ERR_ALIGN;
-  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
-  if (!packed_qkv || !x || !y_q || !y_k || !y_v) return Q4GSW_ERR_NULL;
-  if (!aligned16(packed_qkv) || !aligned16(x) || !aligned16(y_q) || !aligned16(y_k) || !aligned16(y_v))
-    return Q4GSW_ERR_ALIGN;
-  OutSplit out{y_q, y_k, y_v, Nq, Nq + Nk, N};
-  char route[120];
-  cudaError_t e = M <= kGemvMaxM ? launch_gemv_fwd(packed_qkv, N, K, group_size, x, M, out, stream, route, sizeof(route))
-                                 : launch_gemm_fwd(packed_qkv, N, K, group_size, x, M, out, stream, route, sizeof(route));
-  char full[160];
-  snprintf(full, sizeof(full), "qkv %s", route);
-  set_route(full);
-  return from_cuda(e);
+  return qkv_fwd_impl(packed_qkv, Nq, Nk, Nv, K, group_size, false, x, M, y_q, y_k, y_v, stream);
+}
+
+q4gsw_status q4gsw_qkv_fwd_f32s(const void* packed_qkv, int Nq, int Nk, int Nv, int K, int group_size,
+                                const uint16_t* x, int M, float* y_q, float* y_k, float* y_v,
+                                q4gsw_stream_t stream) {
+  return qkv_fwd_impl(packed_qkv, Nq, Nk, Nv, K, group_size, true, x, M, y_q, y_k, y_v, stream);
 }
 
 q4gsw_status q4gsw_device_error_check(q4gsw_stream_t stream) {
@@ -185,17 +261,12 @@ q4gsw_status q4gsw_device_error_check(q4gsw_stream_t stream) {
 
 q4gsw_status q4gsw_embedding(const void* packed, int N, int K, int group_size, const int32_t* indices, int T,
                              float* out, q4gsw_stream_t stream) {
-  if (T < 0) return Q4GSW_ERR_SHAPE;
-  q4gsw_status st = check_weight_shape(N, K, group_size);
-  if (st != Q4GSW_OK) return st;
-  if (T == 0) {
-    set_route("empty");
-    return Q4GSW_OK;
-  }
-  if (!packed || !indices || !out) return Q4GSW_ERR_NULL;
-  if (!aligned16(packed) || !aligned16(out) || (reinterpret_cast<uintptr_t>(indices) & 3u)) return Q4GSW_ERR_ALIGN;
-  set_route("embedding_gather launches=1");
-  return from_cuda(launch_embedding(packed, N, K, group_size, indices, T, out, stream));
+  return embedding_impl(packed, N, K, group_size, false, indices, T, out, stream);
+}
+
+q4gsw_status q4gsw_embedding_f32s(const void* packed, int N, int K, int group_size, const int32_t* indices, int T,
+                                  float* out, q4gsw_stream_t stream) {
+  return embedding_impl(packed, N, K, group_size, true, indices, T, out, stream);
 }
 
 q4gsw_status q4gsw_debug_pin_routes(int gemv, int gemm) {
@@ -223,12 +294,12 @@ q4gsw_status q4gsw_unpack(const void* packed, int N, int K, int group_size, uint
 
 q4gsw_status q4gsw_dequant(const void* packed, int N, int K, int group_size, float* w32, uint16_t* w16,
                            q4gsw_stream_t stream) {
-  if (!packed || (!w32 && !w16)) return Q4GSW_ERR_NULL;
-  q4gsw_status st = check_weight_shape(N, K, group_size);
-  if (st != Q4GSW_OK) return st;
-  if (!aligned16(packed) || (w32 && !aligned16(w32)) || (w16 && !aligned16(w16))) return Q4GSW_ERR_ALIGN;
-  set_route("dequant");
-  return from_cuda(launch_dequant(packed, N, K, group_size, w32, w16, stream));
+  return dequant_impl(packed, N, K, group_size, false, w32, w16, stream);
+}
+
+q4gsw_status q4gsw_dequant_f32s(const void* packed, int N, int K, int group_size, float* w32, uint16_t* w16,
+                                q4gsw_stream_t stream) {
+  return dequant_impl(packed, N, K, group_size, true, w32, w16, stream);
 }
 
 }  // extern "C"

@@ -8,7 +8,7 @@
 //           (same PR, "Key changes": even-N low nibble, odd-N high), placed
 //           inside its 64-byte block: column r = 16 i + 4 t + e goes to word
 //           slot 4 t + i, byte slot {0, 2, 1, 3}[e];
-//   scales  fp16 [G][N] at round_up(N/2*K, 256);
+//   scales  fp16 [G][N] at round_up(N/2*K, 256) (version 2: fp32 [G][N]);
 //   trailer 64 bytes at round_up(scales end, 256).
 //
 // Why this byte order: a 16-byte load at offset 16 t of a block gives word i
@@ -27,7 +27,8 @@ namespace q4gsw {
 constexpr int kRegionAlign = 256;
 constexpr int kTrailerBytes = 64;
 constexpr uint32_t kTrailerMagic = 0x53473451u;  // "Q4GS"
-constexpr int kLayoutVersion = 1;
+constexpr int kLayoutVersion = 1;      // fp16 scales
+constexpr int kLayoutVersionF32S = 2;  // fp32 scales
 
 struct Layout {
   size_t codes_bytes;
@@ -39,11 +40,13 @@ struct Layout {
 
 __host__ __device__ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline Layout layout_of(int N, int K, int gs) {
+// sbytes: bytes per scale, 2 (fp16, layout version 1) or 4 (fp32, version 2;
+// the codes region is the same in both versions)
+__host__ __device__ inline Layout layout_of(int N, int K, int gs, int sbytes = 2) {
   Layout L;
   L.codes_bytes = size_t(N / 2) * size_t(K);
   L.scales_offset = round_up(L.codes_bytes, kRegionAlign);
-  L.scales_bytes = size_t(2) * size_t(K / gs) * size_t(N);
+  L.scales_bytes = size_t(sbytes) * size_t(K / gs) * size_t(N);
   L.trailer_offset = round_up(L.scales_offset + L.scales_bytes, kRegionAlign);
   L.total_bytes = L.trailer_offset + kTrailerBytes;
   return L;
@@ -174,6 +177,32 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Scale words of one nibble pair (rows 2p, 2p+1) in the packed blob: a half2
+// for fp16 scales (layout version 1, in .x) or a float2 for fp32 scales
+// (version 2).  Returns them as two floats.
+template <bool F32S>
+__device__ __forceinline__ float2 scale_pair(uint2 w) {
+  if (F32S) return make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+  const __half2 h = u32_as_h2(w.x);
+  return make_float2(__low2float(h), __high2float(h));
+}
+
+// Tensor-core operand of two weights with fp32 scales (layout version 2):
+// fp16_RNE(fp32_RNE((code - 8) * s)) for the exact integers c = code - 8.
+__device__ __forceinline__ uint32_t weight_pair_f32s(__half2 c, float s_lo, float s_hi) {
+  return h2_as_u32(__floats2half2_rn(__fmul_rn(__low2float(c), s_lo), __fmul_rn(__high2float(c), s_hi)));
+}
+
+// D(16x8, f32) = A(16x16, f16, row) * B(16x8, f16, col): the accumulator
+// starts from zero (no register moves to clear it)
+__device__ __forceinline__ void mma_16816_zero(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "f"(0.f));
 }
 
 }  // namespace q4gsw

@@ -23,11 +23,11 @@ constexpr int kEmbThreads = 128;
 
 namespace emb {
 
+template <bool F32S>
 __global__ void __launch_bounds__(kEmbThreads)
 q4gsw_embedding_kernel(const uint8_t* __restrict__ packed, const int32_t* __restrict__ indices, float* __restrict__ out,
-                 int N, int K, int gs, int T) {
-  const Layout L = layout_of(N, K, gs);
-  const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
+                       int N, int K, int gs, int T) {
+  const Layout L = layout_of(N, K, gs, F32S ? 4 : 2);
   const int gsl = __ffs(gs) - 1;
   const int c = blockIdx.x * kEmbThreads + threadIdx.x;   // 16-byte chunk of the row
   if (c >= K / 16) return;
@@ -48,13 +48,16 @@ q4gsw_embedding_kernel(const uint8_t* __restrict__ packed, const int32_t* __rest
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int k0 = 64 * b + 16 * i + 4 * tq;   // columns k0 .. k0 + 3 share one group (gs >= 16)
-      const float s = __half2float(__ldg(scales + (size_t)(k0 >> gsl) * N + r));
+      const size_t si = (size_t)(k0 >> gsl) * N + r;
+      const float s = F32S ? __ldg(reinterpret_cast<const float*>(packed + L.scales_offset) + si)
+                           : __half2float(__ldg(reinterpret_cast<const __half*>(packed + L.scales_offset) + si));
       const uint32_t w = words[i] >> shift;
-      // byte slots (0, 1, 2, 3) hold columns (+0, +2, +1, +3)
-      const float v0 = (float)((int)(w & 0xFu) - 8) * s;
-      const float v2 = (float)((int)((w >> 8) & 0xFu) - 8) * s;
-      const float v1 = (float)((int)((w >> 16) & 0xFu) - 8) * s;
-      const float v3 = (float)((int)((w >> 24) & 0xFu) - 8) * s;
+      // byte slots (0, 1, 2, 3) hold columns (+0, +2, +1, +3); with fp16 scales
+      // the products are exact, with fp32 scales each is rounded once
+      const float v0 = __fmul_rn((float)((int)(w & 0xFu) - 8), s);
+      const float v2 = __fmul_rn((float)((int)((w >> 8) & 0xFu) - 8), s);
+      const float v1 = __fmul_rn((float)((int)((w >> 16) & 0xFu) - 8), s);
+      const float v3 = __fmul_rn((float)((int)((w >> 24) & 0xFu) - 8), s);
       *reinterpret_cast<float4*>(dst + 16 * i) = make_float4(v0, v1, v2, v3);
     }
   }
@@ -62,12 +65,15 @@ q4gsw_embedding_kernel(const uint8_t* __restrict__ packed, const int32_t* __rest
 
 }  // namespace emb
 
-cudaError_t launch_embedding(const void* packed, int N, int K, int gs, const int32_t* indices, int T, float* out,
-                             cudaStream_t stream) {
+cudaError_t launch_embedding(const void* packed, int N, int K, int gs, bool f32s, const int32_t* indices, int T,
+                             float* out, cudaStream_t stream) {
   const int chunks = K / 16;
   const dim3 grid((chunks + kEmbThreads - 1) / kEmbThreads, T < 65535 ? T : 65535);
-  emb::q4gsw_embedding_kernel<<<grid, kEmbThreads, 0, stream>>>(static_cast<const uint8_t*>(packed), indices, out, N,
-                                                                K, gs, T);
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  if (f32s)
+    emb::q4gsw_embedding_kernel<true><<<grid, kEmbThreads, 0, stream>>>(pk, indices, out, N, K, gs, T);
+  else
+    emb::q4gsw_embedding_kernel<false><<<grid, kEmbThreads, 0, stream>>>(pk, indices, out, N, K, gs, T);
   return cudaGetLastError();
 }
 

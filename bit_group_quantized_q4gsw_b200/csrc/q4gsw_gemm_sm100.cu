@@ -120,12 +120,13 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
-template <bool BWD, int ST, int SCB, int MSUB>
+template <bool BWD, int ST, int SCB, int MSUB, bool F32S>
 __global__ void __launch_bounds__(kThreads, 1)
 q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
                   const __grid_constant__ CUtensorMap map_sc, const Args args) {
   using namespace sm100;
   using SM = Smem<ST, SCB, MSUB>;
+  constexpr int SB = F32S ? 4 : 2;   // bytes per scale
   constexpr int OFF_A = SM::OFF_A, OFF_P = SM::OFF_P, OFF_W = SM::OFF_W, OFF_SC = SM::OFF_SC,
                 OFF_CTL = SM::OFF_CTL, SC_BYTES = SCB, A_STAGE = SM::A_STAGE,
                 TMEM_COLS = SM::TMEM_COLS;
@@ -274,9 +275,9 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
         // stage base column kc: with gs >= 64 the 64 columns sit in one group,
         // with gs < 64 the stage starts a group; either way the row is
         // ((kc mod gs) + 16 i + 8 u) >> gsl = (16 i + 8 u) >> gsl for gs < 64, else 0
-        sc_off[ii] = (args.gs < 64 ? ((16 * i + 8 * u) >> gsl) : 0) * 512 + 4 * p;
+        sc_off[ii] = (args.gs < 64 ? ((16 * i + 8 * u) >> gsl) : 0) * 256 * SB + 2 * SB * p;
       } else {
-        sc_off[ii] = (((n0 & (args.gs - 1)) + 64 * j + 16 * i + 8 * u) >> gsl) * 128 + 4 * p;
+        sc_off[ii] = (((n0 & (args.gs - 1)) + 64 * j + 16 * i + 8 * u) >> gsl) * 64 * SB + 2 * SB * p;
       }
       const int chunk = 2 * i + u;
       st_off_e[ii] = (BWD ? j * 8192 : 0) + re * 128 + 16 * (chunk ^ (re & 7));
@@ -293,21 +294,30 @@ q4gsw_gemm_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_cons
       const uint32_t sc = sbase + OFF_SC + s * SC_BYTES;
       const uint2 c0 = lds64(pk + pk_off0);
       const uint2 c1 = lds64(pk + pk_off1);
-      const uint32_t sw0 = lds32(sc + sc_off[0]), sw1 = lds32(sc + sc_off[1]);
+      const uint2 sw[2] = {F32S ? lds64(sc + sc_off[0]) : make_uint2(lds32(sc + sc_off[0]), 0u),
+                           F32S ? lds64(sc + sc_off[1]) : make_uint2(lds32(sc + sc_off[1]), 0u)};
       const uint32_t wlo[2] = {c0.x, c0.y};
       const uint32_t whi[2] = {c1.x, c1.y};
-      const uint32_t sw[2] = {sw0, sw1};
       const uint32_t wt = sbase + OFF_W + w * W_BYTES;
 #pragma unroll
       for (int ii = 0; ii < 2; ++ii) {
         const RowPairs a = codes_minus8_rows(wlo[ii]);   // columns +0..3 of this 8-column chunk
         const RowPairs b = codes_minus8_rows(whi[ii]);   // columns +4..7
-        const __half2 s2 = u32_as_h2(sw[ii]);
-        const __half2 se = __low2half2(s2), so = __high2half2(s2);
-        const uint4 ve = make_uint4(h2_as_u32(__hmul2(a.ev01, se)), h2_as_u32(__hmul2(a.ev23, se)),
-                                    h2_as_u32(__hmul2(b.ev01, se)), h2_as_u32(__hmul2(b.ev23, se)));
-        const uint4 vo = make_uint4(h2_as_u32(__hmul2(a.od01, so)), h2_as_u32(__hmul2(a.od23, so)),
-                                    h2_as_u32(__hmul2(b.od01, so)), h2_as_u32(__hmul2(b.od23, so)));
+        uint4 ve, vo;
+        if (F32S) {
+          const float se = __uint_as_float(sw[ii].x), so = __uint_as_float(sw[ii].y);
+          ve = make_uint4(weight_pair_f32s(a.ev01, se, se), weight_pair_f32s(a.ev23, se, se),
+                          weight_pair_f32s(b.ev01, se, se), weight_pair_f32s(b.ev23, se, se));
+          vo = make_uint4(weight_pair_f32s(a.od01, so, so), weight_pair_f32s(a.od23, so, so),
+                          weight_pair_f32s(b.od01, so, so), weight_pair_f32s(b.od23, so, so));
+        } else {
+          const __half2 s2 = u32_as_h2(sw[ii].x);
+          const __half2 se = __low2half2(s2), so = __high2half2(s2);
+          ve = make_uint4(h2_as_u32(__hmul2(a.ev01, se)), h2_as_u32(__hmul2(a.ev23, se)),
+                          h2_as_u32(__hmul2(b.ev01, se)), h2_as_u32(__hmul2(b.ev23, se)));
+          vo = make_uint4(h2_as_u32(__hmul2(a.od01, so)), h2_as_u32(__hmul2(a.od23, so)),
+                          h2_as_u32(__hmul2(b.od01, so)), h2_as_u32(__hmul2(b.od23, so)));
+        }
         sts128(wt + st_off_e[ii], ve);
         sts128(wt + st_off_o[ii], vo);
       }
@@ -457,12 +467,12 @@ static double stage_time(int msub) { return msub == 2 ? 1.6 : 1.0; }
 // (stages / S * stage time + fixed overhead: 2 stage times per accumulator, or
 // 8 with the cluster reduction), where waves(S) uses how many S-CTA clusters
 // the device can hold at once (a GPC must host a whole cluster).
-template <bool BWD, int ST, int SCB, int MSUB>
+template <bool BWD, int ST, int SCB, int MSUB, bool F32S>
 static cudaError_t gemm_variant(const CUtensorMap& map_act, const CUtensorMap& map_pk, const CUtensorMap& map_sc,
                                 const gemm::Args& a, int tiles_n, cudaStream_t stream, bool launch, int* S_out,
                                 double* cost_out) {
   using namespace gemm;
-  auto kern = q4gsw_gemm_kernel<BWD, ST, SCB, MSUB>;
+  auto kern = q4gsw_gemm_kernel<BWD, ST, SCB, MSUB, F32S>;
   constexpr int smem = Smem<ST, SCB, MSUB>::BYTES;
   static PerDeviceOnce attr_once;
   static std::atomic<int> max_clusters[kMaxDevices][9];
@@ -524,32 +534,32 @@ static int forced_msub() {
   return g == kGemmSs1 ? 1 : g == kGemmSs2 ? 2 : 0;
 }
 
-template <bool BWD>
+template <bool BWD, bool F32S>
 static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, const uint16_t* act, int M,
                                     OutSplit out, cudaStream_t stream, char* route, int route_len) {
   using namespace gemm;
+  constexpr int SB = F32S ? 4 : 2;
+  const CUtensorMapDataType sdt = F32S ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
   CUtensorMap map_pk, map_sc;
-  const Layout L = layout_of(N, K, gs);
+  const Layout L = layout_of(N, K, gs, SB);
   const void* scales = pk + L.scales_offset;
   const int G = K / gs;
   bool ok;
   int sc_bytes;
   if (!BWD) {
     const int rows = TK / gs > 1 ? TK / gs : 1;   // scale groups of one 64-column stage
-    sc_bytes = rows * BN * 2;
+    sc_bytes = rows * BN * SB;
     ok = make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BN / 2, CU_TENSOR_MAP_SWIZZLE_64B) &&
-         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, BN, rows,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
+         make_map_2d(&map_sc, sdt, scales, N, G, (uint64_t)N * SB, BN, rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
     const int rows = BN / gs > 1 ? BN / gs : 1;   // scale groups of one 256-column tile
-    sc_bytes = rows * TK * 2;
+    sc_bytes = rows * TK * SB;
     ok = make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, TK / 2,
                      CU_TENSOR_MAP_SWIZZLE_64B) &&
-         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, TK, rows,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
+         make_map_2d(&map_sc, sdt, scales, N, G, (uint64_t)N * SB, TK, rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   }
-  if (!ok || sc_bytes > 2048) return cudaErrorInvalidValue;
+  if (!ok || sc_bytes > (F32S ? 4096 : 2048)) return cudaErrorInvalidValue;
 
   Args a;
   a.sc_bytes = sc_bytes;
@@ -562,6 +572,9 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
   const int contraction = BWD ? N : K;
   a.stages_total = (contraction + TK - 1) / TK;
   const int tiles_n = (a.out_cols + BN - 1) / BN;
+  // Scale slots of 4 KB (fp32 scales with 16-column groups) leave room for one
+  // 128-token accumulator per CTA only.
+  const bool one_acc_only = sc_bytes > 2048;
   // The activation box is re-encoded per variant (128 or 256 tokens high).
   auto run = [&](int msub, bool launch, int* S, double* cost) -> cudaError_t {
     CUtensorMap map_a;
@@ -570,12 +583,14 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     if (sc_bytes <= 1024)
-      return msub == 2 ? gemm_variant<BWD, 3, 1024, 2>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost)
-                       : gemm_variant<BWD, 5, 1024, 1>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost);
-    return msub == 2 ? gemm_variant<BWD, 3, 2048, 2>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost)
-                     : gemm_variant<BWD, 4, 2048, 1>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost);
+      return msub == 2 ? gemm_variant<BWD, 3, 1024, 2, F32S>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost)
+                       : gemm_variant<BWD, 5, 1024, 1, F32S>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost);
+    if (sc_bytes <= 2048)
+      return msub == 2 ? gemm_variant<BWD, 3, 2048, 2, F32S>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost)
+                       : gemm_variant<BWD, 4, 2048, 1, F32S>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost);
+    return gemm_variant<BWD, 4, 4096, 1, F32S>(map_a, map_pk, map_sc, a, tiles_n, stream, launch, S, cost);
   };
-  int msub = forced_msub();
+  int msub = one_acc_only ? 1 : forced_msub();
   int S = 1;
   double cost = 0;
   cudaError_t e = cudaSuccess;
@@ -615,17 +630,23 @@ static bool use_ss_route(int M) {
   return M > 512;
 }
 
-cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
-                            cudaStream_t stream, char* route, int route_len) {
-  if (use_ss_route(M)) return launch_gemm_impl<false>(packed, N, K, gs, x, M, out, stream, route, route_len);
-  return launch_gemm_ts_impl<false>(packed, N, K, gs, x, M, out, stream, route, route_len);
-}
-
-cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
+cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M, OutSplit out,
                             cudaStream_t stream, char* route, int route_len) {
   if (use_ss_route(M))
-    return launch_gemm_impl<true>(packed, N, K, gs, d_out, M, single_output(d_x, K), stream, route, route_len);
-  return launch_gemm_ts_impl<true>(packed, N, K, gs, d_out, M, single_output(d_x, K), stream, route, route_len);
+    return f32s ? launch_gemm_impl<false, true>(packed, N, K, gs, x, M, out, stream, route, route_len)
+                : launch_gemm_impl<false, false>(packed, N, K, gs, x, M, out, stream, route, route_len);
+  return f32s ? launch_gemm_ts_impl<false, true>(packed, N, K, gs, x, M, out, stream, route, route_len)
+              : launch_gemm_ts_impl<false, false>(packed, N, K, gs, x, M, out, stream, route, route_len);
+}
+
+cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M,
+                            float* d_x, cudaStream_t stream, char* route, int route_len) {
+  const OutSplit o = single_output(d_x, K);
+  if (use_ss_route(M))
+    return f32s ? launch_gemm_impl<true, true>(packed, N, K, gs, d_out, M, o, stream, route, route_len)
+                : launch_gemm_impl<true, false>(packed, N, K, gs, d_out, M, o, stream, route, route_len);
+  return f32s ? launch_gemm_ts_impl<true, true>(packed, N, K, gs, d_out, M, o, stream, route, route_len)
+              : launch_gemm_ts_impl<true, false>(packed, N, K, gs, d_out, M, o, stream, route, route_len);
 }
 
 __global__ void q4gsw_error_exchange_kernel(unsigned int slot) {

@@ -42,19 +42,21 @@ constexpr int kDequantWarps = 16;
 constexpr int kThreads = 32 * (2 + kDequantWarps);
 constexpr int X_BYTES = BT_MAX * TK * 2;   // activation tile, 32 KB
 constexpr int P_BYTES = BW / 2 * TK;       // packed codes of one stage, 4 KB
-constexpr int SC_BYTES = 1024;             // scale rows of one stage (at most)
 constexpr int CTL_BYTES = 256;
 constexpr int ACC_COLS = 256;              // fp32 accumulator columns (tokens)
 constexpr int A_COLS = TK / 2;             // one dequantised stage: 64 fp16 per lane = 32 columns
 constexpr int TMEM_COLS = 512;
 static_assert(ACC_COLS + WST * A_COLS <= TMEM_COLS, "tensor memory budget");
 
-template <int ST>
+// ST stages; SCB bytes of scale rows per stage (1 KB for fp16 scales, 2 KB for
+// fp32 scales, packed layout version 2).
+template <int ST, int SCB>
 struct Smem {
+  static constexpr int SC_BYTES = SCB;
   static constexpr int OFF_X = 0;
   static constexpr int OFF_P = OFF_X + ST * X_BYTES;
   static constexpr int OFF_SC = OFF_P + ST * P_BYTES;
-  static constexpr int OFF_CTL = OFF_SC + ST * SC_BYTES;
+  static constexpr int OFF_CTL = OFF_SC + ST * SCB;
   static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
   static_assert(OFF_P % 1024 == 0 && OFF_SC % 1024 == 0, "1024-byte aligned regions");
   static_assert(BT_MAX * BW * 4 <= OFF_SC, "split-K staging must fit below the scale slots");
@@ -106,14 +108,16 @@ __device__ __forceinline__ uint32_t nibbles_minus8(uint32_t v) {
   return h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(v, 0x000F000Fu, 0x64006400u)), kSub));
 }
 
-template <bool BWD, int ST>
+template <bool BWD, int ST, bool F32S>
 __global__ void __launch_bounds__(kThreads, 1)
 q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
                      const __grid_constant__ CUtensorMap map_sc, const __grid_constant__ CUtensorMap map_y0,
                      const __grid_constant__ CUtensorMap map_y1, const __grid_constant__ CUtensorMap map_y2,
                      const Args args) {
   using namespace sm100;
-  using SM = Smem<ST>;
+  using SM = Smem<ST, F32S ? 2048 : 1024>;
+  constexpr int SC_BYTES = SM::SC_BYTES;
+  constexpr int SB = F32S ? 4 : 2;   // bytes per scale
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + SM::OFF_CTL);
@@ -247,7 +251,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       for (int t = 0; t < 4; ++t) off[t] = p * 64 + 16 * (t ^ ((p >> 1) & 3)) + 4 * kq;
       // the 16 columns share one scale: row ((kc mod gs) + 16 kq) >> gsl of
       // the stage's box (stages start on 64-column boundaries)
-      sc_off = (args.gs < 64 ? ((16 * kq) >> gsl) : 0) * 256 + 2 * r;
+      sc_off = (args.gs < 64 ? ((16 * kq) >> gsl) : 0) * BW * SB + SB * r;
     } else {
       // Row r = output feature k = f0 + r.  Pair row p (contraction rows 2p,
       // 2p+1) holds it in byte column_offset(r) of its 128-byte box row; the
@@ -255,7 +259,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       const uint32_t boff = (uint32_t)column_offset(r);
 #pragma unroll
       for (int j = 0; j < 8; ++j) off[j] = (8 * kq + j) * 128 + boff;
-      sc_off = (uint32_t)((((f0 & (args.gs - 1)) + r) >> gsl) * 128 + 4 * 8 * kq);
+      sc_off = (uint32_t)((((f0 & (args.gs - 1)) + r) >> gsl) * TK * SB + 2 * SB * 8 * kq);
     }
     for (int it = 0; it < nit; ++it) {
       const int s = it % ST, w = it % WST;
@@ -272,20 +276,36 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
         uint32_t wd[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) wd[t] = lds32(pk + off[t]);
-        const uint32_t sb = lds_u16(sc + sc_off);
-        const __half2 s2 = u32_as_h2(sb | (sb << 16));
+        if (F32S) {
+          const float sf = __uint_as_float(lds32(sc + sc_off));
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const uint32_t W = wd[t] >> shift;                                      // this row's nibbles
-          v[2 * t] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W)), s2));       // columns 4t, 4t+1
-          v[2 * t + 1] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W >> 8)), s2));  // 4t+2, 4t+3
+          for (int t = 0; t < 4; ++t) {
+            const uint32_t W = wd[t] >> shift;                                           // this row's nibbles
+            v[2 * t] = weight_pair_f32s(u32_as_h2(nibbles_minus8(W)), sf, sf);          // columns 4t, 4t+1
+            v[2 * t + 1] = weight_pair_f32s(u32_as_h2(nibbles_minus8(W >> 8)), sf, sf); // 4t+2, 4t+3
+          }
+        } else {
+          const uint32_t sb = lds_u16(sc + sc_off);
+          const __half2 s2 = u32_as_h2(sb | (sb << 16));
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const uint32_t W = wd[t] >> shift;                                      // this row's nibbles
+            v[2 * t] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W)), s2));       // columns 4t, 4t+1
+            v[2 * t + 1] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W >> 8)), s2));  // 4t+2, 4t+3
+          }
         }
       } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t b = lds_u8(pk + off[j]);                 // code[2p, k] | code[2p+1, k] << 4
-          const uint32_t s2 = lds32(sc + sc_off + 4 * j);          // s[g, 2p], s[g, 2p+1]
-          v[j] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(b * 0x1001u)), u32_as_h2(s2)));
+          const __half2 c2 = u32_as_h2(nibbles_minus8(b * 0x1001u));
+          if (F32S) {
+            const uint32_t a = sc + sc_off + 8 * j;                 // s32[g, 2p], s32[g, 2p+1]
+            v[j] = weight_pair_f32s(c2, __uint_as_float(lds32(a)), __uint_as_float(lds32(a + 4)));
+          } else {
+            const uint32_t s2 = lds32(sc + sc_off + 4 * j);        // s[g, 2p], s[g, 2p+1]
+            v[j] = h2_as_u32(__hmul2(c2, u32_as_h2(s2)));
+          }
         }
       }
       tmem_st_32x32b_x8(tmem + lane_base + (uint32_t)(ACC_COLS + w * A_COLS + 8 * kq), v);
@@ -418,13 +438,16 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <bool BWD>
+template <bool BWD, bool F32S>
 static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs, const uint16_t* act, int M,
                                        OutSplit out, cudaStream_t stream, char* route, int route_len) {
   using namespace ts;
-  constexpr int ST = 6;
+  constexpr int ST = F32S ? 5 : 6;
+  constexpr int SB = F32S ? 4 : 2;
+  constexpr int SC_BYTES = Smem<ST, F32S ? 2048 : 1024>::SC_BYTES;
+  const CUtensorMapDataType sdt = F32S ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
-  const Layout L = layout_of(N, K, gs);
+  const Layout L = layout_of(N, K, gs, SB);
   const void* scales = pk + L.scales_offset;
   const int G = K / gs;
   Args a;
@@ -446,18 +469,16 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
                         (uint64_t)contraction * 2, TK, a.bt, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!BWD) {
     const int rows = TK / gs > 1 ? TK / gs : 1;   // scale groups of one 64-column stage
-    a.sc_bytes = rows * BW * 2;
+    a.sc_bytes = rows * BW * SB;
     ok = ok && make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, TK, BW / 2,
                            CU_TENSOR_MAP_SWIZZLE_64B) &&
-         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, BW, rows,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
+         make_map_2d(&map_sc, sdt, scales, N, G, (uint64_t)N * SB, BW, rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
     const int rows = BW / gs > 1 ? BW / gs : 1;   // scale groups of one 128-feature tile
-    a.sc_bytes = rows * TK * 2;
+    a.sc_bytes = rows * TK * SB;
     ok = ok && make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, BW, TK / 2,
                            CU_TENSOR_MAP_SWIZZLE_NONE) &&
-         make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, N, G, (uint64_t)N * 2, TK, rows,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
+         make_map_2d(&map_sc, sdt, scales, N, G, (uint64_t)N * SB, TK, rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   }
   if (!ok || a.sc_bytes > SC_BYTES) return cudaErrorInvalidValue;
 
@@ -484,8 +505,8 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
     if (!tma_out) map_y[0] = map_y[1] = map_y[2] = map_act;   // never read
   }
 
-  auto kern = q4gsw_gemm_ts_kernel<BWD, ST>;
-  constexpr int smem = Smem<ST>::BYTES;
+  auto kern = q4gsw_gemm_ts_kernel<BWD, ST, F32S>;
+  constexpr int smem = Smem<ST, SC_BYTES>::BYTES;
   static PerDeviceOnce attr_once;
   static std::atomic<int> max_clusters[kMaxDevices][9];
   const int dev = current_device();

@@ -44,7 +44,7 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // blocks [u*KB/U, (u+1)*KB/U) of its row tile (KB = K/64, U = 4 S).
 // NT = number of 8-token MMA tiles (1: M <= 8 per slice, 2: M <= 16).
 // SPG = 16-column steps per scale group (1: gs 16, 2: gs 32, 4: gs >= 64).
-template <int NT, int SPG>
+template <int NT, int SPG, bool F32S>
 __global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 7 : 4)
 q4gsw_gemv_fwd_reg_kernel(const uint8_t* __restrict__ packed, const __half* __restrict__ x, OutSplit out, int M, int N,
                 int K, int gs) {
@@ -59,8 +59,7 @@ q4gsw_gemv_fwd_reg_kernel(const uint8_t* __restrict__ packed, const __half* __re
   const int tok0 = blockIdx.z * 16;
   const int Mz = min(16, M - tok0);
 
-  const Layout L = layout_of(N, K, gs);
-  const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
+  const Layout L = layout_of(N, K, gs, F32S ? 4 : 2);
   const int gsl = __ffs(gs) - 1;  // gs is a power of two
   const int p_raw = tile * 8 + g;  // nibble pair of this lane: rows 2p (even) and 2p+1 (odd)
   const bool pvalid = p_raw < (N >> 1);  // the last tile holds 4 pairs when N % 16 == 8
@@ -79,9 +78,9 @@ q4gsw_gemv_fwd_reg_kernel(const uint8_t* __restrict__ packed, const __half* __re
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[j][c] = part[0][j][c] = part[1][j][c] = 0.f;
 
-  auto flush = [&](uint32_t s_word) {  // scale one finished group into acc
-    const __half2 s2 = u32_as_h2(s_word);
-    const float se = __low2float(s2), so = __high2float(s2);
+  auto flush = [&](uint2 s_word) {  // scale one finished group into acc
+    const float2 sp = scale_pair<F32S>(s_word);
+    const float se = sp.x, so = sp.y;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       acc[j][0] = fmaf(part[0][j][0] + part[1][j][0], se, acc[j][0]);
@@ -104,12 +103,14 @@ q4gsw_gemv_fwd_reg_kernel(const uint8_t* __restrict__ packed, const __half* __re
   }
   constexpr int NGB = (SPG == 4) ? 1 : 4 / SPG;            // scale groups per block
   const int bpg_mask = (SPG == 4) ? (gs >> 6) - 1 : 0;      // blocks per group - 1 (gs >= 64)
-  const __half* srow = scales + 2 * p;
+  // scale words of pair p: half2 (fp16 scales) or float2 (fp32 scales), one row per group
+  const uint8_t* srow = packed + L.scales_offset + (size_t)(F32S ? 8 : 4) * p;
+  const size_t srow_stride = (size_t)(F32S ? 4 : 2) * N;
 
   // One 64-column block of this lane: packed word quad, scale words, x fragments.
   struct Blk {
     uint4 w;
-    uint32_t s[NGB];
+    uint2 s[NGB];
     uint2 xv[NT][4];
   };
   const int b_last = b_end - 1;
@@ -117,7 +118,10 @@ q4gsw_gemv_fwd_reg_kernel(const uint8_t* __restrict__ packed, const __half* __re
     b = min(b, b_last);
     d.w = ldg_stream_v4(row + 64 * b);
 #pragma unroll
-    for (int r = 0; r < NGB; ++r) d.s[r] = ldg_nc_u32(srow + (size_t)((64 * b + r * (64 / NGB)) >> gsl) * N);
+    for (int r = 0; r < NGB; ++r) {
+      const uint8_t* sp = srow + (size_t)((64 * b + r * (64 / NGB)) >> gsl) * srow_stride;
+      d.s[r] = F32S ? ldg_nc_v2(sp) : make_uint2(ldg_nc_u32(sp), 0u);
+    }
   };
   auto load_x = [&](int b, Blk& d) {
     b = min(b, b_last);
@@ -224,7 +228,7 @@ q4gsw_gemv_fwd_reg_kernel(const uint8_t* __restrict__ packed, const __half* __re
 constexpr int kBwdWarps = 8;
 constexpr int kBwdThreads = 32 * kBwdWarps;
 
-template <int NT, int SPB>  // NT 8-token tiles; SPB scale groups per block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
+template <int NT, int SPB, bool F32S>  // NT 8-token tiles; SPB scale groups per block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
 __global__ void __launch_bounds__(kBwdThreads) q4gsw_gemv_bwd_reg_kernel(const uint8_t* __restrict__ packed,
                                                                const __half* __restrict__ dout,
                                                                float* __restrict__ dx,
@@ -243,8 +247,9 @@ __global__ void __launch_bounds__(kBwdThreads) q4gsw_gemv_bwd_reg_kernel(const u
   const bool jvalid = J < KB;
   const int Jc = jvalid ? J : 0;            // lanes past the last block read block 0, never stored
 
-  const Layout L = layout_of(N, K, gs);
-  const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
+  const Layout L = layout_of(N, K, gs, F32S ? 4 : 2);
+  const uint8_t* scales = packed + L.scales_offset;
+  const size_t sstride = (size_t)(F32S ? 4 : 2) * N;   // bytes per scale row
   const int NS = (N + 15) >> 4;   // the last step holds 4 pairs when N % 16 == 8
   const int NP = N >> 1;
   const int U = S * kBwdWarps, u = split * kBwdWarps + warp;
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(kBwdThreads) q4gsw_gemv_bwd_reg_kernel(const u
   struct StepData {
     uint4 va, vb;              // packed bytes of pairs pA and pB
     uint32_t b[NT][2];         // d_out fragments
-    uint32_t sa[SPB], sb[SPB]; // scale half2 of pairs pA, pB per group
+    uint2 sa[SPB], sb[SPB];    // scale words of pairs pA, pB per group
   };
   const int s_last = s_end - 1;
   auto load_step = [&](int st, StepData& d) {
@@ -290,9 +295,11 @@ __global__ void __launch_bounds__(kBwdThreads) q4gsw_gemv_bwd_reg_kernel(const u
     }
 #pragma unroll
     for (int q = 0; q < SPB; ++q) {
-      d.sa[q] = ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pA);
-      const uint32_t v = ldg_nc_u32(scales + (size_t)grp[q] * N + 2 * pB);
-      d.sb[q] = bvalid ? v : 0u;
+      const uint8_t* ra = scales + (size_t)grp[q] * sstride + (size_t)(F32S ? 8 : 4) * pA;
+      const uint8_t* rb = scales + (size_t)grp[q] * sstride + (size_t)(F32S ? 8 : 4) * pB;
+      d.sa[q] = F32S ? ldg_nc_v2(ra) : make_uint2(ldg_nc_u32(ra), 0u);
+      const uint2 v = F32S ? ldg_nc_v2(rb) : make_uint2(ldg_nc_u32(rb), 0u);
+      d.sb[q] = bvalid ? v : make_uint2(0u, 0u);
     }
   };
   auto compute_step = [&](const StepData& d) {
@@ -301,15 +308,18 @@ __global__ void __launch_bounds__(kBwdThreads) q4gsw_gemv_bwd_reg_kernel(const u
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int q = i / (4 / SPB);
-      const __half2 sa = u32_as_h2(d.sa[q]), sb = u32_as_h2(d.sb[q]);
       const ColPairs ca = codes_minus8_cols(wa[i]);
       const ColPairs cb = codes_minus8_cols(wb[i]);
       const __half2 la[4] = {ca.c0, ca.c1, ca.c2, ca.c3};
       const __half2 lb[4] = {cb.c0, cb.c1, cb.c2, cb.c3};
+      auto op = [&](__half2 c, uint2 sw) -> uint32_t {   // one byte's (even n, odd n) weights, scaled
+        if (F32S) return weight_pair_f32s(c, __uint_as_float(sw.x), __uint_as_float(sw.y));
+        return h2_as_u32(__hmul2(c, u32_as_h2(sw.x)));
+      };
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint32_t af[4] = {h2_as_u32(__hmul2(la[2 * h], sa)), h2_as_u32(__hmul2(la[2 * h + 1], sa)),
-                                h2_as_u32(__hmul2(lb[2 * h], sb)), h2_as_u32(__hmul2(lb[2 * h + 1], sb))};
+        const uint32_t af[4] = {op(la[2 * h], d.sa[q]), op(la[2 * h + 1], d.sa[q]), op(lb[2 * h], d.sb[q]),
+                                op(lb[2 * h + 1], d.sb[q])};
 #pragma unroll
         for (int j = 0; j < NT; ++j) mma_16816(acc[j][2 * i + h], af, d.b[j]);
       }
@@ -428,29 +438,13 @@ static cudaError_t launch_cluster(Kern kernel, dim3 grid, int threads, int clust
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// Route between the two forward GEMVs.  The TMA-ring kernel (64-row CTAs,
-// two per SM for up to 8 tokens) is taken for 9..16 tokens, and for up to 8
-// tokens when its CTAs spread evenly over the SMs (each SM's share within 15 %
-// of the busiest SM's); otherwise the register-fed kernel, whose 16-row CTAs
-// balance better, is faster (measured on B200: 14336x4096 at M=1, 224 CTAs on
-// 148 SMs, 13.4 vs 11.3 us).  q4gsw_debug_pin_routes can pin either kernel.
-static bool use_reg_gemv(int N, int K, int M) {
-  const int pin = route_pins().gemv;
-  if (pin == kGemvReg) return true;
-  if (pin == kGemvTma) return false;
-  if (M > 8) return false;
-  const int sms = sm_count(current_device());
-  const int tiles = (N + 63) / 64, stages = (K + 255) / 256;
-  int S = 2 * sms / tiles;
-  S = S < 1 ? 1 : (S > 8 ? 8 : S);
-  while (S > 1 && stages / S < 2) --S;
-  const double per_sm = (double)tiles * S / sms;
-  return per_sm / ceil(per_sm) < 0.85;
-}
+// Route between the two forward GEMVs: the TMA-ring kernel by default; the
+// register-fed kernel only when q4gsw_debug_pin_routes pins it.
+static bool use_reg_gemv() { return route_pins().gemv == kGemvReg; }
 
-cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M,
+cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M,
                             OutSplit out, cudaStream_t stream, char* route, int route_len) {
-  if (!use_reg_gemv(N, K, M)) return launch_gemv_tma_fwd(packed, N, K, gs, x, M, out, stream, route, route_len);
+  if (!use_reg_gemv()) return launch_gemv_tma_fwd(packed, N, K, gs, f32s, x, M, out, stream, route, route_len);
   const int tiles = (N + 15) / 16;
   const int zs = (M + 15) / 16;
   const int NT = (M <= 8) ? 1 : 2;
@@ -459,11 +453,13 @@ cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint
   const __half* xh = reinterpret_cast<const __half*>(x);
   cudaError_t err;
   int S = 1;
-#define Q4_FWD(NT_, SPG_)                                                                                       \
-  do {                                                                                                          \
-    S = fwd_splits((long long)tiles * zs, K / 64, (size_t)N * K / 2);                                        \
-    err = launch_cluster(rg::q4gsw_gemv_fwd_reg_kernel<NT_, SPG_>, dim3(tiles, S, zs), kGemvThreads, S, 0, stream, pk, xh, out, \
-                         M, N, K, gs);                                                                          \
+#define Q4_FWD(NT_, SPG_)                                                                                        \
+  do {                                                                                                           \
+    S = fwd_splits((long long)tiles * zs, K / 64, (size_t)N * K / 2);                                            \
+    err = f32s ? launch_cluster(rg::q4gsw_gemv_fwd_reg_kernel<NT_, SPG_, true>, dim3(tiles, S, zs), kGemvThreads, \
+                                S, 0, stream, pk, xh, out, M, N, K, gs)                                          \
+               : launch_cluster(rg::q4gsw_gemv_fwd_reg_kernel<NT_, SPG_, false>, dim3(tiles, S, zs), kGemvThreads,\
+                                S, 0, stream, pk, xh, out, M, N, K, gs);                                         \
   } while (0)
   if (NT == 1) {
     if (spg == 1) Q4_FWD(1, 1); else if (spg == 2) Q4_FWD(1, 2); else Q4_FWD(1, 4);
@@ -475,10 +471,11 @@ cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint
   return err;
 }
 
-cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M,
+cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M,
                             float* d_x, cudaStream_t stream, char* route, int route_len) {
   // the TMA-ring input gradient is the default; the register-fed one runs only when pinned
-  if (route_pins().gemv != kGemvReg) return launch_gemv_tma_bwd(packed, N, K, gs, d_out, M, d_x, stream, route, route_len);
+  if (route_pins().gemv != kGemvReg)
+    return launch_gemv_tma_bwd(packed, N, K, gs, f32s, d_out, M, d_x, stream, route, route_len);
   const int tiles = (K + 127) / 128;
   const int zs = (M + 15) / 16;
   const int NT = (M <= 8) ? 1 : 2;
@@ -488,14 +485,20 @@ cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
   const __half* dh = reinterpret_cast<const __half*>(d_out);
   cudaError_t err;
-#define Q4_BWD(NT_, SPB_)                                                                                         \
+#define Q4_BWD_F(NT_, SPB_, F_)                                                                                   \
   do {                                                                                                            \
-    err = cudaFuncSetAttribute(rg::q4gsw_gemv_bwd_reg_kernel<NT_, SPB_>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    err = cudaFuncSetAttribute(rg::q4gsw_gemv_bwd_reg_kernel<NT_, SPB_, F_>,                                      \
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                           \
     if (err == cudaSuccess) {                                                                                     \
       S = bwd_splits((long long)tiles * zs, (N + 15) / 16, kBwdWarps);                                           \
-      err = launch_cluster(rg::q4gsw_gemv_bwd_reg_kernel<NT_, SPB_>, dim3(tiles, S, zs), kBwdThreads, S, smem, stream, pk, dh,  \
-                           d_x, M, N, K, gs);                                                                     \
+      err = launch_cluster(rg::q4gsw_gemv_bwd_reg_kernel<NT_, SPB_, F_>, dim3(tiles, S, zs), kBwdThreads, S, smem, \
+                           stream, pk, dh, d_x, M, N, K, gs);                                                     \
     }                                                                                                             \
+  } while (0)
+#define Q4_BWD(NT_, SPB_)                     \
+  do {                                        \
+    if (f32s) Q4_BWD_F(NT_, SPB_, true);      \
+    else Q4_BWD_F(NT_, SPB_, false);          \
   } while (0)
   if (NT == 1) {
     if (spb == 1) Q4_BWD(1, 1); else if (spb == 2) Q4_BWD(1, 2); else Q4_BWD(1, 4);
@@ -503,6 +506,7 @@ cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint
     if (spb == 1) Q4_BWD(2, 1); else if (spb == 2) Q4_BWD(2, 2); else Q4_BWD(2, 4);
   }
 #undef Q4_BWD
+#undef Q4_BWD_F
   if (route) snprintf(route, route_len, "gemv_bwd launches=1 nt=%d splits=%d zslices=%d", NT, S, zs);
   return err;
 }

@@ -10,46 +10,48 @@
 //
 // At M <= 16 the layer is a weight stream: every code byte is read once and
 // used for at most 16 tokens, so the kernel lives or dies by the bytes it keeps
-// in flight.  One producer thread per CTA keeps ST stages of 256 contraction
-// columns in flight with TMA (codes of 32 nibble pairs, their scale rows, the
-// activation columns); sixteen consumer warps (four row groups of 8 pairs x
-// the four 64-column blocks of a stage) turn each stage into mma.sync m16n8k16
-// steps (A = 16 weight rows, B = 8 tokens), with the codes entering the MMA as
-// exact integers code - 8 and the fp16 scale applied to the fp32 partial sum
-// of each group, as in the register-fed GEMV.  The four block slices are summed
-// in shared memory, split-K CTAs of a cluster through distributed shared
-// memory, both in a fixed order.
+// in flight and by the instructions it spends per weight.  Forward: one
+// producer thread per CTA keeps ST stages of 256 contraction columns in flight
+// with TMA (codes of 32 nibble pairs = 64 output rows, their scale rows, the
+// activation columns); each of four consumer warps takes one 64-column block
+// of every stage for all four 16-row MMA tiles, so one activation fragment
+// feeds four mma.sync m16n8k16 (A = 16 weight rows, B = 8 tokens).  The codes
+// enter the MMA as exact integers code - 8; the fp16 scale multiplies the fp32
+// partial sum of each group, whose first MMA starts from a zero accumulator.
+// The four block slices are summed in shared memory, split-K CTAs of a cluster
+// through distributed shared memory, both in a fixed order.
 #pragma once
 
 namespace q4gsw {
 namespace gv {
 
-constexpr int kRowGroups = 4;                         // 8 nibble pairs (16 rows) each
-constexpr int kBlockSlices = 4;                       // 64-column block of the stage
-constexpr int kConsumerWarps = kRowGroups * kBlockSlices;
-constexpr int kThreads = 32 * (1 + kConsumerWarps);   // warp 0 produces
-constexpr int RP = 8 * kRowGroups;                    // nibble pairs per CTA (64 output rows)
-constexpr int SK = 256;                               // contraction columns per stage
-constexpr int CODE_BYTES = RP * SK;                   // two [32 pairs][128 B] boxes, 8 KB
-constexpr int SC_BYTES = 16 * 128;                    // scale rows of a stage (gs 16: 16 rows of 64 n)
+constexpr int kFwdConsumers = 4;                        // one 64-column block of every stage each
+constexpr int kFwdThreads = 32 * (kFwdConsumers + 1);   // the last warp produces
+constexpr int RP = 32;                                  // nibble pairs per CTA (64 rows = 4 MMA row tiles)
+constexpr int SK = 256;                                 // contraction columns per stage
+constexpr int CODE_BYTES = RP * SK;                     // two [32 pairs][128 B] boxes, 8 KB
 constexpr int CTL_BYTES = 256;
 
-template <int NT>
-struct Cfg {
-  static constexpr int MB = 8 * NT;                   // token rows of the activation boxes
-  static constexpr int XBOX = MB * 128 < 1024 ? 1024 : MB * 128;   // one [MB][64] box, 1 KB aligned
-  static constexpr int X_BYTES = 4 * XBOX;
-  static constexpr int STAGE = CODE_BYTES + SC_BYTES + X_BYTES;
-  // one 8-token tile: two CTAs per SM (registers capped at 60); two tiles:
-  // one CTA per SM with a deeper ring
-  static constexpr int kCtasPerSm = NT == 1 ? 2 : 1;
-  static constexpr int ST = NT == 1 ? 6 : 10;
+// Shared-memory map of the forward: ST stages of [codes | 4 activation boxes
+// | scale rows].  Each activation box is [<= 8 NT tokens][64 columns] fp16
+// (128-byte swizzle) in a 1 KB-aligned slot; the scale rows of one stage are
+// 256 / gs rows (at least one) of 64 scales (fp16, or fp32 in layout version 2).
+template <int NT, int SPG, bool F32S>
+struct FwdCfg {
+  static constexpr int SB = F32S ? 4 : 2;   // bytes per scale
+  static constexpr int XBOX = 1024 * NT;
+  static constexpr int SCB = (SPG == 1 ? 2048 : 1024) * (SB / 2);
+  static constexpr int OFF_X = CODE_BYTES;
+  static constexpr int OFF_SC = CODE_BYTES + 4 * XBOX;
+  static constexpr int STAGE = OFF_SC + SCB;
+  static constexpr int ST = 4;
   static constexpr int OFF_CTL = ST * STAGE;
-  static constexpr int OFF_RED = OFF_CTL + CTL_BYTES;   // [slice][16 tokens][64 rows] fp32 partial tiles
-  static constexpr int BYTES = OFF_RED + kBlockSlices * 16 * 64 * 4 + 1024;
+  static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
+  // CTAs per SM that fit in 228 KB (1 KB of each is reserved by the system)
+  static constexpr int CTAS = 4 * (BYTES + 1024) <= 233472 ? 4 : 3;
+  static constexpr int RED_FLOATS = kFwdConsumers * 16 * 64;   // [warp][token][row], reuses the ring
   static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
-  static_assert(ST <= 12, "barrier arrays");
-  static_assert(BYTES <= (kCtasPerSm == 2 ? 116 * 1024 : 226 * 1024), "CTAs per SM");
+  static_assert(RED_FLOATS * 4 <= OFF_CTL, "warp partials fit in the ring");
 };
 
 struct Ctl {
@@ -59,10 +61,10 @@ struct Ctl {
 };
 static_assert(sizeof(Ctl) <= CTL_BYTES, "control block");
 
-// MMA row g of row group w reads pair row 8 w + perm(g): the two pairs a
+// MMA row g of row tile rt reads pair row 8 rt + perm(g): the two pairs a
 // quarter of the warp reads together then differ in bit 2, so under the
 // 128-byte swizzle their 16-byte code chunks fall on distinct banks.
-__device__ __forceinline__ int pair_of(int w, int g) { return 8 * w + ((g & 1) << 2) + (g >> 1); }
+__device__ __forceinline__ int pair_of(int rt, int g) { return 8 * rt + ((g & 1) << 2) + (g >> 1); }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -83,18 +85,19 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 
 // grid = (ceil(N / 64) row tiles, S contraction splits, ceil(M / 16) token
 // slices), cluster = (1, S, 1).  SPG = 16-column steps per scale group
-// (1: gs 16, 2: gs 32, 4: gs >= 64).
-template <int NT, int SPG>
-__global__ void __launch_bounds__(kThreads, Cfg<NT>::kCtasPerSm)
+// (1: gs 16, 2: gs 32, 4: gs >= 64).  x_rows = rows of each activation box
+// (the tokens of a slice: min(M, 8) for one 8-token tile, 16 for two).
+template <int NT, int SPG, bool F32S>
+__global__ void __launch_bounds__(kFwdThreads, FwdCfg<NT, SPG, F32S>::CTAS)
 q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
-                    const __grid_constant__ CUtensorMap map_x, OutSplit out, int M, int N, int K, int gs,
-                    int stages_total) {
+                          const __grid_constant__ CUtensorMap map_x, OutSplit out, int M, int N, int K, int gs,
+                          int stages_total, int x_rows) {
   using namespace sm100;
-  using C = Cfg<NT>;
+  using C = FwdCfg<NT, SPG, F32S>;
+  constexpr int NGB = SPG == 4 ? 1 : 4 / SPG;   // scale groups per 64-column block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);   // [slice][token][64 rows]
   volatile int* abort_flag = &ctl->abort;
   const uint32_t sbase = smem_u32(smem);
 
@@ -112,7 +115,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::ST; ++i) {
       mbar_init(&ctl->full[i], 1);
-      mbar_init(&ctl->empty[i], kConsumerWarps);
+      mbar_init(&ctl->empty[i], kFwdConsumers);
     }
     ctl->abort = 0;
     fence_mbar_init();
@@ -122,11 +125,20 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   }
   __syncthreads();
 
-  // scale rows per stage: (SK / gs) for gs <= SK, else 1
+  // scale rows per stage: 256 / gs for gs <= 256, else 1
   const int sc_rows = gs < SK ? SK / gs : 1;
-  const uint32_t tx = CODE_BYTES + sc_rows * 128 + 4 * C::MB * 128;
+  const uint32_t tx = CODE_BYTES + 4 * x_rows * 128 + sc_rows * 64 * C::SB;
 
-  if (warp == 0) {
+  float acc[4][NT][4];
+#pragma unroll
+  for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[rt][j][c] = 0.f;
+  const int g = lane >> 2, t = lane & 3;
+
+  if (warp == kFwdConsumers) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       auto load_weights = [&](int it) {
@@ -135,12 +147,12 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         uint8_t* st = smem + s * C::STAGE;
         tma_load_2d(st, &map_pk, &ctl->full[s], kc, n0 / 2);
         tma_load_2d(st + CODE_BYTES / 2, &map_pk, &ctl->full[s], kc + 128, n0 / 2);
-        tma_load_2d(st + CODE_BYTES, &map_sc, &ctl->full[s], n0, kc >> gsl);
+        tma_load_2d(st + C::OFF_SC, &map_sc, &ctl->full[s], n0, kc >> gsl);
       };
       auto load_x = [&](int it) {
         const int s = it % C::ST;
         const int kc = (st_begin + it) * SK;
-        uint8_t* xs = smem + s * C::STAGE + CODE_BYTES + SC_BYTES;
+        uint8_t* xs = smem + s * C::STAGE + C::OFF_X;
 #pragma unroll
         for (int b = 0; b < 4; ++b) tma_load_2d(xs + b * C::XBOX, &map_x, &ctl->full[s], kc + 64 * b, tok0);
       };
@@ -168,96 +180,121 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   } else {
     // ------------------------------------------------------------ consumers
     griddep_wait();   // outputs of this kernel may still be read by the previous one
-    const int cw = warp - 1, w = cw & (kRowGroups - 1), bs = cw >> 2, g = lane >> 2, t = lane & 3;
-    const int r = pair_of(w, g);   // pair row in the CTA: rows n0 + 2r (even), n0 + 2r + 1 (odd)
+    const int w = warp;   // 64-column block of every stage
     // per-thread shared-memory offsets inside a stage: 16-byte code chunk t of
-    // block bs (128-byte swizzle inside the [32 pairs][128 B] box bs / 2)
-    const uint32_t code_off = (bs >> 1) * (CODE_BYTES / 2) + r * 128 + 16 * ((4 * (bs & 1) + t) ^ (r & 7));
-    uint32_t x_off[NT][4];  // token 8 j + g, columns 16 i + 4 t .. + 3 of the [MB][64] box bs
+    // block w (128-byte swizzle inside the [32 pairs][128 B] box w / 2) for the
+    // pair row of each row tile
+    uint32_t code_off[4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+    for (int rt = 0; rt < 4; ++rt) {
+      const int r = pair_of(rt, g);
+      code_off[rt] = (w >> 1) * (CODE_BYTES / 2) + r * 128 + 16 * ((4 * (w & 1) + t) ^ (r & 7));
+    }
+    // activation fragment: token row min(8 j + g, Mz - 1) of box w, columns
+    // 16 i + 4 t .. + 3 (lanes past the last token repeat it: for one token
+    // every lane of a quad position reads the same 8 bytes)
+    uint32_t x_off[NT][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int row = 8 * j + g;
-        x_off[j][i] = CODE_BYTES + SC_BYTES + bs * C::XBOX + row * 128 + 16 * ((2 * i + (t >> 1)) ^ (row & 7)) +
-                      8 * (t & 1);
-      }
-    // scale words of block bs: row (64 bs + 16 SPG q) >> gsl of the stage's box
-    // (stages start on multiples of 256 columns), half2 of pair r
-    uint32_t sc_off[4];
+    for (int j = 0; j < NT; ++j) {
+      const int row = min(8 * j + g, Mz - 1);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int col = 64 * bs + (SPG == 4 ? 0 : 16 * SPG * q);
-      sc_off[q] = CODE_BYTES + (uint32_t)(gs < SK ? (col >> gsl) : 0) * 128 + 4 * r;
+      for (int i = 0; i < 4; ++i)
+        x_off[j][i] = C::OFF_X + w * C::XBOX + row * 128 + 16 * ((2 * i + (t >> 1)) ^ (row & 7)) + 8 * (t & 1);
+    }
+    // scale words of block w: row (64 w + 16 SPG q) >> gsl of the stage's box
+    // (stages start on multiples of 256 columns), the (even, odd) pair of pair
+    // perm(g) of row tile 0 (+ 16 scales per row tile)
+    uint32_t sc_off[NGB];
+#pragma unroll
+    for (int q = 0; q < NGB; ++q) {
+      const int col = 64 * w + (SPG == 4 ? 0 : 16 * SPG * q);
+      sc_off[q] = C::OFF_SC + (uint32_t)(gs < SK ? (col >> gsl) : 0) * 64 * C::SB + 2 * C::SB * pair_of(0, g);
     }
 
-    float acc[NT][4], part[2][NT][4];
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[j][c] = part[0][j][c] = part[1][j][c] = 0.f;
-    auto flush = [&](uint32_t s_word) {
-      const __half2 s2 = u32_as_h2(s_word);
-      const float se = __low2float(s2), so = __high2float(s2);
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        acc[j][0] = fmaf(part[0][j][0] + part[1][j][0], se, acc[j][0]);
-        acc[j][1] = fmaf(part[0][j][1] + part[1][j][1], se, acc[j][1]);
-        acc[j][2] = fmaf(part[0][j][2] + part[1][j][2], so, acc[j][2]);
-        acc[j][3] = fmaf(part[0][j][3] + part[1][j][3], so, acc[j][3]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) part[0][j][c] = part[1][j][c] = 0.f;
-      }
-    };
-
+    float part[4][NT][4];
+    bool fresh = true;   // the next MMA starts a new group (zero accumulator)
     for (int it = 0; it < nit; ++it) {
       const int s = it % C::ST;
       if (!mbar_wait(&ctl->full[s], (it / C::ST) & 1, abort_flag, &g_device_error, 128u)) break;
       const uint32_t st = sbase + s * C::STAGE;
-      const uint4 wv = lds128(st + code_off);
-      const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+      uint4 wv[4];
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt) wv[rt] = lds128(st + code_off[rt]);
       uint2 xv[NT][4];
 #pragma unroll
       for (int j = 0; j < NT; ++j)
 #pragma unroll
         for (int i = 0; i < 4; ++i) xv[j][i] = lds64(st + x_off[j][i]);
-      uint32_t sw[4];
+      uint2 sw[4][NGB];
 #pragma unroll
-      for (int q = 0; q < (SPG == 4 ? 1 : 4 / SPG); ++q) sw[q] = lds32(st + sc_off[q]);
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int q = 0; q < NGB; ++q) {
+          const uint32_t a = st + sc_off[q] + 16 * C::SB * rt;
+          sw[rt][q] = F32S ? lds64(a) : make_uint2(lds32(a), 0u);
+        }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
+
+      auto flush = [&](int q) {   // scale the finished group of every row tile into acc
+#pragma unroll
+        for (int rt = 0; rt < 4; ++rt) {
+          const float2 sp = scale_pair<F32S>(sw[rt][q]);
+          const float se = sp.x, so = sp.y;
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            acc[rt][j][0] = fmaf(part[rt][j][0], se, acc[rt][j][0]);
+            acc[rt][j][1] = fmaf(part[rt][j][1], se, acc[rt][j][1]);
+            acc[rt][j][2] = fmaf(part[rt][j][2], so, acc[rt][j][2]);
+            acc[rt][j][3] = fmaf(part[rt][j][3], so, acc[rt][j][3]);
+          }
+        }
+      };
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const RowPairs rp = codes_minus8_rows(words[i]);
-        const uint32_t a[4] = {h2_as_u32(rp.ev01), h2_as_u32(rp.od01), h2_as_u32(rp.ev23), h2_as_u32(rp.od23)};
+        const bool first = SPG == 4 ? (i == 0 && fresh) : (i % SPG == 0);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          const uint32_t bf[2] = {xv[j][i].x, xv[j][i].y};
-          mma_16816(part[i & 1][j], a, bf);
+        for (int rt = 0; rt < 4; ++rt) {
+          const uint32_t word = i == 0 ? wv[rt].x : i == 1 ? wv[rt].y : i == 2 ? wv[rt].z : wv[rt].w;
+          const RowPairs rp = codes_minus8_rows(word);
+          const uint32_t a[4] = {h2_as_u32(rp.ev01), h2_as_u32(rp.od01), h2_as_u32(rp.ev23), h2_as_u32(rp.od23)};
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            const uint32_t bf[2] = {xv[j][i].x, xv[j][i].y};
+            if (first) mma_16816_zero(part[rt][j], a, bf);
+            else mma_16816(part[rt][j], a, bf);
+          }
         }
-        if (SPG == 1) flush(sw[i]);
-        if (SPG == 2 && (i & 1)) flush(sw[i >> 1]);
+        if (SPG < 4 && (i % SPG) == SPG - 1) flush(i / SPG);
       }
       if (SPG == 4) {
-        // this warp's next block (one stage later) starts another group, or
-        // the split ends here
-        const int k0 = (st_begin + it) * SK + 64 * bs;
-        if (((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1) flush(sw[0]);
+        // this warp's block of the next stage starts another group, or the split ends here
+        const int k0 = (st_begin + it) * SK + 64 * w;
+        fresh = ((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1;
+        if (fresh) flush(0);
       }
     }
-    // D fragment: rows g (even n of pair r) and g + 8 (odd n), tokens 2t, 2t+1 of tile j
-    float* rs = red + bs * 16 * 64;
+  }
+
+  // warp partials -> [warp][token][row]; the four block slices summed in order
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(smem);
+  if (warp < kFwdConsumers) {
+    float* rs = red + warp * 16 * 64;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      rs[(8 * j + 2 * t) * 64 + 2 * r] = acc[j][0];
-      rs[(8 * j + 2 * t + 1) * 64 + 2 * r] = acc[j][1];
-      rs[(8 * j + 2 * t) * 64 + 2 * r + 1] = acc[j][2];
-      rs[(8 * j + 2 * t + 1) * 64 + 2 * r + 1] = acc[j][3];
+    for (int rt = 0; rt < 4; ++rt) {
+      const int r = pair_of(rt, g);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        rs[(8 * j + 2 * t) * 64 + 2 * r] = acc[rt][j][0];
+        rs[(8 * j + 2 * t + 1) * 64 + 2 * r] = acc[rt][j][1];
+        rs[(8 * j + 2 * t) * 64 + 2 * r + 1] = acc[rt][j][2];
+        rs[(8 * j + 2 * t + 1) * 64 + 2 * r + 1] = acc[rt][j][3];
+      }
     }
   }
-  // the four block slices, summed in order into slice 0
   __syncthreads();
-  for (int e = threadIdx.x; e < Mz * 64; e += kThreads)
+  for (int e = threadIdx.x; e < Mz * 64; e += kFwdThreads)
     red[e] = ((red[e] + red[16 * 64 + e]) + red[2 * 16 * 64 + e]) + red[3 * 16 * 64 + e];
 
   // Rank rk of the cluster sums tokens [rk Mz / S, (rk + 1) Mz / S) of the S
@@ -268,7 +305,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   if (!(S > 1 ? cluster_any_abort(cluster, &ctl->abort, S) : *abort_flag)) {
     const int rk = S > 1 ? (int)cluster.block_rank() : 0;
     const int tb = rk * Mz / S, te = (rk + 1) * Mz / S;
-    for (int e = threadIdx.x; e < (te - tb) * 64; e += kThreads) {
+    for (int e = threadIdx.x; e < (te - tb) * 64; e += kFwdThreads) {
       const int tok = tb + (e >> 6), nl = e & 63;
       const int n = n0 + nl;
       if (n >= N) continue;
@@ -301,14 +338,15 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
 constexpr int kBwdConsumers = 8;
 constexpr int kBwdThreads = 32 * (1 + kBwdConsumers);
 constexpr int BWD_CODE_BYTES = 64 * 128;   // 64 pairs x 128 columns
-constexpr int BWD_SC_BYTES = 8 * 256;      // up to 8 scale rows of 128 n
 
-template <int NT>
+template <int NT, bool F32S>
 struct BwdCfg {
+  static constexpr int SB = F32S ? 4 : 2;                          // bytes per scale
+  static constexpr int SCB = 8 * 128 * SB;                         // up to 8 scale rows of 128 n
   static constexpr int MB = 8 * NT;
   static constexpr int DBOX = MB * 128 < 1024 ? 1024 : MB * 128;   // one [MB][64 n] box
-  static constexpr int STAGE = BWD_CODE_BYTES + BWD_SC_BYTES + 2 * DBOX;
-  static constexpr int ST = NT == 1 ? 8 : 7;
+  static constexpr int STAGE = BWD_CODE_BYTES + SCB + 2 * DBOX;
+  static constexpr int ST = NT == 1 ? (F32S ? 7 : 8) : (F32S ? 6 : 7);
   static constexpr int OFF_CTL = ST * STAGE;
   static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
   static constexpr int RED_FLOATS = kBwdConsumers * MB * 128;   // warp partials, reuse the ring
@@ -317,13 +355,13 @@ struct BwdCfg {
   static_assert(BYTES <= 113 * 1024, "two CTAs per SM");
 };
 
-template <int NT, int SPB>  // SPB scale groups per 64-column block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
+template <int NT, int SPB, bool F32S>  // SPB scale groups per 64-column block: 1 (gs >= 64), 2 (gs 32), 4 (gs 16)
 __global__ void __launch_bounds__(kBwdThreads, 2)
 q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
                     const __grid_constant__ CUtensorMap map_d, float* __restrict__ dx, int M, int N, int K,
                     int gs, int stages_total) {
   using namespace sm100;
-  using C = BwdCfg<NT>;
+  using C = BwdCfg<NT, F32S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
@@ -354,7 +392,7 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     prefetch_tmap(&map_d);
   }
   __syncthreads();
-  const uint32_t tx = BWD_CODE_BYTES + sc_rows * 256 + 2 * C::MB * 128;
+  const uint32_t tx = BWD_CODE_BYTES + sc_rows * 128 * C::SB + 2 * C::MB * 128;
 
   float acc[NT][8][4];
 #pragma unroll
@@ -378,7 +416,7 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
       auto load_d = [&](int it) {
         const int s = it % C::ST;
         const int n0 = (st_begin + it) * 128;
-        uint8_t* ds = smem + s * C::STAGE + BWD_CODE_BYTES + BWD_SC_BYTES;
+        uint8_t* ds = smem + s * C::STAGE + BWD_CODE_BYTES + C::SCB;
         tma_load_2d(ds, &map_d, &ctl->full[s], n0, tok0);
         tma_load_2d(ds + C::DBOX, &map_d, &ctl->full[s], n0 + 64, tok0);
       };
@@ -415,9 +453,9 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     for (int j = 0; j < NT; ++j) {
       const int row = 8 * j + g;
       const int nA = 2 * rowA, nB = 2 * rowB;      // 0..127 within the stage
-      dA[j] = BWD_CODE_BYTES + BWD_SC_BYTES + (nA >> 6) * C::DBOX + row * 128 +
+      dA[j] = BWD_CODE_BYTES + C::SCB + (nA >> 6) * C::DBOX + row * 128 +
               16 * ((((nA & 63) * 2) >> 4) ^ (row & 7)) + (((nA & 63) * 2) & 15);
-      dB[j] = BWD_CODE_BYTES + BWD_SC_BYTES + (nB >> 6) * C::DBOX + row * 128 +
+      dB[j] = BWD_CODE_BYTES + C::SCB + (nB >> 6) * C::DBOX + row * 128 +
               16 * ((((nB & 63) * 2) >> 4) ^ (row & 7)) + (((nB & 63) * 2) & 15);
     }
     // scale half2 of pairs rowA / rowB in the row of each column group
@@ -426,8 +464,8 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     for (int q = 0; q < SPB; ++q) {
       const int col = 64 * J + 16 * (q * (4 / SPB)) + 4 * (g & 3);
       const int r = ((kbase + col) >> gsl) - (kbase >> gsl);
-      scA[q] = BWD_CODE_BYTES + r * 256 + 4 * rowA;
-      scB[q] = BWD_CODE_BYTES + r * 256 + 4 * rowB;
+      scA[q] = BWD_CODE_BYTES + r * 128 * C::SB + 2 * C::SB * rowA;
+      scB[q] = BWD_CODE_BYTES + r * 128 * C::SB + 2 * C::SB * rowB;
     }
     for (int it = 0; it < nit; ++it) {
       const int s = it % C::ST;
@@ -440,11 +478,11 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         bfr[j][0] = lds32(st + dA[j]);
         bfr[j][1] = lds32(st + dB[j]);
       }
-      uint32_t sa[SPB], sb[SPB];
+      uint2 sa[SPB], sb[SPB];
 #pragma unroll
       for (int q = 0; q < SPB; ++q) {
-        sa[q] = lds32(st + scA[q]);
-        sb[q] = lds32(st + scB[q]);
+        sa[q] = F32S ? lds64(st + scA[q]) : make_uint2(lds32(st + scA[q]), 0u);
+        sb[q] = F32S ? lds64(st + scB[q]) : make_uint2(lds32(st + scB[q]), 0u);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
@@ -453,15 +491,18 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int q = i / (4 / SPB);
-        const __half2 hsa = u32_as_h2(sa[q]), hsb = u32_as_h2(sb[q]);
+        auto op = [&](__half2 c, uint2 sw) -> uint32_t {   // one byte's (even n, odd n) weights, scaled
+          if (F32S) return weight_pair_f32s(c, __uint_as_float(sw.x), __uint_as_float(sw.y));
+          return h2_as_u32(__hmul2(c, u32_as_h2(sw.x)));
+        };
         const ColPairs ca = codes_minus8_cols(wa[i]);
         const ColPairs cb = codes_minus8_cols(wb[i]);
         const __half2 la[4] = {ca.c0, ca.c1, ca.c2, ca.c3};
         const __half2 lb[4] = {cb.c0, cb.c1, cb.c2, cb.c3};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint32_t af[4] = {h2_as_u32(__hmul2(la[2 * h], hsa)), h2_as_u32(__hmul2(la[2 * h + 1], hsa)),
-                                  h2_as_u32(__hmul2(lb[2 * h], hsb)), h2_as_u32(__hmul2(lb[2 * h + 1], hsb))};
+          const uint32_t af[4] = {op(la[2 * h], sa[q]), op(la[2 * h + 1], sa[q]), op(lb[2 * h], sb[q]),
+                                  op(lb[2 * h + 1], sb[q])};
 #pragma unroll
           for (int j = 0; j < NT; ++j) mma_16816(acc[j][2 * i + h], af, bfr[j]);
         }
@@ -519,12 +560,12 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int NT, int SPG>
+template <int NT, int SPG, bool F32S>
 static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUtensorMap& map_sc,
                                            const CUtensorMap& map_x, OutSplit out, int M, int N, int K, int gs,
-                                           int stages_total, dim3 grid, cudaStream_t stream) {
-  using C = gv::Cfg<NT>;
-  auto kern = gv::q4gsw_gemv_fwd_tma_kernel<NT, SPG>;
+                                           int stages_total, int x_rows, dim3 grid, cudaStream_t stream) {
+  using C = gv::FwdCfg<NT, SPG, F32S>;
+  auto kern = gv::q4gsw_gemv_fwd_tma_kernel<NT, SPG, F32S>;
   static PerDeviceOnce attr_once;
   {
     cudaError_t e = once_per_device(attr_once, current_device(), [&] {
@@ -534,7 +575,7 @@ static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUte
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(gv::kThreads, 1, 1);
+  cfg.blockDim = dim3(gv::kFwdThreads, 1, 1);
   cfg.dynamicSmemBytes = C::BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -546,55 +587,63 @@ static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUte
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, map_x, out, M, N, K, gs, stages_total);
+  return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, x_rows);
 }
 
-cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
-                                cudaStream_t stream, char* route, int route_len) {
+cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M,
+                                OutSplit out, cudaStream_t stream, char* route, int route_len) {
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
-  const Layout L = layout_of(N, K, gs);
+  const int sb = f32s ? 4 : 2;
+  const Layout L = layout_of(N, K, gs, sb);
   const int G = K / gs;
   const int NT = (M <= 8) ? 1 : 2;
   const int zs = (M + 15) / 16;
   const int tiles = (N + 63) / 64;
   const int stages_total = (K + gv::SK - 1) / gv::SK;
-  // fill the resident CTA slots in one wave, at least two stages per split,
-  // clusters of at most 8
-  const int sms = sm_count(current_device());
-  const int slots = sms * (NT == 1 ? gv::Cfg<1>::kCtasPerSm : gv::Cfg<2>::kCtasPerSm);
+  const int spg = gs == 16 ? 1 : gs == 32 ? 2 : 4;
+  // Contraction splits: fill the resident CTA slots in one wave, at least two
+  // stages per split, clusters of at most 8.
+  const int per_sm = f32s ? (NT == 1 ? (spg == 1 ? gv::FwdCfg<1, 1, true>::CTAS : gv::FwdCfg<1, 4, true>::CTAS)
+                                     : (spg == 1 ? gv::FwdCfg<2, 1, true>::CTAS : gv::FwdCfg<2, 4, true>::CTAS))
+                          : (NT == 1 ? (spg == 1 ? gv::FwdCfg<1, 1, false>::CTAS : gv::FwdCfg<1, 4, false>::CTAS)
+                                     : (spg == 1 ? gv::FwdCfg<2, 1, false>::CTAS : gv::FwdCfg<2, 4, false>::CTAS));
+  const int slots = sm_count(current_device()) * per_sm;
   int S = slots / (tiles * zs);
   S = S < 1 ? 1 : (S > 8 ? 8 : S);
   while (S > 1 && stages_total / S < 2) --S;
   const int sc_rows = gs < gv::SK ? gv::SK / gs : 1;
+  const int x_rows = NT == 1 ? (M < 8 ? M : 8) : 16;
   CUtensorMap map_pk, map_sc, map_x;
   const bool ok =
       make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, gv::RP, CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pk + L.scales_offset, N, G, (uint64_t)N * 2, 64, sc_rows,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, (uint64_t)K * 2, 64, 8 * NT,
+      make_map_2d(&map_sc, f32s ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  pk + L.scales_offset, N, G, (uint64_t)N * sb, 64, sc_rows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, (uint64_t)K * 2, 64, x_rows,
                   CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
-  const int spg = gs == 16 ? 1 : gs == 32 ? 2 : 4;
   const dim3 grid(tiles, S, zs);
   cudaError_t e;
+#define Q4_TMA_FWD(NT_, SPG_)                                                                                         \
+  (f32s ? launch_gemv_tma_variant<NT_, SPG_, true>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, x_rows, grid, \
+                                                   stream)                                                             \
+        : launch_gemv_tma_variant<NT_, SPG_, false>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, x_rows,     \
+                                                    grid, stream))
   if (NT == 1)
-    e = spg == 1 ? launch_gemv_tma_variant<1, 1>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
-      : spg == 2 ? launch_gemv_tma_variant<1, 2>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
-                 : launch_gemv_tma_variant<1, 4>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream);
+    e = spg == 1 ? Q4_TMA_FWD(1, 1) : spg == 2 ? Q4_TMA_FWD(1, 2) : Q4_TMA_FWD(1, 4);
   else
-    e = spg == 1 ? launch_gemv_tma_variant<2, 1>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
-      : spg == 2 ? launch_gemv_tma_variant<2, 2>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream)
-                 : launch_gemv_tma_variant<2, 4>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, grid, stream);
+    e = spg == 1 ? Q4_TMA_FWD(2, 1) : spg == 2 ? Q4_TMA_FWD(2, 2) : Q4_TMA_FWD(2, 4);
+#undef Q4_TMA_FWD
   if (route)
     snprintf(route, route_len, "gemv_tma_fwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S,
              zs, stages_total);
   return e;
 }
 
-cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
-                                cudaStream_t stream, char* route, int route_len) {
+cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M,
+                                float* d_x, cudaStream_t stream, char* route, int route_len) {
   const uint8_t* pk = static_cast<const uint8_t*>(packed);
-  const Layout L = layout_of(N, K, gs);
+  const int sb = f32s ? 4 : 2;
+  const Layout L = layout_of(N, K, gs, sb);
   const int G = K / gs;
   const int NT = (M <= 8) ? 1 : 2;
   const int zs = (M + 15) / 16;
@@ -609,7 +658,8 @@ cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const 
   CUtensorMap map_pk, map_sc, map_d;
   const bool ok =
       make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_map_2d(&map_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pk + L.scales_offset, N, G, (uint64_t)N * 2, 128,
+      make_map_2d(&map_sc, f32s ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  pk + L.scales_offset, N, G, (uint64_t)N * sb, 128,
                   sc_rows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
       make_map_2d(&map_d, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, d_out, N, M, (uint64_t)N * 2, 64, 8 * NT,
                   CU_TENSOR_MAP_SWIZZLE_128B);
@@ -636,14 +686,14 @@ cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const 
     return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, map_d, d_x, M, N, K, gs, stages_total);
   };
   cudaError_t e;
+#define Q4_TMA_BWD(NT_, SPB_)                                                                        \
+  (f32s ? launch(gv::q4gsw_gemv_bwd_tma_kernel<NT_, SPB_, true>, gv::BwdCfg<NT_, true>::BYTES)       \
+        : launch(gv::q4gsw_gemv_bwd_tma_kernel<NT_, SPB_, false>, gv::BwdCfg<NT_, false>::BYTES))
   if (NT == 1)
-    e = spb == 1 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<1, 1>, gv::BwdCfg<1>::BYTES)
-      : spb == 2 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<1, 2>, gv::BwdCfg<1>::BYTES)
-                 : launch(gv::q4gsw_gemv_bwd_tma_kernel<1, 4>, gv::BwdCfg<1>::BYTES);
+    e = spb == 1 ? Q4_TMA_BWD(1, 1) : spb == 2 ? Q4_TMA_BWD(1, 2) : Q4_TMA_BWD(1, 4);
   else
-    e = spb == 1 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<2, 1>, gv::BwdCfg<2>::BYTES)
-      : spb == 2 ? launch(gv::q4gsw_gemv_bwd_tma_kernel<2, 2>, gv::BwdCfg<2>::BYTES)
-                 : launch(gv::q4gsw_gemv_bwd_tma_kernel<2, 4>, gv::BwdCfg<2>::BYTES);
+    e = spb == 1 ? Q4_TMA_BWD(2, 1) : spb == 2 ? Q4_TMA_BWD(2, 2) : Q4_TMA_BWD(2, 4);
+#undef Q4_TMA_BWD
   if (route)
     snprintf(route, route_len, "gemv_tma_bwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S,
              zs, stages_total);

@@ -38,10 +38,11 @@ inline cudaError_t once_per_device(PerDeviceOnce& o, int dev, F&& fn) {
 int current_device();
 int sm_count(int dev);
 
-cudaError_t launch_prepack(const uint8_t* codes, const uint16_t* scales, int N, int K, int gs,
-                           void* packed, cudaStream_t stream, uint32_t* host_flag);
+// f32s: the blob holds fp32 scales (packed layout version 2) instead of fp16.
+cudaError_t launch_prepack(const uint8_t* codes, const void* scales, int N, int K, int gs, bool f32s, void* packed,
+                           cudaStream_t stream, uint32_t* host_flag);
 cudaError_t launch_unpack(const void* packed, int N, int K, uint8_t* codes, cudaStream_t stream);
-cudaError_t launch_dequant(const void* packed, int N, int K, int gs, float* w32, uint16_t* w16,
+cudaError_t launch_dequant(const void* packed, int N, int K, int gs, bool f32s, float* w32, uint16_t* w16,
                            cudaStream_t stream);
 
 // Output columns [0, N) of a forward split over up to three row-major
@@ -56,29 +57,31 @@ struct OutSplit {
 
 __host__ __device__ inline OutSplit single_output(float* y, int N) { return OutSplit{y, y, y, N, N, N}; }
 
+// The compute launchers take f32s = the packed blob has fp32 scales (layout
+// version 2) instead of fp16 (version 1).
 // Tensor-core GEMV routes for small token counts.  `M` may exceed 16: token
 // chunks of 16 then run as grid z-slices (each re-reads the weight).
-cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M,
+cudaError_t launch_gemv_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M,
                             OutSplit out, cudaStream_t stream, char* route, int route_len);
-cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M,
+cudaError_t launch_gemv_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M,
                             float* d_x, cudaStream_t stream, char* route, int route_len);
 
 // Forward GEMV that streams the packed weight through a TMA ring (M <= 16
 // per z-slice).
-cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
+cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M, OutSplit out,
                                 cudaStream_t stream, char* route, int route_len);
-cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
+cudaError_t launch_gemv_tma_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M, float* d_x,
                                 cudaStream_t stream, char* route, int route_len);
 
 // tcgen05 GEMM routes (any M >= 1; used above the GEMV range).
-cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, const uint16_t* x, int M, OutSplit out,
+cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M, OutSplit out,
                             cudaStream_t stream, char* route, int route_len);
-cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, const uint16_t* d_out, int M, float* d_x,
+cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M, float* d_x,
                             cudaStream_t stream, char* route, int route_len);
 
 // Embedding rows out[t] = dequant(W)[indices[t]] (fp32); an index outside
 // [0, N) gives a zero row and sets kIndexErrorBit in the device error word.
-cudaError_t launch_embedding(const void* packed, int N, int K, int gs, const int32_t* indices, int T, float* out,
+cudaError_t launch_embedding(const void* packed, int N, int K, int gs, bool f32s, const int32_t* indices, int T, float* out,
                              cudaStream_t stream);
 
 // One thread block that waits on a barrier nothing completes until its

@@ -45,11 +45,12 @@ __global__ void q4gsw_prepack_codes_kernel(const uint8_t* __restrict__ codes, ui
   if (bad) atomicOr(range_flag, 1u);
 }
 
-// Scales copy, zero padding and trailer words 0..4 (word 5, the range flag, is
-// zeroed by the host before this runs and only ever OR-ed).
-__global__ void q4gsw_prepack_tail_kernel(const uint16_t* __restrict__ scales, uint8_t* __restrict__ packed,
-                                    int N, int K, int gs) {
-  const Layout L = layout_of(N, K, gs);
+// Scales copy (fp16 or fp32: sbytes per scale), zero padding and trailer
+// words 0..4 (word 5, the range flag, is zeroed by the host before this runs
+// and only ever OR-ed).
+__global__ void q4gsw_prepack_tail_kernel(const void* __restrict__ scales, uint8_t* __restrict__ packed,
+                                          int N, int K, int gs, int sbytes) {
+  const Layout L = layout_of(N, K, gs, sbytes);
   const size_t tid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   const size_t n16 = L.scales_bytes / 16;  // N % 8 == 0 -> a whole number of 16-byte vectors
@@ -61,7 +62,7 @@ __global__ void q4gsw_prepack_tail_kernel(const uint16_t* __restrict__ scales, u
   if (tid == 0) {
     uint32_t* tr = reinterpret_cast<uint32_t*>(packed + L.trailer_offset);
     tr[0] = kTrailerMagic;
-    tr[1] = kLayoutVersion;
+    tr[1] = sbytes == 4 ? kLayoutVersionF32S : kLayoutVersion;
     tr[2] = uint32_t(N);
     tr[3] = uint32_t(K);
     tr[4] = uint32_t(gs);
@@ -91,12 +92,13 @@ __global__ void q4gsw_unpack_kernel(const uint8_t* __restrict__ packed, uint8_t*
 }
 
 // The dequantised weight, produced with the same conversions the GEMM
-// kernels use: w16 = fp16((code - 8)) * scale rounded once (HMUL2), and the
-// exact fp32 product w32.
+// kernels use.  fp16 scales (F32S false): w16 = fp16((code - 8)) * scale
+// rounded once (HMUL2), and the exact fp32 product w32.  fp32 scales (layout
+// version 2): w32 = (code - 8) * s32 rounded once in fp32, w16 = fp16_RNE(w32).
+template <bool F32S>
 __global__ void q4gsw_dequant_kernel(const uint8_t* __restrict__ packed, float* __restrict__ w32,
-                               uint16_t* __restrict__ w16, int N, int K, int gs) {
-  const Layout L = layout_of(N, K, gs);
-  const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
+                                     uint16_t* __restrict__ w16, int N, int K, int gs) {
+  const Layout L = layout_of(N, K, gs, F32S ? 4 : 2);
   const int blocks_per_row = K / 64;
   const long long chunks = (long long)(N / 2) * blocks_per_row * 4;
   for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < chunks;
@@ -111,24 +113,39 @@ __global__ void q4gsw_dequant_kernel(const uint8_t* __restrict__ packed, float* 
     for (int i = 0; i < 4; ++i) {
       const int k0 = 64 * b + 16 * i + 4 * t;  // columns k0 .. k0+3
       const int g = k0 >> (__ffs(gs) - 1);
-      const __half2 s2 = *reinterpret_cast<const __half2*>(scales + (size_t)g * N + 2 * p);
-      const __half2 se = __low2half2(s2), so = __high2half2(s2);
       const RowPairs r = codes_minus8_rows(w[i]);
-      const __half2 e01 = __hmul2(r.ev01, se), e23 = __hmul2(r.ev23, se);
-      const __half2 o01 = __hmul2(r.od01, so), o23 = __hmul2(r.od23, so);
       const size_t re = (size_t)(2 * p) * K + k0, ro = re + K;
-      if (w16) {
-        *reinterpret_cast<uint2*>(w16 + re) = make_uint2(h2_as_u32(e01), h2_as_u32(e23));
-        *reinterpret_cast<uint2*>(w16 + ro) = make_uint2(h2_as_u32(o01), h2_as_u32(o23));
+      float4 fe, fo;
+      if (F32S) {
+        const float2 s2 = *reinterpret_cast<const float2*>(
+            reinterpret_cast<const float*>(packed + L.scales_offset) + (size_t)g * N + 2 * p);
+        fe = make_float4(__fmul_rn(__low2float(r.ev01), s2.x), __fmul_rn(__high2float(r.ev01), s2.x),
+                         __fmul_rn(__low2float(r.ev23), s2.x), __fmul_rn(__high2float(r.ev23), s2.x));
+        fo = make_float4(__fmul_rn(__low2float(r.od01), s2.y), __fmul_rn(__high2float(r.od01), s2.y),
+                         __fmul_rn(__low2float(r.od23), s2.y), __fmul_rn(__high2float(r.od23), s2.y));
+        if (w16) {
+          *reinterpret_cast<uint2*>(w16 + re) = make_uint2(h2_as_u32(__floats2half2_rn(fe.x, fe.y)),
+                                                           h2_as_u32(__floats2half2_rn(fe.z, fe.w)));
+          *reinterpret_cast<uint2*>(w16 + ro) = make_uint2(h2_as_u32(__floats2half2_rn(fo.x, fo.y)),
+                                                           h2_as_u32(__floats2half2_rn(fo.z, fo.w)));
+        }
+      } else {
+        const __half2 s2 = *reinterpret_cast<const __half2*>(
+            reinterpret_cast<const __half*>(packed + L.scales_offset) + (size_t)g * N + 2 * p);
+        const __half2 se = __low2half2(s2), so = __high2half2(s2);
+        if (w16) {
+          *reinterpret_cast<uint2*>(w16 + re) = make_uint2(h2_as_u32(__hmul2(r.ev01, se)), h2_as_u32(__hmul2(r.ev23, se)));
+          *reinterpret_cast<uint2*>(w16 + ro) = make_uint2(h2_as_u32(__hmul2(r.od01, so)), h2_as_u32(__hmul2(r.od23, so)));
+        }
+        const float ffe = __low2float(s2), ffo = __high2float(s2);
+        fe = make_float4(__low2float(r.ev01) * ffe, __high2float(r.ev01) * ffe, __low2float(r.ev23) * ffe,
+                         __high2float(r.ev23) * ffe);
+        fo = make_float4(__low2float(r.od01) * ffo, __high2float(r.od01) * ffo, __low2float(r.od23) * ffo,
+                         __high2float(r.od23) * ffo);
       }
       if (w32) {
-        const float fe = __low2float(s2), fo = __high2float(s2);
-        *reinterpret_cast<float4*>(w32 + re) =
-            make_float4(__low2float(r.ev01) * fe, __high2float(r.ev01) * fe,
-                        __low2float(r.ev23) * fe, __high2float(r.ev23) * fe);
-        *reinterpret_cast<float4*>(w32 + ro) =
-            make_float4(__low2float(r.od01) * fo, __high2float(r.od01) * fo,
-                        __low2float(r.od23) * fo, __high2float(r.od23) * fo);
+        *reinterpret_cast<float4*>(w32 + re) = fe;
+        *reinterpret_cast<float4*>(w32 + ro) = fo;
       }
     }
   }
@@ -143,16 +160,18 @@ static int grid_for(long long work, int threads) {
   return int(g);
 }
 
-cudaError_t launch_prepack(const uint8_t* codes, const uint16_t* scales, int N, int K, int gs,
-                           void* packed, cudaStream_t stream, uint32_t* host_flag) {
-  const Layout L = layout_of(N, K, gs);
+cudaError_t launch_prepack(const uint8_t* codes, const void* scales, int N, int K, int gs, bool f32s, void* packed,
+                           cudaStream_t stream, uint32_t* host_flag) {
+  const int sbytes = f32s ? 4 : 2;
+  const Layout L = layout_of(N, K, gs, sbytes);
   uint8_t* out = static_cast<uint8_t*>(packed);
   uint32_t* flag = reinterpret_cast<uint32_t*>(out + L.trailer_offset) + 5;
   cudaError_t err = cudaMemsetAsync(out + L.trailer_offset, 0, kTrailerBytes, stream);
   if (err != cudaSuccess) return err;
   const long long chunks = (long long)(N / 2) * (K / 64) * 4;
   pk::q4gsw_prepack_codes_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(codes, out, N, K, flag);
-  pk::q4gsw_prepack_tail_kernel<<<grid_for((long long)(L.scales_bytes / 16) + 256, 256), 256, 0, stream>>>(scales, out, N, K, gs);
+  pk::q4gsw_prepack_tail_kernel<<<grid_for((long long)(L.scales_bytes / 16) + 256, 256), 256, 0, stream>>>(
+      scales, out, N, K, gs, sbytes);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   err = cudaMemcpyAsync(host_flag, flag, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream);
@@ -166,10 +185,14 @@ cudaError_t launch_unpack(const void* packed, int N, int K, uint8_t* codes, cuda
   return cudaGetLastError();
 }
 
-cudaError_t launch_dequant(const void* packed, int N, int K, int gs, float* w32, uint16_t* w16,
+cudaError_t launch_dequant(const void* packed, int N, int K, int gs, bool f32s, float* w32, uint16_t* w16,
                            cudaStream_t stream) {
   const long long chunks = (long long)(N / 2) * (K / 64) * 4;
-  pk::q4gsw_dequant_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(static_cast<const uint8_t*>(packed), w32, w16, N, K, gs);
+  const uint8_t* pk = static_cast<const uint8_t*>(packed);
+  if (f32s)
+    pk::q4gsw_dequant_kernel<true><<<grid_for(chunks, 256), 256, 0, stream>>>(pk, w32, w16, N, K, gs);
+  else
+    pk::q4gsw_dequant_kernel<false><<<grid_for(chunks, 256), 256, 0, stream>>>(pk, w32, w16, N, K, gs);
   return cudaGetLastError();
 }
 

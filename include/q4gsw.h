@@ -170,6 +170,64 @@ Q4GSW_API q4gsw_status q4gsw_embedding(const void *packed, int N, int K, int gro
                              const int32_t *indices, int T, float *out,
                              q4gsw_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * fp32-scale variant (packed layout version 2)
+ *
+ * "Upstream the Gemma 4 Vulkan support we carry on our ExecuTorch fork",
+ * issue #1361: the fork carries an fp32-scale dequantise-and-accumulate shader
+ * helper (linear_fp32_scale_dq_acc) beside the fp16-scale q4gsw path; the
+ * Oct 20 comment reports no measurable accuracy gain from it.  The pages name
+ * it only; this library's reading:
+ *   - layout version 2 = the version 1 codes region unchanged, the scales as
+ *     fp32 [G][N] (4 bytes each) at the same 256-byte-aligned offset, then the
+ *     64-byte trailer with version word 2;
+ *   - the dequantised weight is w32[n,k] = fp32_RNE((code[n,k] - 8) * s32[k/gs, n]),
+ *     one rounding (the product of a 4-bit integer and a 24-bit significand
+ *     needs up to 27 bits);
+ *   - the tensor-core GEMMs and the input-gradient GEMVs take fp16_RNE(w32) as
+ *     their operand and accumulate in fp32; the forward GEMVs (M <= 16)
+ *     multiply the fp32 partial sum of each group by s32 in fp32, so they never
+ *     round the weight;
+ *   - every output is fp32 and satisfies the same bound as the fp16-scale path.
+ * The functions below take the same arguments, checks and routes as their
+ * fp16-scale counterparts; a version-1 blob must not be passed to them, nor a
+ * version-2 blob to the fp16-scale functions (the blob's trailer records its
+ * version; the compute calls do not read it).
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of a version-2 blob for (N, K, gs); 0 if the shape is not accepted. */
+Q4GSW_API size_t q4gsw_packed_bytes_f32s(int N, int K, int group_size);
+
+/* One-time packer for fp32 scales: codes uint8 [N, K] (0..15), scales fp32
+ * [K/gs, N] -> version-2 blob.  Same checks, single wait and range-flag
+ * behaviour as q4gsw_prepack. */
+Q4GSW_API q4gsw_status q4gsw_prepack_f32s(const uint8_t *codes, const float *scales,
+                                int N, int K, int group_size,
+                                void *packed, size_t packed_bytes,
+                                q4gsw_stream_t stream);
+
+/* Forward, input gradient and fused Q/K/V forward on a version-2 blob. */
+Q4GSW_API q4gsw_status q4gsw_linear_fwd_f32s(const void *packed, int N, int K, int group_size,
+                                   const uint16_t *x, int M, float *y,
+                                   q4gsw_stream_t stream);
+Q4GSW_API q4gsw_status q4gsw_linear_bwd_input_f32s(const void *packed, int N, int K, int group_size,
+                                         const uint16_t *d_out, int M, float *d_x,
+                                         q4gsw_stream_t stream);
+Q4GSW_API q4gsw_status q4gsw_qkv_fwd_f32s(const void *packed_qkv, int Nq, int Nk, int Nv,
+                                int K, int group_size,
+                                const uint16_t *x, int M,
+                                float *y_q, float *y_k, float *y_v,
+                                q4gsw_stream_t stream);
+
+/* Embedding rows from a version-2 blob: out[t, k] = w32[idx[t], k]. */
+Q4GSW_API q4gsw_status q4gsw_embedding_f32s(const void *packed, int N, int K, int group_size,
+                                  const int32_t *indices, int T, float *out,
+                                  q4gsw_stream_t stream);
+
+/* Debug export: w32 and w16 = fp16_RNE(w32) of a version-2 blob. */
+Q4GSW_API q4gsw_status q4gsw_dequant_f32s(const void *packed, int N, int K, int group_size,
+                                float *w32, uint16_t *w16, q4gsw_stream_t stream);
+
 /*
  * Kernel health check.  Every wait inside this library's kernels is bounded
  * (one second of wall-clock time); a wait that runs out makes its kernel stop

@@ -21,7 +21,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = b.library()
     names = declared_functions()
-    assert len(names) == 14
+    assert len(names) == 21
     assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
     for n in names:
         assert hasattr(lib, n), n
@@ -142,3 +142,20 @@ def test_wait_probe_limit_is_checked_on_the_host():
     lib = b.library()
     assert lib.q4gsw_debug_wait_timeout(0, None) == 2
     assert lib.q4gsw_debug_wait_timeout(1000001, None) == 2
+
+
+def test_f32s_entry_points_check_arguments_on_the_host():
+    import oracle.q4gsw_variants as v
+    lib = b.library()
+    fake = 0x100000
+    assert lib.q4gsw_packed_bytes_f32s(64, 128, 32) == v.packed_layout_f32s(64, 128, 32)["total_bytes"]
+    assert lib.q4gsw_packed_bytes_f32s(62, 128, 32) == 0
+    need = lib.q4gsw_packed_bytes_f32s(64, 128, 32)
+    assert lib.q4gsw_prepack_f32s(fake, fake, 64, 128, 32, fake, need - 1, None) == 7
+    assert lib.q4gsw_prepack_f32s(fake, None, 64, 128, 32, fake, need, None) == 1
+    assert lib.q4gsw_linear_fwd_f32s(fake, 64, 96, 32, fake, 4, fake, None) == 3
+    assert lib.q4gsw_linear_bwd_input_f32s(None, 64, 128, 32, fake, 4, fake, None) == 1
+    assert lib.q4gsw_qkv_fwd_f32s(fake, 64, 20, 20, 128, 32, fake, 4, fake, fake, fake, None) == 3
+    assert lib.q4gsw_embedding_f32s(fake, 64, 128, 32, fake, -1, fake, None) == 2
+    assert lib.q4gsw_dequant_f32s(fake, 64, 128, 32, None, None, None) == 1
+    assert lib.q4gsw_linear_fwd_f32s(None, 64, 128, 32, None, 0, None, None) == 0
