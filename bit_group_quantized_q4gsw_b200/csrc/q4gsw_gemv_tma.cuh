@@ -25,33 +25,43 @@
 namespace q4gsw {
 namespace gv {
 
-constexpr int kFwdConsumers = 4;                        // one 64-column block of every stage each
-constexpr int kFwdThreads = 32 * (kFwdConsumers + 1);   // the last warp produces
 constexpr int RP = 32;                                  // nibble pairs per CTA (64 rows = 4 MMA row tiles)
 constexpr int SK = 256;                                 // contraction columns per stage
 constexpr int CODE_BYTES = RP * SK;                     // two [32 pairs][128 B] boxes, 8 KB
 constexpr int CTL_BYTES = 256;
 
-// Shared-memory map of the forward: ST stages of [codes | 4 activation boxes
-// | scale rows].  Each activation box is [<= 8 NT tokens][64 columns] fp16
-// (128-byte swizzle) in a 1 KB-aligned slot; the scale rows of one stage are
-// 256 / gs rows (at least one) of 64 scales (fp16, or fp32 in layout version 2).
+// Forward configuration for NT 8-token MMA tiles, SPG 16-column steps per
+// scale group, fp32 or fp16 scales.
+//   consumer warps: 4 (one 64-column block of every stage each, all four row
+//   tiles, so one activation fragment feeds four MMAs) for up to 8 tokens;
+//   8 (two per block, two row tiles each) for 9..16, whose twice as many MMAs
+//   per weight need the extra warps (measured on B200, 14336x4096: M=1
+//   12.3 us with 4 warps vs 16.1 us with 8; M=16 17.0 us with 8 vs 20.5 us
+//   with 4).
+//   stage: [codes 8 KB | scale rows], 1 KB aligned.  The scale rows of a stage
+//   are 256 / gs rows (at least one) of 64 scales.  The activations are not
+//   staged: every CTA of the launch reads the same few kilobytes, which stay in
+//   L1 and L2, and each of them would cost the TMA unit a tiny box per stage.
+//   ST: the ring depth that keeps a CTA near 56 KB, so that two CTAs of this
+//   launch and two of the next fit on one SM.
 template <int NT, int SPG, bool F32S>
 struct FwdCfg {
-  static constexpr int SB = F32S ? 4 : 2;   // bytes per scale
-  static constexpr int XBOX = 1024 * NT;
-  static constexpr int SCB = (SPG == 1 ? 2048 : 1024) * (SB / 2);
-  static constexpr int OFF_X = CODE_BYTES;
-  static constexpr int OFF_SC = CODE_BYTES + 4 * XBOX;
-  static constexpr int STAGE = OFF_SC + SCB;
-  static constexpr int ST = 4;
+  static constexpr int CW = NT == 2 ? 8 : 4;                 // consumer warps
+  static constexpr int RTW = 4 / (CW / 4);                   // row tiles per consumer warp
+  static constexpr int THREADS = 32 * (CW + 1);              // the last warp produces
+  // resident CTAs per SM the registers are sized for
+  static constexpr int MINB = NT == 1 ? 4 : 2;
+  static constexpr int SB = F32S ? 4 : 2;                    // bytes per scale
+  static constexpr int SCB = (SPG == 1 ? 16 : SPG == 2 ? 8 : 4) * 64 * SB;
+  static constexpr int OFF_SC = CODE_BYTES;
+  static constexpr int STAGE = (OFF_SC + SCB + 1023) / 1024 * 1024;
+  static constexpr int ST0 = 56 * 1024 / STAGE;
+  static constexpr int ST = ST0 < 3 ? 3 : ST0 > 8 ? 8 : ST0;
   static constexpr int OFF_CTL = ST * STAGE;
   static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
-  // CTAs per SM that fit in 228 KB (1 KB of each is reserved by the system)
-  static constexpr int CTAS = 4 * (BYTES + 1024) <= 233472 ? 4 : 3;
-  static constexpr int RED_FLOATS = kFwdConsumers * 16 * 64;   // [warp][token][row], reuses the ring
-  static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
+  static constexpr int RED_FLOATS = 4 * 16 * 64;             // [block][token][row], reuses the ring
   static_assert(RED_FLOATS * 4 <= OFF_CTL, "warp partials fit in the ring");
+  static_assert(ST <= 12, "barrier arrays");
 };
 
 struct Ctl {
@@ -85,15 +95,15 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 
 // grid = (ceil(N / 64) row tiles, S contraction splits, ceil(M / 16) token
 // slices), cluster = (1, S, 1).  SPG = 16-column steps per scale group
-// (1: gs 16, 2: gs 32, 4: gs >= 64).  x_rows = rows of each activation box
-// (the tokens of a slice: min(M, 8) for one 8-token tile, 16 for two).
+// (1: gs 16, 2: gs 32, 4: gs >= 64).
 template <int NT, int SPG, bool F32S>
-__global__ void __launch_bounds__(kFwdThreads, FwdCfg<NT, SPG, F32S>::CTAS)
+__global__ void __launch_bounds__(FwdCfg<NT, SPG, F32S>::THREADS, FwdCfg<NT, SPG, F32S>::MINB)
 q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
-                          const __grid_constant__ CUtensorMap map_x, OutSplit out, int M, int N, int K, int gs,
-                          int stages_total, int x_rows) {
+                          const __half* __restrict__ x, OutSplit out, int M, int N, int K, int gs,
+                          int stages_total) {
   using namespace sm100;
   using C = FwdCfg<NT, SPG, F32S>;
+  constexpr int RTW = C::RTW;
   constexpr int NGB = SPG == 4 ? 1 : 4 / SPG;   // scale groups per 64-column block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -115,30 +125,29 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::ST; ++i) {
       mbar_init(&ctl->full[i], 1);
-      mbar_init(&ctl->empty[i], kFwdConsumers);
+      mbar_init(&ctl->empty[i], C::CW);
     }
     ctl->abort = 0;
     fence_mbar_init();
     prefetch_tmap(&map_pk);
     prefetch_tmap(&map_sc);
-    prefetch_tmap(&map_x);
   }
   __syncthreads();
 
   // scale rows per stage: 256 / gs for gs <= 256, else 1
   const int sc_rows = gs < SK ? SK / gs : 1;
-  const uint32_t tx = CODE_BYTES + 4 * x_rows * 128 + sc_rows * 64 * C::SB;
+  const uint32_t tx = CODE_BYTES + sc_rows * 64 * C::SB;
 
-  float acc[4][NT][4];
+  float acc[RTW][NT][4];
 #pragma unroll
-  for (int rt = 0; rt < 4; ++rt)
+  for (int rt = 0; rt < RTW; ++rt)
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[rt][j][c] = 0.f;
   const int g = lane >> 2, t = lane & 3;
 
-  if (warp == kFwdConsumers) {
+  if (warp == C::CW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       auto load_weights = [&](int it) {
@@ -149,29 +158,19 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         tma_load_2d(st + CODE_BYTES / 2, &map_pk, &ctl->full[s], kc + 128, n0 / 2);
         tma_load_2d(st + C::OFF_SC, &map_sc, &ctl->full[s], n0, kc >> gsl);
       };
-      auto load_x = [&](int it) {
-        const int s = it % C::ST;
-        const int kc = (st_begin + it) * SK;
-        uint8_t* xs = smem + s * C::STAGE + C::OFF_X;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) tma_load_2d(xs + b * C::XBOX, &map_x, &ctl->full[s], kc + 64 * b, tok0);
-      };
-      // the packed weight is constant: its first stages are requested before
-      // waiting for the kernel that produces x
+      // the packed weight is constant: the ring is filled before (and while)
+      // the consumers wait for the kernel that produces x
       const int pre = nit < C::ST ? nit : C::ST;
       for (int it = 0; it < pre; ++it) {
         mbar_arrive_expect_tx(&ctl->full[it], tx);
         load_weights(it);
       }
-      griddep_wait();
-      for (int it = 0; it < pre; ++it) load_x(it);
       int issued = pre;
       for (int it = pre; it < nit; ++it) {
         const int s = it % C::ST;
         if (!mbar_wait(&ctl->empty[s], ((it / C::ST) - 1) & 1, abort_flag, &g_device_error, 64u)) break;
         mbar_arrive_expect_tx(&ctl->full[s], tx);
         load_weights(it);
-        load_x(it);
         issued = it + 1;
       }
       for (int it = (issued > C::ST ? issued - C::ST : 0); it < issued; ++it)
@@ -180,54 +179,56 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   } else {
     // ------------------------------------------------------------ consumers
     griddep_wait();   // outputs of this kernel may still be read by the previous one
-    const int w = warp;   // 64-column block of every stage
+    const int w = warp & 3;             // 64-column block of every stage
+    const int rt0 = (warp >> 2) * RTW;  // first row tile of this warp
     // per-thread shared-memory offsets inside a stage: 16-byte code chunk t of
     // block w (128-byte swizzle inside the [32 pairs][128 B] box w / 2) for the
     // pair row of each row tile
-    uint32_t code_off[4];
+    uint32_t code_off[RTW];
 #pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
-      const int r = pair_of(rt, g);
+    for (int rt = 0; rt < RTW; ++rt) {
+      const int r = pair_of(rt0 + rt, g);
       code_off[rt] = (w >> 1) * (CODE_BYTES / 2) + r * 128 + 16 * ((4 * (w & 1) + t) ^ (r & 7));
     }
-    // activation fragment: token row min(8 j + g, Mz - 1) of box w, columns
-    // 16 i + 4 t .. + 3 (lanes past the last token repeat it: for one token
-    // every lane of a quad position reads the same 8 bytes)
-    uint32_t x_off[NT][4];
+    // activation fragment of token tile j: token row min(8 j + g, Mz - 1),
+    // columns 16 i + 4 t .. + 3 of the warp's block (lanes past the last token
+    // repeat it, so for one token every lane of a quad position reads the same
+    // 8 bytes); read from global memory one stage ahead of its use
+    const __half* xrow[NT];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int row = min(8 * j + g, Mz - 1);
+    for (int j = 0; j < NT; ++j) xrow[j] = x + (size_t)(tok0 + min(8 * j + g, Mz - 1)) * K + 64 * w + 4 * t;
+    auto load_xf = [&](int it, uint2 (&d)[NT][4]) {
+      const int kb = (st_begin + it) * SK;   // the warp's block starts at kb + 64 w
+      const bool in = kb + 64 * w < K;       // K % 64 == 0: a block is wholly inside or outside
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        x_off[j][i] = C::OFF_X + w * C::XBOX + row * 128 + 16 * ((2 * i + (t >> 1)) ^ (row & 7)) + 8 * (t & 1);
-    }
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[j][i] = in ? ldg_nc_v2(xrow[j] + kb + 16 * i) : make_uint2(0u, 0u);
+    };
     // scale words of block w: row (64 w + 16 SPG q) >> gsl of the stage's box
     // (stages start on multiples of 256 columns), the (even, odd) pair of pair
-    // perm(g) of row tile 0 (+ 16 scales per row tile)
+    // perm(g) of the warp's first row tile (+ 16 scales per row tile)
     uint32_t sc_off[NGB];
 #pragma unroll
     for (int q = 0; q < NGB; ++q) {
       const int col = 64 * w + (SPG == 4 ? 0 : 16 * SPG * q);
-      sc_off[q] = C::OFF_SC + (uint32_t)(gs < SK ? (col >> gsl) : 0) * 64 * C::SB + 2 * C::SB * pair_of(0, g);
+      sc_off[q] = C::OFF_SC + (uint32_t)(gs < SK ? (col >> gsl) : 0) * 64 * C::SB + 2 * C::SB * pair_of(rt0, g);
     }
 
-    float part[4][NT][4];
+    float part[RTW][NT][4];
     bool fresh = true;   // the next MMA starts a new group (zero accumulator)
-    for (int it = 0; it < nit; ++it) {
+    // one stage: wait for its codes and scales, then dequantise and multiply;
+    // false when a wait ran out
+    auto stage = [&](int it, const uint2 (&xv)[NT][4]) -> bool {
       const int s = it % C::ST;
-      if (!mbar_wait(&ctl->full[s], (it / C::ST) & 1, abort_flag, &g_device_error, 128u)) break;
+      if (!mbar_wait(&ctl->full[s], (it / C::ST) & 1, abort_flag, &g_device_error, 128u)) return false;
       const uint32_t st = sbase + s * C::STAGE;
-      uint4 wv[4];
+      uint4 wv[RTW];
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) wv[rt] = lds128(st + code_off[rt]);
-      uint2 xv[NT][4];
+      for (int rt = 0; rt < RTW; ++rt) wv[rt] = lds128(st + code_off[rt]);
+      uint2 sw[RTW][NGB];
 #pragma unroll
-      for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) xv[j][i] = lds64(st + x_off[j][i]);
-      uint2 sw[4][NGB];
-#pragma unroll
-      for (int rt = 0; rt < 4; ++rt)
+      for (int rt = 0; rt < RTW; ++rt)
 #pragma unroll
         for (int q = 0; q < NGB; ++q) {
           const uint32_t a = st + sc_off[q] + 16 * C::SB * rt;
@@ -238,7 +239,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
 
       auto flush = [&](int q) {   // scale the finished group of every row tile into acc
 #pragma unroll
-        for (int rt = 0; rt < 4; ++rt) {
+        for (int rt = 0; rt < RTW; ++rt) {
           const float2 sp = scale_pair<F32S>(sw[rt][q]);
           const float se = sp.x, so = sp.y;
 #pragma unroll
@@ -254,7 +255,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
       for (int i = 0; i < 4; ++i) {
         const bool first = SPG == 4 ? (i == 0 && fresh) : (i % SPG == 0);
 #pragma unroll
-        for (int rt = 0; rt < 4; ++rt) {
+        for (int rt = 0; rt < RTW; ++rt) {
           const uint32_t word = i == 0 ? wv[rt].x : i == 1 ? wv[rt].y : i == 2 ? wv[rt].z : wv[rt].w;
           const RowPairs rp = codes_minus8_rows(word);
           const uint32_t a[4] = {h2_as_u32(rp.ev01), h2_as_u32(rp.od01), h2_as_u32(rp.ev23), h2_as_u32(rp.od23)};
@@ -273,17 +274,29 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         fresh = ((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1;
         if (fresh) flush(0);
       }
+      return true;
+    };
+    // two register sets of activation fragments alternate: the next stage's
+    // are in flight while the current stage is multiplied
+    uint2 xa[NT][4], xb[NT][4];
+    if (nit > 0) load_xf(0, xa);
+    for (int it = 0; it < nit; it += 2) {
+      if (it + 1 < nit) load_xf(it + 1, xb);
+      if (!stage(it, xa) || it + 1 >= nit) break;
+      if (it + 2 < nit) load_xf(it + 2, xa);
+      if (!stage(it + 1, xb)) break;
     }
   }
 
   // warp partials -> [warp][token][row]; the four block slices summed in order
   __syncthreads();
   float* red = reinterpret_cast<float*>(smem);
-  if (warp < kFwdConsumers) {
-    float* rs = red + warp * 16 * 64;
+  if (warp < C::CW) {
+    float* rs = red + (warp & 3) * 16 * 64;
+    const int rt0 = (warp >> 2) * RTW;
 #pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
-      const int r = pair_of(rt, g);
+    for (int rt = 0; rt < RTW; ++rt) {
+      const int r = pair_of(rt0 + rt, g);
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         rs[(8 * j + 2 * t) * 64 + 2 * r] = acc[rt][j][0];
@@ -294,7 +307,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < Mz * 64; e += kFwdThreads)
+  for (int e = threadIdx.x; e < Mz * 64; e += C::THREADS)
     red[e] = ((red[e] + red[16 * 64 + e]) + red[2 * 16 * 64 + e]) + red[3 * 16 * 64 + e];
 
   // Rank rk of the cluster sums tokens [rk Mz / S, (rk + 1) Mz / S) of the S
@@ -305,7 +318,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   if (!(S > 1 ? cluster_any_abort(cluster, &ctl->abort, S) : *abort_flag)) {
     const int rk = S > 1 ? (int)cluster.block_rank() : 0;
     const int tb = rk * Mz / S, te = (rk + 1) * Mz / S;
-    for (int e = threadIdx.x; e < (te - tb) * 64; e += kFwdThreads) {
+    for (int e = threadIdx.x; e < (te - tb) * 64; e += C::THREADS) {
       const int tok = tb + (e >> 6), nl = e & 63;
       const int n = n0 + nl;
       if (n >= N) continue;
@@ -561,9 +574,9 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
 // Host side
 // ---------------------------------------------------------------------------
 template <int NT, int SPG, bool F32S>
-static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUtensorMap& map_sc,
-                                           const CUtensorMap& map_x, OutSplit out, int M, int N, int K, int gs,
-                                           int stages_total, int x_rows, dim3 grid, cudaStream_t stream) {
+static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUtensorMap& map_sc, const __half* x,
+                                           OutSplit out, int M, int N, int K, int gs, int stages_total, dim3 grid,
+                                           cudaStream_t stream) {
   using C = gv::FwdCfg<NT, SPG, F32S>;
   auto kern = gv::q4gsw_gemv_fwd_tma_kernel<NT, SPG, F32S>;
   static PerDeviceOnce attr_once;
@@ -575,7 +588,7 @@ static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUte
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(gv::kFwdThreads, 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -587,7 +600,7 @@ static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUte
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, x_rows);
+  return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, x, out, M, N, K, gs, stages_total);
 }
 
 cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M,
@@ -601,33 +614,26 @@ cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f
   const int tiles = (N + 63) / 64;
   const int stages_total = (K + gv::SK - 1) / gv::SK;
   const int spg = gs == 16 ? 1 : gs == 32 ? 2 : 4;
-  // Contraction splits: fill the resident CTA slots in one wave, at least two
-  // stages per split, clusters of at most 8.
-  const int per_sm = f32s ? (NT == 1 ? (spg == 1 ? gv::FwdCfg<1, 1, true>::CTAS : gv::FwdCfg<1, 4, true>::CTAS)
-                                     : (spg == 1 ? gv::FwdCfg<2, 1, true>::CTAS : gv::FwdCfg<2, 4, true>::CTAS))
-                          : (NT == 1 ? (spg == 1 ? gv::FwdCfg<1, 1, false>::CTAS : gv::FwdCfg<1, 4, false>::CTAS)
-                                     : (spg == 1 ? gv::FwdCfg<2, 1, false>::CTAS : gv::FwdCfg<2, 4, false>::CTAS));
-  const int slots = sm_count(current_device()) * per_sm;
-  int S = slots / (tiles * zs);
+  // Contraction splits: as many CTAs as the SMs hold at once (each CTA's
+  // stages are consumed at a bounded rate, so the stream needs many of them),
+  // at least two stages per split, clusters of at most 8.
+  const int per_sm = NT == 1 ? 4 : 2;
+  int S = sm_count(current_device()) * per_sm / (tiles * zs);
   S = S < 1 ? 1 : (S > 8 ? 8 : S);
   while (S > 1 && stages_total / S < 2) --S;
   const int sc_rows = gs < gv::SK ? gv::SK / gs : 1;
-  const int x_rows = NT == 1 ? (M < 8 ? M : 8) : 16;
-  CUtensorMap map_pk, map_sc, map_x;
+  CUtensorMap map_pk, map_sc;
   const bool ok =
       make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, gv::RP, CU_TENSOR_MAP_SWIZZLE_128B) &&
       make_map_2d(&map_sc, f32s ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                  pk + L.scales_offset, N, G, (uint64_t)N * sb, 64, sc_rows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, (uint64_t)K * 2, 64, x_rows,
-                  CU_TENSOR_MAP_SWIZZLE_128B);
+                  pk + L.scales_offset, N, G, (uint64_t)N * sb, 64, sc_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   const dim3 grid(tiles, S, zs);
   cudaError_t e;
-#define Q4_TMA_FWD(NT_, SPG_)                                                                                         \
-  (f32s ? launch_gemv_tma_variant<NT_, SPG_, true>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, x_rows, grid, \
-                                                   stream)                                                             \
-        : launch_gemv_tma_variant<NT_, SPG_, false>(map_pk, map_sc, map_x, out, M, N, K, gs, stages_total, x_rows,     \
-                                                    grid, stream))
+  const __half* xh = reinterpret_cast<const __half*>(x);
+#define Q4_TMA_FWD(NT_, SPG_)                                                                                    \
+  (f32s ? launch_gemv_tma_variant<NT_, SPG_, true>(map_pk, map_sc, xh, out, M, N, K, gs, stages_total, grid, stream) \
+        : launch_gemv_tma_variant<NT_, SPG_, false>(map_pk, map_sc, xh, out, M, N, K, gs, stages_total, grid, stream))
   if (NT == 1)
     e = spg == 1 ? Q4_TMA_FWD(1, 1) : spg == 2 ? Q4_TMA_FWD(1, 2) : Q4_TMA_FWD(1, 4);
   else
