@@ -77,10 +77,15 @@ def step_ops():
             ("down_bwd", "bwd", down), ("up_bwd", "bwd", up)]
 
 
+ADAPTER_RANK = 16   # rank of the low-rank adapter beside the frozen base in the adapter legs
+
+
 def op_flops(kind, sh, M=None):
     M = sh.M if M is None else M
     if kind == "emb":
         return float(M * sh.K)          # one multiply per gathered element
+    if kind in ("ad_fwd", "ad_bwd"):   # base product plus the two low-rank products
+        return 2.0 * M * sh.N * sh.K + 2.0 * M * ADAPTER_RANK * (sh.N + sh.K)
     return 2.0 * M * sh.N * sh.K
 
 
@@ -92,7 +97,9 @@ def op_bytes(kind, sh, M=None):
         # with its pair), its K/gs fp16 scales, K fp32 outputs; the 4-byte id
         return M * (sh.K + 2 * (sh.K // sh.group_size) + 4 * sh.K + 4)
     w = sh.N * sh.K // 2 + 2 * (sh.K // sh.group_size) * sh.N
-    if kind == "bwd":
+    if kind in ("ad_fwd", "ad_bwd"):   # plus both adapter matrices
+        w += 2 * ADAPTER_RANK * (sh.N + sh.K)
+    if kind in ("bwd", "ad_bwd"):
         return w + 2 * M * sh.N + 4 * M * sh.K
     return w + 2 * M * sh.K + 4 * M * sh.N
 
@@ -563,9 +570,20 @@ def time_shape(q, sh, kind, device, flush, peaks):
     wb = weight_bytes(sh)
     R = max(2, math.ceil(3 * L2_BYTES / wb))
     packs = [first] + [first.clone() for _ in range(R - 1)]
-    src = inp.d_out if kind == "bwd" else inp.x
+    src = inp.d_out if kind in ("bwd", "ad_bwd") else inp.x
     a = torch.from_numpy(src).to(device)
-    if kind == "qkv":
+    if kind in ("ad_fwd", "ad_bwd"):
+        rng = np.random.default_rng(sh.seed + 1)
+        A = torch.from_numpy((rng.standard_normal((ADAPTER_RANK, sh.K)) * 0.05).astype(np.float16)).to(device)
+        B = torch.from_numpy((rng.standard_normal((sh.N, ADAPTER_RANK)) * 0.05).astype(np.float16)).to(device)
+        ws = torch.empty(q.library().q4gsw_adapter_workspace_bytes(sh.M, ADAPTER_RANK), dtype=torch.uint8,
+                         device=device)
+        y = torch.empty((sh.M, sh.N if kind == "ad_fwd" else sh.K), dtype=torch.float32, device=device)
+        if kind == "ad_fwd":
+            fn = lambda pk: q.q4gsw_adapter_fwd(pk, sh.N, sh.K, sh.group_size, A, B, a, y=y, workspace=ws)
+        else:
+            fn = lambda pk: q.q4gsw_adapter_bwd_input(pk, sh.N, sh.K, sh.group_size, A, B, a, d_x=y, workspace=ws)
+    elif kind == "qkv":
         Nq, Nk, Nv = sh.splits
         outs = tuple(torch.empty((sh.M, n), dtype=torch.float32, device=device) for n in (Nq, Nk, Nv))
         fn = lambda pk: q.q4gsw_qkv_fwd(pk, Nq, Nk, Nv, sh.K, sh.group_size, a, outs=outs)
@@ -641,7 +659,9 @@ SHAPE_LEGS = [("decode_N2048_K2048", "fwd"), ("decode_N8192_K2048", "fwd"), ("de
               ("sweep_M16_N14336_K4096", "fwd"), ("sweep_M16_N14336_K4096", "bwd"),
               ("sweep_M16_N4096_K14336", "fwd"), ("sweep_M16_N4096_K14336", "bwd"),
               ("sweep_M4096_N14336_K4096", "fwd"), ("sweep_M4096_N14336_K4096", "bwd"),
-              ("sweep_M4096_N4096_K14336", "fwd"), ("sweep_M4096_N4096_K14336", "bwd")]
+              ("sweep_M4096_N4096_K14336", "fwd"), ("sweep_M4096_N4096_K14336", "bwd"),
+              ("adapter_up_M512", "ad_fwd"), ("adapter_up_M512", "ad_bwd"),
+              ("adapter_down_M512", "ad_fwd"), ("adapter_down_M512", "ad_bwd")]
 
 
 def shape_legs(device, peaks, world):

@@ -43,6 +43,9 @@ SIGNATURES = [
     ("q4gsw_qkv_fwd_f32s", _I, [_VP, _I, _I, _I, _I, _I, _VP, _I, _VP, _VP, _VP, _VP]),
     ("q4gsw_embedding_f32s", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP]),
     ("q4gsw_dequant_f32s", _I, [_VP, _I, _I, _I, _VP, _VP, _VP]),
+    ("q4gsw_adapter_workspace_bytes", _SZ, [_I, _I]),
+    ("q4gsw_adapter_fwd", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP, _SZ, _VP]),
+    ("q4gsw_adapter_bwd_input", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP, _SZ, _VP]),
     ("q4gsw_debug_pin_routes", _I, [_I, _I]),
     ("q4gsw_debug_wait_timeout", _I, [ctypes.c_uint, _VP]),
     ("q4gsw_last_route", ctypes.c_char_p, []),
@@ -212,6 +215,33 @@ def q4gsw_device_error_check(device=None) -> None:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     st = library().q4gsw_device_error_check(torch.cuda.current_stream(dev).cuda_stream)
     _check("q4gsw_device_error_check", st)
+
+
+def _adapter(name, packed, N, K, group_size, a, b, act, out, workspace, out_cols):
+    lib = library()
+    r = a.shape[0]
+    M = act.shape[0]
+    if out is None:
+        out = torch.empty((M, out_cols), dtype=torch.float32, device=act.device)
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.q4gsw_adapter_workspace_bytes(M, r)), 16), dtype=torch.uint8,
+                                device=act.device)
+    st = getattr(lib, name)(_dev(packed, torch.uint8, "packed"), N, K, group_size, _dev(a, torch.float16, "a", 2),
+                            _dev(b, torch.float16, "b", 2), r, _dev(act, torch.float16, "act", 2), M,
+                            _dev(out, torch.float32, "out", 2), _dev(workspace, torch.uint8, "workspace"),
+                            workspace.numel(), _stream(act))
+    _check(name, st)
+    return out
+
+
+def q4gsw_adapter_fwd(packed, N: int, K: int, group_size: int, a, b, x, y=None, workspace=None):
+    """y = x dequant(W)^T + (x a^T) b^T with a fp16 [r, K], b fp16 [N, r] (frozen-base adapter)."""
+    return _adapter("q4gsw_adapter_fwd", packed, N, K, group_size, a, b, x, y, workspace, N)
+
+
+def q4gsw_adapter_bwd_input(packed, N: int, K: int, group_size: int, a, b, d_out, d_x=None, workspace=None):
+    """d_x = d_out dequant(W) + (d_out b) a (input gradient of the adapter forward)."""
+    return _adapter("q4gsw_adapter_bwd_input", packed, N, K, group_size, a, b, d_out, d_x, workspace, K)
 
 
 GEMV_ROUTES = {"auto": 0, "reg": 1, "tma": 2}

@@ -1,0 +1,120 @@
+// q4gsw_adapter.cu - the low-rank intermediate of the frozen-base adapter step.
+//
+// The q4gsw input gradient exists for on-device adapter training on a frozen
+// 4-bit base ("[ExecuTorch][Vulkan] Add et_vk.linear_q4gsw_backward kernel
+// (4-bit input-grad)", PR description).  With a rank-r adapter beside the base,
+//   forward    y   = x dequant(W)^T + (x A^T) B^T      A fp16 [r, K], B fp16 [N, r]
+//   backward   d_x = d_out dequant(W) + (d_out B) A
+// this file computes the intermediate u = x A^T (forward) or v = d_out B
+// (backward), [M][r] with fp32 accumulation, rounded to fp16 and stored as
+// rows of 64 halves (columns r..63 zero) in the caller's workspace.  The GEMM
+// then adds u B^T (or v A) as one more 64-deep contraction stage of its
+// accumulator.
+//
+// One CTA per 16 tokens; eight warps split the contraction, each running
+// mma.sync m16n8k16 (A = 16 tokens x 16 contraction indices of the activation,
+// B = 16 contraction indices x 8 rank columns of the projection), and the
+// eight partial tiles are summed in shared memory in a fixed order.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "q4gsw_common.cuh"
+#include "q4gsw_internal.h"
+
+namespace q4gsw {
+namespace ad {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kRankMax = 64;
+
+// act [M][C] fp16 row-major; the projection P(c, j) is proj[j * C + c] when
+// BY_ROWS (forward: A [r, C]) or proj[c * r + j] (backward: B [C, r]).
+template <bool BY_ROWS>
+__global__ void __launch_bounds__(kThreads)
+q4gsw_adapter_proj_kernel(const __half* __restrict__ act, const __half* __restrict__ proj, __half* __restrict__ out,
+                          int M, int C, int r) {
+  __shared__ float red[kWarps][16][kRankMax];
+  griddep_launch_dependents();
+  griddep_wait();   // the activations may come from the previous kernel of the stream
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int m0 = blockIdx.x * 16;
+  const int steps = (C + 15) / 16;   // C % 8 == 0: the last step may hold only 8 columns
+  const int s_begin = warp * steps / kWarps, s_end = (warp + 1) * steps / kWarps;
+  const int nj = (r + 7) / 8;  // 8-column rank tiles
+  // rows past M read row M - 1 (never stored)
+  const __half* a0 = act + (size_t)min(m0 + g, M - 1) * C;
+  const __half* a1 = act + (size_t)min(m0 + g + 8, M - 1) * C;
+  float acc[8][4];
+#pragma unroll
+  for (int jt = 0; jt < 8; ++jt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[jt][c] = 0.f;
+  auto pval = [&](int c, int j) -> uint32_t {   // P(c, j) as fp16 bits, zero past the rank
+    if (j >= r) return 0u;
+    const __half v = BY_ROWS ? proj[(size_t)j * C + c] : proj[(size_t)c * r + j];
+    return __half_as_ushort(v);
+  };
+#pragma unroll 2
+  for (int st = s_begin; st < s_end; ++st) {
+    const int c0 = 16 * st;
+    const bool hi_ok = c0 + 8 < C;   // columns c0 + 8 .. c0 + 15 exist
+    const uint32_t af[4] = {ldg_nc_u32(a0 + c0 + 2 * t), ldg_nc_u32(a1 + c0 + 2 * t),
+                            hi_ok ? ldg_nc_u32(a0 + c0 + 2 * t + 8) : 0u, hi_ok ? ldg_nc_u32(a1 + c0 + 2 * t + 8) : 0u};
+#pragma unroll
+    for (int jt = 0; jt < 8; ++jt) {
+      if (jt >= nj) break;
+      const int j = 8 * jt + g;
+      uint32_t bf[2];
+      if (BY_ROWS) {
+        // A[j][c], A[j][c + 1] are adjacent
+        bf[0] = j < r ? ldg_nc_u32(proj + (size_t)j * C + c0 + 2 * t) : 0u;
+        bf[1] = (j < r && hi_ok) ? ldg_nc_u32(proj + (size_t)j * C + c0 + 2 * t + 8) : 0u;
+      } else {
+        bf[0] = pval(c0 + 2 * t, j) | (pval(c0 + 2 * t + 1, j) << 16);
+        bf[1] = hi_ok ? pval(c0 + 2 * t + 8, j) | (pval(c0 + 2 * t + 9, j) << 16) : 0u;
+      }
+      mma_16816(acc[jt], af, bf);
+    }
+  }
+  // D fragment: rows g, g + 8 (tokens), columns 2t, 2t + 1 of rank tile jt
+#pragma unroll
+  for (int jt = 0; jt < 8; ++jt) {
+    red[warp][g][8 * jt + 2 * t] = acc[jt][0];
+    red[warp][g][8 * jt + 2 * t + 1] = acc[jt][1];
+    red[warp][g + 8][8 * jt + 2 * t] = acc[jt][2];
+    red[warp][g + 8][8 * jt + 2 * t + 1] = acc[jt][3];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 16 * kRankMax; e += kThreads) {
+    const int row = e / kRankMax, j = e % kRankMax;
+    if (m0 + row >= M) continue;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += red[w][row][j];
+    out[(size_t)(m0 + row) * kRankMax + j] = j < r ? __float2half_rn(s) : __float2half_rn(0.f);
+  }
+}
+
+}  // namespace ad
+
+cudaError_t launch_adapter_proj(const uint16_t* act, const uint16_t* proj, bool by_rows, int M, int C, int r,
+                                void* workspace, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((M + 15) / 16, 1, 1);
+  cfg.blockDim = dim3(ad::kThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const __half* a = reinterpret_cast<const __half*>(act);
+  const __half* p = reinterpret_cast<const __half*>(proj);
+  __half* o = static_cast<__half*>(workspace);
+  return by_rows ? cudaLaunchKernelEx(&cfg, ad::q4gsw_adapter_proj_kernel<true>, a, p, o, M, C, r)
+                 : cudaLaunchKernelEx(&cfg, ad::q4gsw_adapter_proj_kernel<false>, a, p, o, M, C, r);
+}
+
+}  // namespace q4gsw

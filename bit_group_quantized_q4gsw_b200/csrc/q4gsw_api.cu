@@ -175,6 +175,32 @@ q4gsw_status dequant_impl(const void* packed, int N, int K, int group_size, bool
   return from_cuda(launch_dequant(packed, N, K, group_size, f32s, w32, w16, stream));
 }
 
+q4gsw_status adapter_impl(bool bwd, const void* packed, int N, int K, int group_size, const uint16_t* a,
+                          const uint16_t* b, int r, const uint16_t* act, int M, float* out, void* workspace,
+                          size_t workspace_bytes, q4gsw_stream_t stream) {
+  if (M < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (r < 8 || r > 64 || r % 8) return Q4GSW_ERR_SHAPE;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed || !a || !b || !act || !out || !workspace) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(a) || !aligned16(b) || !aligned16(act) || !aligned16(out) ||
+      !aligned16(workspace))
+    return Q4GSW_ERR_ALIGN;
+  if (workspace_bytes < (size_t)M * 128) return Q4GSW_ERR_SIZE;
+  // the intermediate: forward x A^T (A [r, K] by rows), backward d_out B (B [N, r])
+  cudaError_t e = bwd ? launch_adapter_proj(act, b, false, M, N, r, workspace, stream)
+                      : launch_adapter_proj(act, a, true, M, K, r, workspace, stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  char route[160];
+  const AdapterRef ad{bwd ? a : b, r, workspace};
+  e = launch_gemm_adapter(bwd, packed, N, K, group_size, act, M, out, ad, stream, route, sizeof(route));
+  char full[200];
+  snprintf(full, sizeof(full), "adapter_%s launches=2 proj + %s", bwd ? "bwd" : "fwd", route);
+  set_route(full);
+  return from_cuda(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -267,6 +293,23 @@ q4gsw_status q4gsw_embedding(const void* packed, int N, int K, int group_size, c
 q4gsw_status q4gsw_embedding_f32s(const void* packed, int N, int K, int group_size, const int32_t* indices, int T,
                                   float* out, q4gsw_stream_t stream) {
   return embedding_impl(packed, N, K, group_size, true, indices, T, out, stream);
+}
+
+size_t q4gsw_adapter_workspace_bytes(int M, int r) {
+  if (M < 0 || r < 8 || r > 64 || r % 8) return 0;
+  return (size_t)M * 128;
+}
+
+q4gsw_status q4gsw_adapter_fwd(const void* packed, int N, int K, int group_size, const uint16_t* a,
+                               const uint16_t* b, int r, const uint16_t* x, int M, float* y, void* workspace,
+                               size_t workspace_bytes, q4gsw_stream_t stream) {
+  return adapter_impl(false, packed, N, K, group_size, a, b, r, x, M, y, workspace, workspace_bytes, stream);
+}
+
+q4gsw_status q4gsw_adapter_bwd_input(const void* packed, int N, int K, int group_size, const uint16_t* a,
+                                     const uint16_t* b, int r, const uint16_t* d_out, int M, float* d_x,
+                                     void* workspace, size_t workspace_bytes, q4gsw_stream_t stream) {
+  return adapter_impl(true, packed, N, K, group_size, a, b, r, d_out, M, d_x, workspace, workspace_bytes, stream);
 }
 
 q4gsw_status q4gsw_debug_pin_routes(int gemv, int gemm) {

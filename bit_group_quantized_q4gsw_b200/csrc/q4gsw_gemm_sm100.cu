@@ -639,6 +639,16 @@ cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, bool f32s,
               : launch_gemm_ts_impl<false, false>(packed, N, K, gs, x, M, out, stream, route, route_len);
 }
 
+cudaError_t launch_gemm_adapter(bool bwd, const void* packed, int N, int K, int gs, const uint16_t* act, int M,
+                                float* out, const AdapterRef& ad, cudaStream_t stream, char* route, int route_len) {
+  // the adapter stage exists in the tensor-memory route, which takes any M
+  if (bwd)
+    return launch_gemm_ts_impl<true, false>(packed, N, K, gs, act, M, single_output(out, K), stream, route, route_len,
+                                            &ad);
+  return launch_gemm_ts_impl<false, false>(packed, N, K, gs, act, M, single_output(out, N), stream, route, route_len,
+                                           &ad);
+}
+
 cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M,
                             float* d_x, cudaStream_t stream, char* route, int route_len) {
   const OutSplit o = single_output(d_x, K);

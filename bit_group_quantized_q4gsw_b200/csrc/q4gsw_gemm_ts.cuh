@@ -71,6 +71,13 @@ struct Args {
   int sc_bytes;       // bytes of the scale box of one stage
   int bt;             // tokens per tile
   int tma_out;        // outputs written by tensor store / reduce-add (map_y*), else by threads
+  // Low-rank adapter stage (ad_r > 0): one more 64-deep stage of the last
+  // split whose weight operand is the adapter matrix (forward: rows of B
+  // [N, r]; backward: columns of A [r, K]; leading dimension ad_ld) and whose
+  // activation operand is the fp16 intermediate [M][64] (map_ad).
+  const __half* ad_mat;
+  int ad_r;
+  int ad_ld;
 };
 
 struct Ctl {
@@ -113,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_constant__ CUtensorMap map_pk,
                      const __grid_constant__ CUtensorMap map_sc, const __grid_constant__ CUtensorMap map_y0,
                      const __grid_constant__ CUtensorMap map_y1, const __grid_constant__ CUtensorMap map_y2,
-                     const Args args) {
+                     const __grid_constant__ CUtensorMap map_ad, const Args args) {
   using namespace sm100;
   using SM = Smem<ST, F32S ? 2048 : 1024>;
   constexpr int SC_BYTES = SM::SC_BYTES;
@@ -130,7 +137,8 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
   const int S = gridDim.z, split = blockIdx.z;
   const int st_begin = (int)((long long)split * args.stages_total / S);
   const int st_end = (int)((long long)(split + 1) * args.stages_total / S);
-  const int nit = st_end - st_begin;
+  const int nit = st_end - st_begin;          // stages of the packed weight
+  const int nitx = nit + ((args.ad_r > 0 && split == S - 1) ? 1 : 0);   // plus the adapter stage
   const int gsl = __ffs(args.gs) - 1;
 
   griddep_launch_dependents();
@@ -176,24 +184,28 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       };
       auto load_act = [&](int it) {
         const int s = it % ST;
-        tma_load_2d(smem + SM::OFF_X + s * X_BYTES, &map_act, &ctl->full[s], (st_begin + it) * TK, t0);
+        if (it < nit)
+          tma_load_2d(smem + SM::OFF_X + s * X_BYTES, &map_act, &ctl->full[s], (st_begin + it) * TK, t0);
+        else   // the adapter stage: the low-rank intermediate of the tile's tokens
+          tma_load_2d(smem + SM::OFF_X + s * X_BYTES, &map_ad, &ctl->full[s], 0, t0);
       };
+      const uint32_t tx_ad = (uint32_t)args.bt * TK * 2;
       // The packed weight is constant: the first stages' codes and scales are
       // requested before waiting for the previous kernel of the stream, which
       // may still be producing the activations.
-      const int pre = nit < ST ? nit : ST;
+      const int pre = nitx < ST ? nitx : ST;
       for (int it = 0; it < pre; ++it) {
-        mbar_arrive_expect_tx(&ctl->full[it], tx);
-        load_weights(it);
+        mbar_arrive_expect_tx(&ctl->full[it], it < nit ? tx : tx_ad);
+        if (it < nit) load_weights(it);
       }
       griddep_wait();
       for (int it = 0; it < pre; ++it) load_act(it);
       int issued = pre;
-      for (int it = pre; it < nit; ++it) {
+      for (int it = pre; it < nitx; ++it) {
         const int s = it % ST;
         if (!mbar_wait(&ctl->consumed[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 1u)) break;
-        mbar_arrive_expect_tx(&ctl->full[s], tx);
-        load_weights(it);
+        mbar_arrive_expect_tx(&ctl->full[s], it < nit ? tx : tx_ad);
+        if (it < nit) load_weights(it);
         load_act(it);
         issued = it + 1;
       }
@@ -212,7 +224,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(BW, args.bt, false);
       bool next_ready = false;
-      for (int it = 0; it < nit; ++it) {
+      for (int it = 0; it < nitx; ++it) {
         const int s = it % ST, w = it % WST;
         if (!next_ready && !mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
         tc_fence_after();
@@ -220,7 +232,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
 #pragma unroll
         for (int ks = 0; ks < TK / 16; ++ks) {
           if (ks == TK / 16 - 1)
-            next_ready = it + 1 < nit && mbar_test_wait(&ctl->wready[(it + 1) % WST], ((it + 1) / WST) & 1);
+            next_ready = it + 1 < nitx && mbar_test_wait(&ctl->wready[(it + 1) % WST], ((it + 1) / WST) & 1);
           const uint64_t bd = smem_desc_sw128(x0 + 32 * ks, 16, 1024);
           mma_f16_ts(tmem, tmem + ACC_COLS + w * A_COLS + 8 * ks, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
         }
@@ -261,7 +273,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       for (int j = 0; j < 8; ++j) off[j] = (8 * kq + j) * 128 + boff;
       sc_off = (uint32_t)((((f0 & (args.gs - 1)) + r) >> gsl) * TK * SB + 2 * SB * 8 * kq);
     }
-    for (int it = 0; it < nit; ++it) {
+    for (int it = 0; it < nitx; ++it) {
       const int s = it % ST, w = it % WST;
       if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
       // TMEM slot w is free once the MMAs of stage it - WST completed
@@ -272,7 +284,24 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       const uint32_t pk = sbase + SM::OFF_P + s * P_BYTES;
       const uint32_t sc = sbase + SM::OFF_SC + s * SC_BYTES;
       uint32_t v[8];
-      if (!BWD) {
+      if (it >= nit) {
+        // The adapter stage: rank columns j = 16 kq .. 16 kq + 15 of this
+        // thread's output feature, straight from the fp16 adapter matrix
+        // (forward B[f][j], backward A[j][f]; zero past the rank or the extent).
+        const int f = f0 + r;
+        const bool fin = f < args.rows_out;
+        const unsigned short* am = reinterpret_cast<const unsigned short*>(args.ad_mat);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int j = 16 * kq + 2 * m;
+          uint32_t lo = 0u, hi = 0u;
+          if (fin && j < args.ad_r)
+            lo = BWD ? __ldg(am + (size_t)j * args.ad_ld + f) : __ldg(am + (size_t)f * args.ad_ld + j);
+          if (fin && j + 1 < args.ad_r)
+            hi = BWD ? __ldg(am + (size_t)(j + 1) * args.ad_ld + f) : __ldg(am + (size_t)f * args.ad_ld + j + 1);
+          v[m] = lo | (hi << 16);
+        }
+      } else if (!BWD) {
         uint32_t wd[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) wd[t] = lds32(pk + off[t]);
@@ -440,7 +469,8 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
 // ---------------------------------------------------------------------------
 template <bool BWD, bool F32S>
 static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs, const uint16_t* act, int M,
-                                       OutSplit out, cudaStream_t stream, char* route, int route_len) {
+                                       OutSplit out, cudaStream_t stream, char* route, int route_len,
+                                       const AdapterRef* ad = nullptr) {
   using namespace ts;
   constexpr int ST = F32S ? 5 : 6;
   constexpr int SB = F32S ? 4 : 2;
@@ -505,6 +535,19 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
     if (!tma_out) map_y[0] = map_y[1] = map_y[2] = map_act;   // never read
   }
 
+  // adapter stage: the intermediate [M][64] fp16 as the activation operand
+  CUtensorMap map_ad = map_act;   // never read without an adapter
+  a.ad_mat = nullptr;
+  a.ad_r = 0;
+  a.ad_ld = 0;
+  if (ad) {
+    if (!make_map_2d(&map_ad, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ad->inter, 64, M, 128, TK, a.bt,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    a.ad_mat = reinterpret_cast<const __half*>(ad->mat);
+    a.ad_r = ad->r;
+    a.ad_ld = BWD ? K : ad->r;
+  }
   auto kern = q4gsw_gemm_ts_kernel<BWD, ST, F32S>;
   constexpr int smem = Smem<ST, SC_BYTES>::BYTES;
   static PerDeviceOnce attr_once;
@@ -556,9 +599,10 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
   attr[0].val.clusterDim.z = best_S;
   cfg.gridDim = dim3(tiles_f, tiles_t, best_S);
   if (route)
-    snprintf(route, route_len, "tcgen05_ts_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d out=%s",
-             BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, WST, tiles_f, tiles_t, best_S, a.tma_out ? "tma" : "st");
-  return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, map_y[0], map_y[1], map_y[2], a);
+    snprintf(route, route_len, "tcgen05_ts_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d out=%s%s",
+             BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, WST, tiles_f, tiles_t, best_S, a.tma_out ? "tma" : "st",
+             ad ? " adapter_stage=1" : "");
+  return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, map_y[0], map_y[1], map_y[2], map_ad, a);
 }
 
 }  // namespace q4gsw

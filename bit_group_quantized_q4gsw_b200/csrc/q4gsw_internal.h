@@ -79,6 +79,23 @@ cudaError_t launch_gemm_fwd(const void* packed, int N, int K, int gs, bool f32s,
 cudaError_t launch_gemm_bwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* d_out, int M, float* d_x,
                             cudaStream_t stream, char* route, int route_len);
 
+// Frozen-base low-rank adapter: the fp16 adapter matrix (forward B [N, r],
+// backward A [r, K]), its rank (8 <= r <= 64, r % 8 == 0) and the fp16
+// intermediate [M][64] (forward x A^T, backward d_out B; columns r..63 zero).
+struct AdapterRef {
+  const uint16_t* mat;
+  int r;
+  const void* inter;
+};
+// The intermediate: act [M][C] times the projection (by_rows: A [r, C], used
+// as A^T; else B [C, r]) into `workspace` as [M][64] fp16.
+cudaError_t launch_adapter_proj(const uint16_t* act, const uint16_t* proj, bool by_rows, int M, int C, int r,
+                                void* workspace, cudaStream_t stream);
+// The tensor-memory GEMM (forward when !bwd) with the adapter stage added to
+// the accumulator of the last contraction split.
+cudaError_t launch_gemm_adapter(bool bwd, const void* packed, int N, int K, int gs, const uint16_t* act, int M,
+                                float* out, const AdapterRef& ad, cudaStream_t stream, char* route, int route_len);
+
 // Embedding rows out[t] = dequant(W)[indices[t]] (fp32); an index outside
 // [0, N) gives a zero row and sets kIndexErrorBit in the device error word.
 cudaError_t launch_embedding(const void* packed, int N, int K, int gs, bool f32s, const int32_t* indices, int T, float* out,

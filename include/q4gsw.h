@@ -228,6 +228,48 @@ Q4GSW_API q4gsw_status q4gsw_embedding_f32s(const void *packed, int N, int K, in
 Q4GSW_API q4gsw_status q4gsw_dequant_f32s(const void *packed, int N, int K, int group_size,
                                 float *w32, uint16_t *w16, q4gsw_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Frozen-base low-rank adapter step
+ *
+ * "[ExecuTorch][Vulkan] Add et_vk.linear_q4gsw_backward kernel (4-bit
+ * input-grad)", PR description: the input gradient of the frozen 4-bit base
+ * exists for on-device adapter training.  The page does not define the
+ * adapter; this library's reading is a rank-r low-rank adapter beside the
+ * frozen q4gsw base, with no scaling factor (fold one into B):
+ *   forward         y   = x dequant(W)^T + (x A^T) B^T
+ *   input gradient  d_x = d_out dequant(W) + (d_out B) A    (its adjoint)
+ *   a  fp16 [r, K] row-major,  b  fp16 [N, r] row-major,  8 <= r <= 64, r % 8 == 0
+ * Two launches on `stream`: the intermediate u = x A^T (or v = d_out B) is
+ * accumulated in fp32, rounded to fp16 and written to `workspace` as rows of
+ * 64 halves; then the tensor-memory GEMM of the base adds u B^T (or v A) to
+ * its fp32 accumulator as one more 64-deep contraction stage, so the output
+ * is written once.  Every token count takes the tensor-memory GEMM route.
+ * Error bound per output element: 4e-3 * (sum |x||w| + sum_j (sum_k |x||A_jk|) |B_nj|)
+ * (the second term covers the fp16 rounding of the intermediate, which must
+ * stay within the fp16 range).
+ *   workspace  device, at least q4gsw_adapter_workspace_bytes(M, r) bytes,
+ *              owned by the caller, overwritten; calls that share one
+ *              workspace must be ordered on the GPU.
+ * Only layout-version-1 blobs (fp16 scales).  Same checks and statuses as
+ * q4gsw_linear_fwd, plus Q4GSW_ERR_SHAPE for a rank outside the rule and
+ * Q4GSW_ERR_SIZE for a workspace that is too small.
+ * ---------------------------------------------------------------------- */
+
+/* Workspace bytes of one adapter call (M * 128); 0 for a rank outside the rule. */
+Q4GSW_API size_t q4gsw_adapter_workspace_bytes(int M, int r);
+
+Q4GSW_API q4gsw_status q4gsw_adapter_fwd(const void *packed, int N, int K, int group_size,
+                               const uint16_t *a, const uint16_t *b, int r,
+                               const uint16_t *x, int M, float *y,
+                               void *workspace, size_t workspace_bytes,
+                               q4gsw_stream_t stream);
+
+Q4GSW_API q4gsw_status q4gsw_adapter_bwd_input(const void *packed, int N, int K, int group_size,
+                                     const uint16_t *a, const uint16_t *b, int r,
+                                     const uint16_t *d_out, int M, float *d_x,
+                                     void *workspace, size_t workspace_bytes,
+                                     q4gsw_stream_t stream);
+
 /*
  * Kernel health check.  Every wait inside this library's kernels is bounded
  * (one second of wall-clock time); a wait that runs out makes its kernel stop

@@ -21,7 +21,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = b.library()
     names = declared_functions()
-    assert len(names) == 21
+    assert len(names) == 24
     assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
     for n in names:
         assert hasattr(lib, n), n
@@ -159,3 +159,20 @@ def test_f32s_entry_points_check_arguments_on_the_host():
     assert lib.q4gsw_embedding_f32s(fake, 64, 128, 32, fake, -1, fake, None) == 2
     assert lib.q4gsw_dequant_f32s(fake, 64, 128, 32, None, None, None) == 1
     assert lib.q4gsw_linear_fwd_f32s(None, 64, 128, 32, None, 0, None, None) == 0
+
+
+def test_adapter_entry_points_check_arguments_on_the_host():
+    lib = b.library()
+    fake = 0x100000
+    assert lib.q4gsw_adapter_workspace_bytes(512, 16) == 512 * 128
+    assert lib.q4gsw_adapter_workspace_bytes(512, 12) == 0
+    assert lib.q4gsw_adapter_workspace_bytes(512, 72) == 0
+    f = lib.q4gsw_adapter_fwd
+    assert f(fake, 64, 128, 32, fake, fake, 12, fake, 4, fake, fake, 4 * 128, None) == 2    # rank rule
+    assert f(fake, 64, 128, 32, fake, fake, 16, fake, 4, fake, fake, 4 * 128 - 1, None) == 7   # workspace
+    assert f(fake, 64, 128, 32, None, fake, 16, fake, 4, fake, fake, 4 * 128, None) == 1
+    assert f(fake, 64, 128, 32, fake, fake, 16, fake, 4, fake, fake + 8, 4 * 128, None) == 3
+    assert f(None, 64, 128, 32, None, None, 16, None, 0, None, None, 0, None) == 0            # empty batch
+    g = lib.q4gsw_adapter_bwd_input
+    assert g(fake, 62, 128, 32, fake, fake, 16, fake, 4, fake, fake, 4 * 128, None) == 2
+    assert g(fake, 64, 128, 32, fake, fake, 16, fake, -1, fake, fake, 4 * 128, None) == 2
