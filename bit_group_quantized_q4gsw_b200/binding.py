@@ -46,6 +46,7 @@ SIGNATURES = [
     ("q4gsw_adapter_workspace_bytes", _SZ, [_I, _I]),
     ("q4gsw_adapter_fwd", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP, _SZ, _VP]),
     ("q4gsw_adapter_bwd_input", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP, _SZ, _VP]),
+    ("q4gsw_adapter_fwd_noalloc", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP]),
     ("q4gsw_debug_pin_routes", _I, [_I, _I]),
     ("q4gsw_debug_wait_timeout", _I, [ctypes.c_uint, _VP]),
     ("q4gsw_last_route", ctypes.c_char_p, []),

@@ -99,6 +99,28 @@ q4gsw_adapter_proj_kernel(const __half* __restrict__ act, const __half* __restri
 
 }  // namespace ad
 
+// Scratch of the allocation-free adapter entry point (q4gsw_adapter_fwd_noalloc):
+// the intermediate [M][64] fp16 of one call, M <= kNoAllocScratchBytes / 128.
+// It is a fixed array in the library's device image, so every GPU that loads
+// the library holds it until the process exits, and every call shares it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
+  // In host code the array's name is only a stand-in for the symbol, never a
+  // device address: its address on the current device is looked up once per
+  // device (with that device current) and reused.
+  static std::once_flag once[kMaxDevices];
+  static void* addr[kMaxDevices];
+  static cudaError_t err[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] { err[dev] = cudaGetSymbolAddress(&addr[dev], g_noalloc_scratch); });
+  if (err[dev] != cudaSuccess) return err[dev];
+  *ptr = addr[dev];
+  *bytes = kNoAllocScratchBytes;
+  return cudaSuccess;
+}
+
 cudaError_t launch_adapter_proj(const uint16_t* act, const uint16_t* proj, bool by_rows, int M, int C, int r,
                                 void* workspace, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};

@@ -312,6 +312,19 @@ q4gsw_status q4gsw_adapter_bwd_input(const void* packed, int N, int K, int group
   return adapter_impl(true, packed, N, K, group_size, a, b, r, d_out, M, d_x, workspace, workspace_bytes, stream);
 }
 
+q4gsw_status q4gsw_adapter_fwd_noalloc(const void* packed, int N, int K, int group_size, const uint16_t* a,
+                                       const uint16_t* b, int r, const uint16_t* x, int M, float* y,
+                                       q4gsw_stream_t stream) {
+  if (M < 0) return Q4GSW_ERR_SHAPE;
+  if ((size_t)M * 128 > kNoAllocScratchBytes) return Q4GSW_ERR_SIZE;
+  void* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  if (noalloc_scratch(&scratch, &scratch_bytes) != cudaSuccess) return Q4GSW_ERR_CUDA;
+  // the projection kernel writes every byte of the rows the GEMM reads, so
+  // nothing left in the array by an earlier call needs clearing
+  return adapter_impl(false, packed, N, K, group_size, a, b, r, x, M, y, scratch, scratch_bytes, stream);
+}
+
 q4gsw_status q4gsw_debug_pin_routes(int gemv, int gemm) {
   if (gemv < kGemvAuto || gemv > kGemvTma || gemm < kGemmAuto || gemm > kGemmSs2) return Q4GSW_ERR_SHAPE;
   route_pins().gemv = gemv;

@@ -91,6 +91,11 @@ struct AdapterRef {
 // as A^T; else B [C, r]) into `workspace` as [M][64] fp16.
 cudaError_t launch_adapter_proj(const uint16_t* act, const uint16_t* proj, bool by_rows, int M, int C, int r,
                                 void* workspace, cudaStream_t stream);
+// Device address (on the current device) and size of the library's own fixed
+// scratch array for the allocation-free adapter entry point.  The first call
+// on a device looks the address up (cudaGetSymbolAddress).
+constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes);
 // The tensor-memory GEMM (forward when !bwd) with the adapter stage added to
 // the accumulator of the last contraction split.
 cudaError_t launch_gemm_adapter(bool bwd, const void* packed, int N, int K, int gs, const uint16_t* act, int M,

@@ -271,6 +271,38 @@ Q4GSW_API q4gsw_status q4gsw_adapter_bwd_input(const void *packed, int N, int K,
                                      q4gsw_stream_t stream);
 
 /*
+ * q4gsw_adapter_fwd without a workspace argument: the same result, with the
+ * intermediate kept in a fixed scratch array inside this library instead of
+ * memory the caller allocates.  (The web pages describe no such call; it is
+ * this library's own addition.)
+ *
+ * For callers that cannot allocate device memory when they make the call:
+ * code on a latency-critical path where cudaMalloc (which may synchronise the
+ * whole device) is not acceptable, plugins hosted by a runtime that owns all
+ * device memory and forbids allocations of their own, or programs whose device
+ * memory is fixed up front.  The call itself allocates nothing: no cudaMalloc,
+ * cudaFree or allocating library routine.  The caller still passes the inputs
+ * and the output y.
+ *
+ * Limit: M <= 8192 tokens (the array holds 1 MiB = 8192 rows of 64 halves);
+ * a larger M returns Q4GSW_ERR_SIZE before anything is enqueued.  Every GPU
+ * that loads the library holds that 1 MiB until the process exits.
+ * Set-up: the first call on a device looks up the array's address on that
+ * device (cudaGetSymbolAddress), once; make that first call before any stream
+ * capture.  A failed look-up returns Q4GSW_ERR_CUDA.
+ * Sharing: all calls on a device use the same array, and it keeps the last
+ * call's contents (nothing read by a call depends on them: each call writes
+ * every byte it reads).  Calls whose work overlaps on the GPU (different
+ * streams, or threads without ordering) race on the array and give wrong
+ * results; order them on one stream or with events.
+ * Other arguments, checks and statuses as q4gsw_adapter_fwd.
+ */
+Q4GSW_API q4gsw_status q4gsw_adapter_fwd_noalloc(const void *packed, int N, int K, int group_size,
+                                       const uint16_t *a, const uint16_t *b, int r,
+                                       const uint16_t *x, int M, float *y,
+                                       q4gsw_stream_t stream);
+
+/*
  * Kernel health check.  Every wait inside this library's kernels is bounded
  * (one second of wall-clock time); a wait that runs out makes its kernel stop
  * early, leaving its outputs partly or wholly unwritten, and record the event

@@ -21,7 +21,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = b.library()
     names = declared_functions()
-    assert len(names) == 24
+    assert len(names) == 25
     assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
     for n in names:
         assert hasattr(lib, n), n
@@ -176,3 +176,11 @@ def test_adapter_entry_points_check_arguments_on_the_host():
     g = lib.q4gsw_adapter_bwd_input
     assert g(fake, 62, 128, 32, fake, fake, 16, fake, 4, fake, fake, 4 * 128, None) == 2
     assert g(fake, 64, 128, 32, fake, fake, 16, fake, -1, fake, fake, 4 * 128, None) == 2
+
+
+def test_noalloc_adapter_rejects_sizes_beyond_its_array_on_the_host():
+    lib = b.library()
+    fake = 0x100000
+    # 8193 tokens need more than the 1 MiB array: rejected before any set-up or launch
+    assert lib.q4gsw_adapter_fwd_noalloc(fake, 64, 128, 32, fake, fake, 16, fake, 8193, fake, None) == 7
+    assert lib.q4gsw_adapter_fwd_noalloc(fake, 64, 128, 32, fake, fake, 16, fake, -1, fake, None) == 2
