@@ -1,4 +1,4 @@
-"""Plain CPU oracle for the two variants of the q4gsw layer beside the fp16-scale path.
+"""Plain CPU oracle for the variants of the q4gsw layer beside the fp16-scale path.
 
 TEST INFRASTRUCTURE ONLY, under the same rule as ``q4gsw_oracle``: only
 ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU legs may import
@@ -24,6 +24,9 @@ it; it shares no code with the CUDA library.
        y   = x dequant(W)^T + (x A^T) B^T          A fp16 [r, K], B fp16 [N, r]
        d_x = d_out dequant(W) + (d_out B) A        (the adjoint of the forward)
    with no scaling factor (a caller folds one into B).
+3. linear_dq8ca_q4gsw (the same fork's shader list): 8-bit dynamically
+   quantised activations times the q4gsw weight; the reading is stated above
+   ``dq8ca_quantize``.
 
 Each function returns the exact value (fp64 sums of exact terms) and the
 per-element bound of the absolute products, as ``q4gsw_oracle`` does.
@@ -158,7 +161,8 @@ def dequant_w32_f32s(codes: np.ndarray, scale_bits32: np.ndarray, group_size: in
     s = fp32_bits_to_float(scale_bits32)                # [G, N] float64, exact
     s_nk = s[np.arange(K) // group_size, :].T            # s32[k // gs, n] -> [N, K]
     exact = (codes - ZERO_POINT).astype(np.float64) * s_nk
-    return exact.astype(np.float32)
+    with np.errstate(over="ignore"):   # products beyond float32 become inf, as in IEEE arithmetic
+        return exact.astype(np.float32)
 
 
 def dequant_w16_bits_f32s(codes: np.ndarray, scale_bits32: np.ndarray, group_size: int) -> np.ndarray:
@@ -171,7 +175,8 @@ def dequant_w16_bits_f32s_fast(codes: np.ndarray, scale_bits32: np.ndarray, grou
     """Same values as ``dequant_w16_bits_f32s`` through numpy's float32 -> float16
     conversion (round to nearest even; the tests check it against the loop)."""
     w = dequant_w32_f32s(codes, scale_bits32, group_size)
-    return w.astype(np.float16).view(np.uint16)
+    with np.errstate(over="ignore"):
+        return w.astype(np.float16).view(np.uint16)
 
 
 def embedding_f32s(codes: np.ndarray, scale_bits32: np.ndarray, group_size: int, indices) -> np.ndarray:
@@ -241,3 +246,59 @@ def adapter_intermediate(act_bits, proj_bits):
 
 __all__ = [n for n in dir() if not n.startswith("_") and n not in ("annotations", "math", "np")]
 _ = dequant_w32  # re-exported helpers above come from the base oracle
+
+
+# ----------------------------------------------------------------------------
+# linear_dq8ca_q4gsw: int8 dynamically quantised activations x q4gsw weights
+# ----------------------------------------------------------------------------
+# "Upstream the Gemma 4 Vulkan support we carry on our ExecuTorch fork", issue
+# #1361, the fork's shader list: linear_dq8ca_q4gsw beside linear_q4gsw.  The
+# page gives only the name: 8-bit dynamically quantised activations ("dq8"),
+# quantised per channel-row with an asymmetric range ("ca"), times the 4-bit
+# group-symmetric weight.  Reading taken here (every step an IEEE fp32 operation,
+# round to nearest even, as a CPU or GPU computes it):
+#   per token m, over its K features:
+#     lo = min(0, min_k x[m, k]),  hi = max(0, max_k x[m, k])
+#     a_s = (hi - lo) / 255            (1 when hi == lo)
+#     a_z = clamp(rint(-128 - lo / a_s), -128, 127)
+#     q[m, k] = clamp(rint(x[m, k] / a_s) + a_z, -128, 127)
+#   y[m, n] = a_s[m] * sum_g s[g, n] * sum_{k in g} (q[m, k] - a_z[m]) (code[n, k] - 8)
+# The inner sums are exact integers; the bound is a_s sum_g |s| sum |q - a_z| |c - 8|.
+def dq8ca_quantize(x_bits):
+    """x fp16 bits [M, K] -> (q int8 [M, K], a_s float32 [M], a_z int32 [M])."""
+    x = fp16_bits_to_float(x_bits).astype(np.float32)          # exact: fp16 values are fp32 values
+    M, K = x.shape
+    q = np.zeros((M, K), np.int8)
+    a_s = np.zeros(M, np.float32)
+    a_z = np.zeros(M, np.int32)
+    for m in range(M):
+        lo = np.float32(min(np.float32(0), x[m].min()))
+        hi = np.float32(max(np.float32(0), x[m].max()))
+        s = np.float32(1) if hi == lo else np.float32(np.float32(hi - lo) / np.float32(255))
+        z = np.rint(np.float32(np.float32(-128) - np.float32(lo / s)))
+        z = int(min(127, max(-128, z)))
+        qm = np.rint(x[m] / s).astype(np.int64) + z            # x / s rounded once in float32
+        q[m] = np.clip(qm, -128, 127).astype(np.int8)
+        a_s[m] = s
+        a_z[m] = z
+    return q, a_s, a_z
+
+
+def linear_dq8ca_fwd(x_bits, codes, scale_bits, group_size):
+    """y = a_s * sum_g s * sum (q - a_z)(c - 8) on the quantised activations; returns (y, bound)."""
+    q, a_s, a_z = dq8ca_quantize(x_bits)
+    codes = np.asarray(codes, dtype=np.int64)
+    N, K = codes.shape
+    G = K // group_size
+    s = fp16_bits_to_float(scale_bits)                          # [G, N]
+    qa = q.astype(np.int64) - a_z[:, None].astype(np.int64)      # [M, K] exact
+    cw = codes - ZERO_POINT                                      # [N, K] exact
+    y = np.zeros((q.shape[0], N))
+    b = np.zeros((q.shape[0], N))
+    for g in range(G):
+        ks = slice(g * group_size, (g + 1) * group_size)
+        t = (qa[:, ks] @ cw[:, ks].T).astype(np.float64)        # exact integers
+        ta = (np.abs(qa[:, ks]) @ np.abs(cw[:, ks]).T).astype(np.float64)
+        y += t * s[g][None, :]
+        b += ta * np.abs(s[g])[None, :]
+    return y * a_s[:, None].astype(np.float64), b * a_s[:, None].astype(np.float64)

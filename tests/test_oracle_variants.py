@@ -333,3 +333,106 @@ def test_adapter_planted_mistakes_fail_a_pin():
     assert pin_ok(v.adapter_fwd)
     for bad in (transposed_product, dropped_adapter, sign_flip):
         assert not pin_ok(bad), bad.__name__
+
+
+# --------------------------------------------------------------------------- dq8ca
+def _dq8ca_fixture():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "dq8ca_rows.txt")):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            name, sb, z, *pairs = line.split()
+            xs = [float(p.split(":")[0]) for p in pairs]
+            qs = [int(p.split(":")[1]) for p in pairs]
+            rows.append((name, int(sb, 16), int(z), xs, qs))
+    return rows
+
+
+def test_dq8ca_quantisation_hand_rows():
+    for name, sb, z, xs, qs in _dq8ca_fixture():
+        x = np.array([xs], np.float16)
+        q, a_s, a_z = v.dq8ca_quantize(bits16(x))
+        assert int(np.float32(a_s[0]).view(np.uint32)) == sb, name
+        assert int(a_z[0]) == z, name
+        assert list(q[0].astype(int)) == qs, name
+
+
+def test_dq8ca_quantisation_properties():
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-4, 4, (64, 1)))).astype(np.float16)
+    x[3] = np.abs(x[3])          # one-signed rows: the range still holds 0
+    x[4] = -np.abs(x[4])
+    q, a_s, a_z = v.dq8ca_quantize(bits16(x))
+    xf = x.astype(np.float64)
+    assert q.min() >= -128 and q.max() <= 127
+    back = (q.astype(np.float64) - a_z[:, None]) * a_s[:, None].astype(np.float64)
+    # every value within half a step (plus the float32 rounding of x / a_s)
+    assert (np.abs(back - xf) <= a_s[:, None] * (0.5 + 1e-5)).all()
+    # zero is represented exactly: (q - a_z) == 0 where x == 0
+    x0 = x.copy()
+    x0[:, :8] = 0
+    q0, _, z0 = v.dq8ca_quantize(bits16(x0))
+    assert (q0[:, :8].astype(int) == z0[:, None]).all()
+
+
+def test_dq8ca_equals_the_base_product_when_quantisation_is_exact():
+    # integer activations spanning exactly [-100, 155]: a_s = 1, q - a_z = x
+    rng = np.random.default_rng(13)
+    M, N, K, gs = 4, 16, 128, 32
+    x = rng.integers(-100, 156, (M, K)).astype(np.float16)
+    x[:, 0], x[:, 1] = -100, 155
+    codes = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    s = np.ldexp(1.0, rng.integers(-6, -2, (K // gs, N))).astype(np.float16)
+    y8, _ = v.linear_dq8ca_fwd(bits16(x), codes, bits16(s), gs)
+    y, _ = o.linear_fwd(bits16(x), codes, bits16(s), gs)
+    assert np.array_equal(y8, y)
+
+
+def test_dq8ca_product_against_exact_rationals():
+    M, N, K, gs = 2, 8, 64, 32
+    inp = wl.random_inputs(M, N, K, gs, seed=14)
+    q, a_s, a_z = v.dq8ca_quantize(bits16(inp.x))
+    y, b = v.linear_dq8ca_fwd(bits16(inp.x), inp.codes, bits16(inp.scales), gs)
+    for m in range(M):
+        for n in range(N):
+            exact = Fraction(0)
+            babs = Fraction(0)
+            for g in range(K // gs):
+                t = sum((int(q[m, k]) - int(a_z[m])) * (int(inp.codes[n, k]) - 8) for k in range(g * gs, (g + 1) * gs))
+                ta = sum(abs((int(q[m, k]) - int(a_z[m])) * (int(inp.codes[n, k]) - 8))
+                         for k in range(g * gs, (g + 1) * gs))
+                exact += t * Fraction(float(inp.scales[g, n]))
+                babs += ta * abs(Fraction(float(inp.scales[g, n])))
+            exact *= Fraction(float(a_s[m]))
+            babs *= Fraction(float(a_s[m]))
+            assert abs(Fraction(float(y[m, n])) - exact) <= Fraction(1, 10 ** 12) * babs
+            assert abs(Fraction(float(b[m, n])) - babs) <= Fraction(1, 10 ** 12) * babs
+
+
+def test_dq8ca_planted_mistakes_fail_the_fixture():
+    def run(fn):
+        for name, sb, z, xs, qs in _dq8ca_fixture():
+            q, a_s, a_z = fn(bits16(np.array([xs], np.float16)))
+            if list(q[0].astype(int)) != qs or int(a_z[0]) != z:
+                return False
+        return True
+
+    def wrong_zero_point_sign(xb):
+        q, s, z = v.dq8ca_quantize(xb)
+        return np.clip(q.astype(int) - 2 * z[:, None], -128, 127).astype(np.int8), s, -z
+
+    def rounds_half_away(xb):   # round-half-away-from-zero instead of to even
+        x = o.fp16_bits_to_float(xb).astype(np.float32)
+        q, s, z = v.dq8ca_quantize(xb)
+        r = np.sign(x / s[:, None]) * np.floor(np.abs(x / s[:, None]) + 0.5)
+        return np.clip(r + z[:, None], -128, 127).astype(np.int8), s, z
+
+    def symmetric_range(xb):    # max |x| / 127, no zero point
+        x = o.fp16_bits_to_float(xb).astype(np.float32)
+        s = np.abs(x).max(axis=1) / np.float32(127)
+        s = np.where(s == 0, np.float32(1), s).astype(np.float32)
+        return np.clip(np.rint(x / s[:, None]), -128, 127).astype(np.int8), s, np.zeros(x.shape[0], np.int32)
+
+    assert run(v.dq8ca_quantize)
+    for bad in (wrong_zero_point_sign, rounds_half_away, symmetric_range):
+        assert not run(bad), bad.__name__
