@@ -590,6 +590,10 @@ def time_shape(q, sh, kind, device, flush, peaks):
     elif kind == "fwd":
         y = torch.empty((sh.M, sh.N), dtype=torch.float32, device=device)
         fn = lambda pk: q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a, y=y)
+    elif kind == "dq8ca":
+        y = torch.empty((sh.M, sh.N), dtype=torch.float32, device=device)
+        ws = torch.empty(q.library().q4gsw_dq8ca_workspace_bytes(sh.M, sh.K), dtype=torch.uint8, device=device)
+        fn = lambda pk: q.q4gsw_linear_dq8ca_fwd(pk, sh.N, sh.K, sh.group_size, a, y=y, workspace=ws)
     elif kind == "emb":
         ids = torch.from_numpy(wl.embedding_indices(sh)).to(device)
         y = torch.empty((sh.M, sh.K), dtype=torch.float32, device=device)
@@ -652,7 +656,9 @@ def time_shape(q, sh, kind, device, flush, peaks):
 
 # The configuration shapes timed beside the step: the memory-bound half of the
 # metric (decode M=1; the sweep's M=1 and M=16 on both 8B-class matrices) and
-# the largest compute-bound shapes (the sweep's M=4096).
+# the largest compute-bound shapes (the sweep's M=4096); the adapter and the
+# int8-activation product (dq8ca: algorithmic bytes as the fp16 forward, the
+# quantised copy of x in the workspace counts as overhead).
 SHAPE_LEGS = [("decode_N2048_K2048", "fwd"), ("decode_N8192_K2048", "fwd"), ("decode_N2048_K8192", "fwd"),
               ("sweep_M1_N14336_K4096", "fwd"), ("sweep_M1_N14336_K4096", "bwd"),
               ("sweep_M1_N4096_K14336", "fwd"), ("sweep_M1_N4096_K14336", "bwd"),
@@ -661,7 +667,9 @@ SHAPE_LEGS = [("decode_N2048_K2048", "fwd"), ("decode_N8192_K2048", "fwd"), ("de
               ("sweep_M4096_N14336_K4096", "fwd"), ("sweep_M4096_N14336_K4096", "bwd"),
               ("sweep_M4096_N4096_K14336", "fwd"), ("sweep_M4096_N4096_K14336", "bwd"),
               ("adapter_up_M512", "ad_fwd"), ("adapter_up_M512", "ad_bwd"),
-              ("adapter_down_M512", "ad_fwd"), ("adapter_down_M512", "ad_bwd")]
+              ("adapter_down_M512", "ad_fwd"), ("adapter_down_M512", "ad_bwd"),
+              ("decode_N8192_K2048", "dq8ca"), ("sweep_M1_N4096_K14336", "dq8ca"),
+              ("sweep_M16_N14336_K4096", "dq8ca")]
 
 
 def shape_legs(device, peaks, world):

@@ -47,6 +47,9 @@ SIGNATURES = [
     ("q4gsw_adapter_fwd", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP, _SZ, _VP]),
     ("q4gsw_adapter_bwd_input", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP, _SZ, _VP]),
     ("q4gsw_adapter_fwd_noalloc", _I, [_VP, _I, _I, _I, _VP, _VP, _I, _VP, _I, _VP, _VP]),
+    ("q4gsw_dq8ca_workspace_bytes", _SZ, [_I, _I]),
+    ("q4gsw_linear_dq8ca_fwd", _I, [_VP, _I, _I, _I, _VP, _I, _VP, _VP, _SZ, _VP]),
+    ("q4gsw_dq8ca_quantize", _I, [_VP, _I, _I, _VP, _SZ, _VP]),
     ("q4gsw_debug_pin_routes", _I, [_I, _I]),
     ("q4gsw_debug_wait_timeout", _I, [ctypes.c_uint, _VP]),
     ("q4gsw_last_route", ctypes.c_char_p, []),
@@ -243,6 +246,35 @@ def q4gsw_adapter_fwd(packed, N: int, K: int, group_size: int, a, b, x, y=None, 
 def q4gsw_adapter_bwd_input(packed, N: int, K: int, group_size: int, a, b, d_out, d_x=None, workspace=None):
     """d_x = d_out dequant(W) + (d_out b) a (input gradient of the adapter forward)."""
     return _adapter("q4gsw_adapter_bwd_input", packed, N, K, group_size, a, b, d_out, d_x, workspace, K)
+
+
+def q4gsw_linear_dq8ca_fwd(packed, N: int, K: int, group_size: int, x, y=None, workspace=None):
+    """y from int8 dynamically quantised x (per token, asymmetric) and the q4gsw weight."""
+    lib = library()
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.q4gsw_dq8ca_workspace_bytes(M, K)), 16), dtype=torch.uint8,
+                                device=x.device)
+    st = lib.q4gsw_linear_dq8ca_fwd(_dev(packed, torch.uint8, "packed"), N, K, group_size,
+                                    _dev(x, torch.float16, "x", 2), M, _dev(y, torch.float32, "y", 2),
+                                    _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(x))
+    _check("q4gsw_linear_dq8ca_fwd", st)
+    return y
+
+
+def q4gsw_dq8ca_quantize(x, workspace=None):
+    """The quantised activations of x: returns the workspace (see include/q4gsw.h for its map)."""
+    lib = library()
+    M, K = x.shape
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.q4gsw_dq8ca_workspace_bytes(M, K)), 16), dtype=torch.uint8,
+                                device=x.device)
+    st = lib.q4gsw_dq8ca_quantize(_dev(x, torch.float16, "x", 2), M, K, _dev(workspace, torch.uint8, "workspace"),
+                                  workspace.numel(), _stream(x))
+    _check("q4gsw_dq8ca_quantize", st)
+    return workspace
 
 
 GEMV_ROUTES = {"auto": 0, "reg": 1, "tma": 2}

@@ -225,7 +225,7 @@ const char* q4gsw_status_str(q4gsw_status s) {
     case Q4GSW_ERR_NULL: return "null pointer";
     case Q4GSW_ERR_SHAPE: return "invalid shape";
     case Q4GSW_ERR_ALIGN: return "misaligned pointer or shape (16-byte pointers, N % 8, K % 64)";
-    case Q4GSW_ERR_UNSUPPORTED: return "unsupported group size (power of two in [16, K])";
+    case Q4GSW_ERR_UNSUPPORTED: return "unsupported group size (power of two in [16, K]; at least 32 for linear_dq8ca)";
     case Q4GSW_ERR_CODE_RANGE: return "code above 15";
     case Q4GSW_ERR_CUDA: return "CUDA runtime error";
     case Q4GSW_ERR_SIZE: return "buffer too small";
@@ -323,6 +323,42 @@ q4gsw_status q4gsw_adapter_fwd_noalloc(const void* packed, int N, int K, int gro
   // the projection kernel writes every byte of the rows the GEMM reads, so
   // nothing left in the array by an earlier call needs clearing
   return adapter_impl(false, packed, N, K, group_size, a, b, r, x, M, y, scratch, scratch_bytes, stream);
+}
+
+size_t q4gsw_dq8ca_workspace_bytes(int M, int K) {
+  if (M < 0 || K <= 0 || K % 64) return 0;
+  return dq8ca_workspace_bytes(M, K);
+}
+
+q4gsw_status q4gsw_dq8ca_quantize(const uint16_t* x, int M, int K, void* workspace, size_t workspace_bytes,
+                                  q4gsw_stream_t stream) {
+  if (M < 0 || K <= 0 || K % 4) return Q4GSW_ERR_SHAPE;
+  if (K % 64) return Q4GSW_ERR_ALIGN;
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!x || !workspace) return Q4GSW_ERR_NULL;
+  if (!aligned16(x) || !aligned16(workspace)) return Q4GSW_ERR_ALIGN;
+  if (workspace_bytes < dq8ca_workspace_bytes(M, K)) return Q4GSW_ERR_SIZE;
+  set_route("dq8ca_quantize launches=1");
+  return from_cuda(launch_dq8ca_quantize(x, M, K, workspace, stream));
+}
+
+q4gsw_status q4gsw_linear_dq8ca_fwd(const void* packed, int N, int K, int group_size, const uint16_t* x, int M,
+                                    float* y, void* workspace, size_t workspace_bytes, q4gsw_stream_t stream) {
+  if (M < 0) return Q4GSW_ERR_SHAPE;
+  q4gsw_status st = check_weight_shape(N, K, group_size);
+  if (st != Q4GSW_OK) return st;
+  if (group_size < 32) return Q4GSW_ERR_UNSUPPORTED;   // a 32-column int8 MMA step lies in one group
+  if (M == 0) { set_route("empty"); return Q4GSW_OK; }
+  if (!packed || !x || !y || !workspace) return Q4GSW_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || !aligned16(workspace)) return Q4GSW_ERR_ALIGN;
+  if (workspace_bytes < dq8ca_workspace_bytes(M, K)) return Q4GSW_ERR_SIZE;
+  cudaError_t e = launch_dq8ca_quantize(x, M, K, workspace, stream);
+  if (e == cudaSuccess) e = launch_dq8ca_gemv(packed, N, K, group_size, M, workspace, single_output(y, N), stream);
+  char route[120];
+  snprintf(route, sizeof(route), "dq8ca launches=2 quantize + int8_gemv tiles=%d tokens_tiles=%d", (N + 15) / 16,
+           (M + 7) / 8);
+  set_route(route);
+  return from_cuda(e);
 }
 
 q4gsw_status q4gsw_debug_pin_routes(int gemv, int gemm) {

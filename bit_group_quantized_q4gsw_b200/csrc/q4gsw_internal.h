@@ -101,6 +101,15 @@ cudaError_t noalloc_scratch(void** ptr, size_t* bytes);
 cudaError_t launch_gemm_adapter(bool bwd, const void* packed, int N, int K, int gs, const uint16_t* act, int M,
                                 float* out, const AdapterRef& ad, cudaStream_t stream, char* route, int route_len);
 
+// int8 dynamically quantised activations (linear_dq8ca_q4gsw): workspace map
+// (q int8 [M][K], a_s fp32 [M], a_z int32 [M]), the quantiser and the product.
+size_t dq8ca_workspace_bytes(int M, int K);
+size_t dq8ca_scale_offset(int M, int K);
+size_t dq8ca_zero_offset(int M, int K);
+cudaError_t launch_dq8ca_quantize(const uint16_t* x, int M, int K, void* workspace, cudaStream_t stream);
+cudaError_t launch_dq8ca_gemv(const void* packed, int N, int K, int gs, int M, const void* workspace, OutSplit out,
+                              cudaStream_t stream);
+
 // Embedding rows out[t] = dequant(W)[indices[t]] (fp32); an index outside
 // [0, N) gives a zero row and sets kIndexErrorBit in the device error word.
 cudaError_t launch_embedding(const void* packed, int N, int K, int gs, bool f32s, const int32_t* indices, int T, float* out,

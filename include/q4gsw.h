@@ -302,6 +302,44 @@ Q4GSW_API q4gsw_status q4gsw_adapter_fwd_noalloc(const void *packed, int N, int 
                                        const uint16_t *x, int M, float *y,
                                        q4gsw_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * linear_dq8ca_q4gsw: int8 dynamically quantised activations x q4gsw weight
+ *
+ * "Upstream the Gemma 4 Vulkan support we carry on our ExecuTorch fork",
+ * issue #1361: the fork's shader list carries linear_dq8ca_q4gsw beside
+ * linear_q4gsw; the page gives only the name.  This library's reading
+ * (asymmetric per-token int8 activations, every step an IEEE fp32 operation
+ * rounding to nearest even):
+ *   lo = min(0, min_k x[m,k]),  hi = max(0, max_k x[m,k]),
+ *   a_s[m] = (hi - lo) / 255  (1 when hi == lo),
+ *   a_z[m] = clamp(rint(-128 - lo / a_s), -128, 127),
+ *   q[m,k] = clamp(rint(x[m,k] / a_s) + a_z, -128, 127),
+ *   y[m,n] = a_s[m] * sum_g s[g,n] * sum_{k in g} (q[m,k] - a_z[m]) * (code[n,k] - 8),
+ * the inner sums exact (int8 tensor-core MMAs into int32), the outer ones fp32.
+ * Error bound per element: 4e-3 * a_s * sum_g |s| * sum |q - a_z| |code - 8|
+ * (relative to the quantised activations, which this call defines).
+ *
+ * Workspace (device, caller-owned, q4gsw_dq8ca_workspace_bytes(M, K) bytes):
+ *   q    int8 [M][K] at 0; inside each 4-column group the bytes hold columns
+ *        +0, +2, +1, +3 (the packed codes' order);
+ *   a_s  fp32 [M]  at round_up(M*K, 256);
+ *   a_z  int32 [M] at that + round_up(4*M, 256).
+ * Two launches on `stream` (quantise, then the product); calls that share a
+ * workspace must be ordered on the GPU.  gs must be at least 32
+ * (Q4GSW_ERR_UNSUPPORTED otherwise); other checks as q4gsw_linear_fwd, plus
+ * Q4GSW_ERR_SIZE for a workspace that is too small.  Layout-version-1 blobs.
+ * ---------------------------------------------------------------------- */
+Q4GSW_API size_t q4gsw_dq8ca_workspace_bytes(int M, int K);
+Q4GSW_API q4gsw_status q4gsw_linear_dq8ca_fwd(const void *packed, int N, int K, int group_size,
+                                    const uint16_t *x, int M, float *y,
+                                    void *workspace, size_t workspace_bytes,
+                                    q4gsw_stream_t stream);
+/* The quantiser alone (the first launch of q4gsw_linear_dq8ca_fwd), for tests
+ * and for callers that reuse the quantised activations. */
+Q4GSW_API q4gsw_status q4gsw_dq8ca_quantize(const uint16_t *x, int M, int K,
+                                  void *workspace, size_t workspace_bytes,
+                                  q4gsw_stream_t stream);
+
 /*
  * Kernel health check.  Every wait inside this library's kernels is bounded
  * (one second of wall-clock time); a wait that runs out makes its kernel stop

@@ -21,7 +21,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = b.library()
     names = declared_functions()
-    assert len(names) == 25
+    assert len(names) == 28
     assert sorted(names) == sorted(n for n, _, _ in b.SIGNATURES)
     for n in names:
         assert hasattr(lib, n), n
@@ -184,3 +184,19 @@ def test_noalloc_adapter_rejects_sizes_beyond_its_array_on_the_host():
     # 8193 tokens need more than the 1 MiB array: rejected before any set-up or launch
     assert lib.q4gsw_adapter_fwd_noalloc(fake, 64, 128, 32, fake, fake, 16, fake, 8193, fake, None) == 7
     assert lib.q4gsw_adapter_fwd_noalloc(fake, 64, 128, 32, fake, fake, 16, fake, -1, fake, None) == 2
+
+
+def test_dq8ca_entry_points_check_arguments_on_the_host():
+    lib = b.library()
+    fake = 0x100000
+    need = lib.q4gsw_dq8ca_workspace_bytes(4, 128)
+    assert need == 512 + 256 + 256 and lib.q4gsw_dq8ca_workspace_bytes(4, 100) == 0
+    f = lib.q4gsw_linear_dq8ca_fwd
+    assert f(fake, 64, 128, 16, fake, 4, fake, fake, need, None) == 4          # gs 16: unsupported
+    assert f(fake, 64, 128, 32, fake, 4, fake, fake, need - 1, None) == 7      # workspace too small
+    assert f(fake, 64, 128, 32, fake, 4, fake, None, need, None) == 1
+    assert f(fake, 64, 96, 32, fake, 4, fake, fake, need, None) == 3
+    assert f(None, 64, 128, 32, None, 0, None, None, 0, None) == 0             # empty batch
+    g = lib.q4gsw_dq8ca_quantize
+    assert g(fake, 4, 100, fake, need, None) == 3 and g(fake, 4, -64, fake, need, None) == 2
+    assert g(fake, 4, 128, fake, need - 1, None) == 7
