@@ -347,16 +347,18 @@ q4gsw_status q4gsw_linear_dq8ca_fwd(const void* packed, int N, int K, int group_
   if (M < 0) return Q4GSW_ERR_SHAPE;
   q4gsw_status st = check_weight_shape(N, K, group_size);
   if (st != Q4GSW_OK) return st;
-  if (group_size < 32) return Q4GSW_ERR_UNSUPPORTED;   // a 32-column int8 MMA step lies in one group
+  // a 32-column int8 MMA step lies in one group; a group's int32 sums stay below 2^31
+  if (group_size < 32 || group_size > 65536) return Q4GSW_ERR_UNSUPPORTED;
   if (M == 0) { set_route("empty"); return Q4GSW_OK; }
   if (!packed || !x || !y || !workspace) return Q4GSW_ERR_NULL;
   if (!aligned16(packed) || !aligned16(x) || !aligned16(y) || !aligned16(workspace)) return Q4GSW_ERR_ALIGN;
   if (workspace_bytes < dq8ca_workspace_bytes(M, K)) return Q4GSW_ERR_SIZE;
+  char inner[96] = "";
   cudaError_t e = launch_dq8ca_quantize(x, M, K, workspace, stream);
-  if (e == cudaSuccess) e = launch_dq8ca_gemv(packed, N, K, group_size, M, workspace, single_output(y, N), stream);
-  char route[120];
-  snprintf(route, sizeof(route), "dq8ca launches=2 quantize + int8_gemv tiles=%d tokens_tiles=%d", (N + 15) / 16,
-           (M + 7) / 8);
+  if (e == cudaSuccess)
+    e = launch_dq8ca_gemv(packed, N, K, group_size, M, workspace, single_output(y, N), stream, inner, sizeof(inner));
+  char route[160];
+  snprintf(route, sizeof(route), "dq8ca launches=2 quantize + %s", inner);
   set_route(route);
   return from_cuda(e);
 }

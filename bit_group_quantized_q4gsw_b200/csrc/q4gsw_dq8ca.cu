@@ -8,16 +8,12 @@
 //                 q[k] = clamp(rint(x[k] / a_s) + a_z, -128, 127)   (fp32, ties to even)
 //   y[m, n] = a_s[m] sum_g s[g, n] sum_{k in g} (q[m, k] - a_z[m]) (code[n, k] - 8).
 //
-// Two kernels.  The quantiser writes q (int8, with the byte order of the packed
-// codes inside each 4-column group: columns +0, +2, +1, +3), a_s and a_z into
-// the caller's workspace.  The product runs int8 tensor-core MMAs
-// (mma.sync m16n8k32, unsigned codes x signed q, exact int32 sums):
-//   sum (q - a_z)(c - 8) = sum q c - 8 sum q - a_z sum c + 8 a_z n
-// over the n columns a warp accumulates; sum q c is the MMA of the codes (one
-// mask per row, no -8), sum c the MMA of the codes with a ones operand, sum q
-// the MMA of a ones operand with q.  A finished group is scaled by its fp16
-// scale in fp32; a_s multiplies at the end.
-#include <cooperative_groups.h>
+// This file holds the quantiser: one CTA per token writes q (int8, in the
+// packed codes' order: inside each 64-column block the 16 bytes at 16 t hold
+// columns 4 t + 16 i + (0, 2, 1, 3), i = 0..3, so that one 16-byte load gives a
+// lane its operand of a 64-column block), a_s and a_z into the caller's
+// workspace.  The product streams the weight through a TMA ring
+// (q4gsw_dq8ca_tma.cuh).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -27,13 +23,49 @@
 namespace q4gsw {
 namespace dq {
 
-constexpr int kQThreads = 256;
+constexpr int kQThreads = 1024;
+constexpr int kQVec = 4;   // 16-byte vectors a thread keeps in registers (K <= 32768 in one pass)
 
 // Workspace map for M tokens of K features (offsets in bytes).
 __host__ __device__ inline size_t off_as(int M, int K) { return round_up((size_t)M * K, 256); }
 __host__ __device__ inline size_t off_az(int M, int K) { return off_as(M, K) + round_up((size_t)4 * M, 256); }
 __host__ __device__ inline size_t ws_bytes(int M, int K) { return off_az(M, K) + round_up((size_t)4 * M, 256); }
 
+// q of one value, the fp32 steps of the reading
+__device__ __forceinline__ uint32_t quant_byte(float v, float as, int az) {
+  int qv = (int)rintf(__fdiv_rn(v, as)) + az;
+  qv = qv < -128 ? -128 : qv > 127 ? 127 : qv;
+  return (uint32_t)(qv & 0xFF);
+}
+
+// four consecutive values -> one word in the packed codes' byte order (+0, +2, +1, +3)
+__device__ __forceinline__ uint32_t quant_word(__half2 a, __half2 b, float as, int az) {
+  const float2 fa = __half22float2(a), fb = __half22float2(b);
+  return quant_byte(fa.x, as, az) | quant_byte(fb.x, as, az) << 8 | quant_byte(fa.y, as, az) << 16 |
+         quant_byte(fb.y, as, az) << 24;
+}
+
+__device__ __forceinline__ void range_of(const uint4& v, float& lo, float& hi) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(h[e]);
+    lo = fminf(lo, fminf(f.x, f.y));
+    hi = fmaxf(hi, fmaxf(f.x, f.y));
+  }
+}
+
+// columns 8 i .. 8 i + 7 of the row -> their q bytes: block i / 8, 16-column
+// step (i % 8) / 2, lanes t = 2 (i % 2) and 2 (i % 2) + 1 of that step
+__device__ __forceinline__ void store_q(uint8_t* qrow, int i, const uint4& v, float as, int az) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  uint8_t* dst = qrow + 64 * (i >> 3) + 32 * (i & 1) + 4 * ((i & 7) >> 1);
+  *reinterpret_cast<uint32_t*>(dst) = quant_word(h[0], h[1], as, az);
+  *reinterpret_cast<uint32_t*>(dst + 16) = quant_word(h[2], h[3], as, az);
+}
+
+// One CTA per token: the row's 16-byte vectors stay in registers between the
+// min/max reduction and the quantisation (rows past 32768 columns reload the rest).
 __global__ void __launch_bounds__(kQThreads)
 q4gsw_dq8ca_quantize_kernel(const __half* __restrict__ x, uint8_t* __restrict__ ws, int M, int K) {
   __shared__ float s_lo[kQThreads / 32], s_hi[kQThreads / 32];
@@ -42,13 +74,18 @@ q4gsw_dq8ca_quantize_kernel(const __half* __restrict__ x, uint8_t* __restrict__ 
   griddep_launch_dependents();
   griddep_wait();   // x may come from the previous kernel of the stream
   const int m = blockIdx.x;
-  const __half* row = x + (size_t)m * K;
-  float lo = 0.f, hi = 0.f;   // the range always holds 0
-  for (int k = threadIdx.x; k < K; k += kQThreads) {
-    const float v = __half2float(row[k]);
-    lo = fminf(lo, v);
-    hi = fmaxf(hi, v);
+  const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)m * K);
+  const int V = K >> 3;
+  uint4 v[kQVec];
+#pragma unroll
+  for (int u = 0; u < kQVec; ++u) {
+    const int i = threadIdx.x + u * kQThreads;
+    v[u] = i < V ? row[i] : make_uint4(0u, 0u, 0u, 0u);   // zeros: the range holds 0 anyway
   }
+  float lo = 0.f, hi = 0.f;   // the range always holds 0
+#pragma unroll
+  for (int u = 0; u < kQVec; ++u) range_of(v[u], lo, hi);
+  for (int i = threadIdx.x + kQVec * kQThreads; i < V; i += kQThreads) range_of(row[i], lo, hi);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -59,135 +96,34 @@ q4gsw_dq8ca_quantize_kernel(const __half* __restrict__ x, uint8_t* __restrict__ 
     s_hi[threadIdx.x >> 5] = hi;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < kQThreads / 32; ++w) {
-      lo = fminf(lo, s_lo[w]);
-      hi = fmaxf(hi, s_hi[w]);
+  if (threadIdx.x < 32) {
+    lo = s_lo[threadIdx.x];
+    hi = s_hi[threadIdx.x];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
-    lo = fminf(lo, s_lo[0]);
-    hi = fmaxf(hi, s_hi[0]);
-    const float as = hi == lo ? 1.f : __fdiv_rn(__fsub_rn(hi, lo), 255.f);
-    float z = rintf(__fsub_rn(-128.f, __fdiv_rn(lo, as)));
-    z = fminf(127.f, fmaxf(-128.f, z));
-    s_as = as;
-    s_az = (int)z;
-    reinterpret_cast<float*>(ws + off_as(M, K))[m] = as;
-    reinterpret_cast<int*>(ws + off_az(M, K))[m] = (int)z;
+    if (threadIdx.x == 0) {
+      const float as = hi == lo ? 1.f : __fdiv_rn(__fsub_rn(hi, lo), 255.f);
+      float z = rintf(__fsub_rn(-128.f, __fdiv_rn(lo, as)));
+      z = fminf(127.f, fmaxf(-128.f, z));
+      s_as = as;
+      s_az = (int)z;
+      reinterpret_cast<float*>(ws + off_as(M, K))[m] = as;
+      reinterpret_cast<int*>(ws + off_az(M, K))[m] = (int)z;
+    }
   }
   __syncthreads();
   const float as = s_as;
   const int az = s_az;
-  uint32_t* qrow = reinterpret_cast<uint32_t*>(ws + (size_t)m * K);
-  for (int c4 = threadIdx.x; c4 < K / 4; c4 += kQThreads) {
-    uint32_t word = 0;
+  uint8_t* qrow = ws + (size_t)m * K;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float v = __half2float(row[4 * c4 + e]);
-      int qv = (int)rintf(__fdiv_rn(v, as)) + az;
-      qv = qv < -128 ? -128 : qv > 127 ? 127 : qv;
-      const int slot = e == 1 ? 2 : e == 2 ? 1 : e;   // the packed codes' byte order
-      word |= (uint32_t)(qv & 0xFF) << (8 * slot);
-    }
-    qrow[c4] = word;
+  for (int u = 0; u < kQVec; ++u) {
+    const int i = threadIdx.x + u * kQThreads;
+    if (i < V) store_q(qrow, i, v[u], as, az);
   }
-}
-
-// D(16x8, s32) += A(16x32, u8, row) * B(32x8, s8, col)
-__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
-
-// grid = (ceil(N / 16) row tiles, 1, ceil(M / 8) token tiles); warp u takes the
-// 64-column blocks [u KB / 4, (u + 1) KB / 4) of the CTA's 16 rows.
-__global__ void __launch_bounds__(kThreads)
-q4gsw_dq8ca_gemv_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ ws, OutSplit out, int M,
-                        int N, int K, int gs) {
-  __shared__ float red[kWarps][8][16];   // [warp][token][row]
-  griddep_launch_dependents();
-  griddep_wait();   // the workspace comes from the quantiser just before
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int tile = blockIdx.x, tok0 = blockIdx.z * 8;
-  const int Mz = min(8, M - tok0);
-  const Layout L = layout_of(N, K, gs);
-  const __half* scales = reinterpret_cast<const __half*>(packed + L.scales_offset);
-  const int p_raw = tile * 8 + g;
-  const int p = p_raw < (N >> 1) ? p_raw : 0;            // rows past N read pair 0, never stored
-  const uint8_t* crow = packed + (size_t)p * K + 16 * t;
-  const int tok = tok0 + min(g, Mz - 1);                  // B column g: this token (repeated past Mz)
-  const uint8_t* qrow = ws + (size_t)tok * K + 4 * t;
-  const float* as_v = reinterpret_cast<const float*>(ws + off_as(M, K));
-  const int* az_v = reinterpret_cast<const int*>(ws + off_az(M, K));
-  // D columns 2t, 2t + 1 are tokens tok0 + 2t, tok0 + 2t + 1
-  const int ta = tok0 + min(2 * t, Mz - 1), tb = tok0 + min(2 * t + 1, Mz - 1);
-  const int az0 = az_v[ta], az1 = az_v[tb];
-  const int gsl = __ffs(gs) - 1;
-  const int KB = K >> 6;
-  const int b_begin = warp * KB / kWarps, b_end = (warp + 1) * KB / kWarps;
-  const uint32_t ones[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
-  const uint32_t ones2[2] = {0x01010101u, 0x01010101u};
-
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  int i1[4] = {0, 0, 0, 0}, i2[4] = {0, 0, 0, 0}, i3[4] = {0, 0, 0, 0};
-  int ncols = 0;
-  auto flush = [&](int grp) {
-    const __half2 s2 = *reinterpret_cast<const __half2*>(scales + (size_t)grp * N + 2 * p);
-    const float se = __low2float(s2), so = __high2float(s2);
-    // D fragment: [0] row g (even), token 2t; [1] row g, token 2t+1; [2] row g+8 (odd), 2t; [3] odd, 2t+1.
-    // i2 (code sums) is the same in every column; i3 (q sums) the same in every row.
-    const int n8 = 8 * ncols;
-    const int t0 = i1[0] - 8 * i3[0] - az0 * i2[0] + n8 * az0;
-    const int t1 = i1[1] - 8 * i3[1] - az1 * i2[1] + n8 * az1;
-    const int t2 = i1[2] - 8 * i3[2] - az0 * i2[2] + n8 * az0;
-    const int t3 = i1[3] - 8 * i3[3] - az1 * i2[3] + n8 * az1;
-    acc[0] = fmaf((float)t0, se, acc[0]);
-    acc[1] = fmaf((float)t1, se, acc[1]);
-    acc[2] = fmaf((float)t2, so, acc[2]);
-    acc[3] = fmaf((float)t3, so, acc[3]);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) i1[c] = i2[c] = i3[c] = 0;
-    ncols = 0;
-  };
-  for (int b = b_begin; b < b_end; ++b) {
-    const uint4 w = ldg_stream_v4(crow + 64 * b);
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {   // two 32-column MMA steps: words 2h, 2h + 1
-      const uint32_t w0 = words[2 * h], w1 = words[2 * h + 1];
-      const uint32_t a[4] = {w0 & 0x0F0F0F0Fu, (w0 >> 4) & 0x0F0F0F0Fu, w1 & 0x0F0F0F0Fu, (w1 >> 4) & 0x0F0F0F0Fu};
-      const int k0 = 64 * b + 32 * h;
-      const uint32_t bq[2] = {ldg_nc_u32(qrow + k0), ldg_nc_u32(qrow + k0 + 16)};
-      mma_u8s8(i1, a, bq);
-      mma_u8s8(i2, a, ones2);     // sum of the codes of each row
-      mma_u8s8(i3, ones, bq);     // sum of q of each token
-      ncols += 32;
-      // flush when the next step starts another group, or the warp's range ends
-      const int kn = k0 + 32;
-      if ((kn >> gsl) != (k0 >> gsl) || (b == b_end - 1 && h == 1)) flush(k0 >> gsl);
-    }
-  }
-  // y = a_s * acc; the warps' column ranges summed in order
-  red[warp][2 * t][2 * g] = acc[0];
-  red[warp][2 * t + 1][2 * g] = acc[1];
-  red[warp][2 * t][2 * g + 1] = acc[2];
-  red[warp][2 * t + 1][2 * g + 1] = acc[3];
-  __syncthreads();
-  for (int e = threadIdx.x; e < Mz * 16; e += kThreads) {
-    const int tk = e >> 4, nl = e & 15;
-    const int n = tile * 16 + nl;
-    if (n >= N) continue;
-    const float s = ((red[0][tk][nl] + red[1][tk][nl]) + red[2][tk][nl]) + red[3][tk][nl];
-    const size_t m = (size_t)(tok0 + tk);
-    const float v = s * as_v[m];
-    if (n < out.n1) out.y0[m * out.n1 + n] = v;
-    else if (n < out.n2) out.y1[m * (out.n2 - out.n1) + (n - out.n1)] = v;
-    else out.y2[m * (out.N - out.n2) + (n - out.n2)] = v;
-  }
+  for (int i = threadIdx.x + kQVec * kQThreads; i < V; i += kQThreads) store_q(qrow, i, row[i], as, az);
 }
 
 }  // namespace dq
@@ -208,21 +144,6 @@ cudaError_t launch_dq8ca_quantize(const uint16_t* x, int M, int K, void* workspa
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, dq::q4gsw_dq8ca_quantize_kernel, reinterpret_cast<const __half*>(x),
                             static_cast<uint8_t*>(workspace), M, K);
-}
-
-cudaError_t launch_dq8ca_gemv(const void* packed, int N, int K, int gs, int M, const void* workspace, OutSplit out,
-                              cudaStream_t stream) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((N + 15) / 16, 1, (M + 7) / 8);
-  cfg.blockDim = dim3(dq::kThreads, 1, 1);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dq::q4gsw_dq8ca_gemv_kernel, static_cast<const uint8_t*>(packed),
-                            static_cast<const uint8_t*>(workspace), out, M, N, K, gs);
 }
 
 }  // namespace q4gsw

@@ -615,6 +615,7 @@ static cudaError_t launch_gemm_impl(const void* packed, int N, int K, int gs, co
 #include "q4gsw_embedding.cuh"
 #include "q4gsw_gemm_ts.cuh"
 #include "q4gsw_gemv_tma.cuh"
+#include "q4gsw_dq8ca_tma.cuh"
 
 namespace q4gsw {
 

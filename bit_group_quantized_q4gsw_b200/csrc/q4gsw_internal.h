@@ -108,7 +108,7 @@ size_t dq8ca_scale_offset(int M, int K);
 size_t dq8ca_zero_offset(int M, int K);
 cudaError_t launch_dq8ca_quantize(const uint16_t* x, int M, int K, void* workspace, cudaStream_t stream);
 cudaError_t launch_dq8ca_gemv(const void* packed, int N, int K, int gs, int M, const void* workspace, OutSplit out,
-                              cudaStream_t stream);
+                              cudaStream_t stream, char* route, int route_len);
 
 // Embedding rows out[t] = dequant(W)[indices[t]] (fp32); an index outside
 // [0, N) gives a zero row and sets kIndexErrorBit in the device error word.

@@ -320,12 +320,13 @@ Q4GSW_API q4gsw_status q4gsw_adapter_fwd_noalloc(const void *packed, int N, int 
  * (relative to the quantised activations, which this call defines).
  *
  * Workspace (device, caller-owned, q4gsw_dq8ca_workspace_bytes(M, K) bytes):
- *   q    int8 [M][K] at 0; inside each 4-column group the bytes hold columns
- *        +0, +2, +1, +3 (the packed codes' order);
+ *   q    int8 [M][K] at 0, in the packed codes' order: inside each 64-column
+ *        block the 16 bytes at 16 t (t = 0..3) hold columns 4 t + 16 i +
+ *        (0, 2, 1, 3) for i = 0..3;
  *   a_s  fp32 [M]  at round_up(M*K, 256);
  *   a_z  int32 [M] at that + round_up(4*M, 256).
  * Two launches on `stream` (quantise, then the product); calls that share a
- * workspace must be ordered on the GPU.  gs must be at least 32
+ * workspace must be ordered on the GPU.  gs must lie in [32, 65536]
  * (Q4GSW_ERR_UNSUPPORTED otherwise); other checks as q4gsw_linear_fwd, plus
  * Q4GSW_ERR_SIZE for a workspace that is too small.  Layout-version-1 blobs.
  * ---------------------------------------------------------------------- */

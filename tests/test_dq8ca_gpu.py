@@ -36,7 +36,9 @@ def read_workspace(ws, M, K):
     """(q [M, K] int8 in column order, a_s fp32 [M], a_z int32 [M]) from the workspace."""
     lib = q().library()
     raw = ws.cpu().numpy()
-    qs = raw[:M * K].view(np.int8).reshape(M, K // 4, 4)[:, :, [0, 2, 1, 3]].reshape(M, K)
+    # byte 16 t + 4 i + slot of a 64-column block holds column 16 i + 4 t + (0, 2, 1, 3)[slot]
+    qs = raw[:M * K].view(np.int8).reshape(M, K // 64, 4, 4, 4)[..., [0, 2, 1, 3]]
+    qs = qs.transpose(0, 1, 3, 2, 4).reshape(M, K)
     o_s = lib.q4gsw_dq8ca_workspace_bytes(M, K) - 2 * (((4 * M) + 255) // 256 * 256)
     o_z = o_s + ((4 * M) + 255) // 256 * 256
     a_s = raw[o_s:o_s + 4 * M].view(np.float32)
