@@ -277,7 +277,7 @@ def q4gsw_dq8ca_quantize(x, workspace=None):
     return workspace
 
 
-GEMV_ROUTES = {"auto": 0, "reg": 1, "tma": 2}
+GEMV_ROUTES = {"auto": 0, "reg": 1, "tma": 2, "tma_xs": 3}
 GEMM_ROUTES = {"auto": 0, "ts": 1, "ss": 2, "ss1": 3, "ss2": 4}
 
 

@@ -364,7 +364,7 @@ q4gsw_status q4gsw_linear_dq8ca_fwd(const void* packed, int N, int K, int group_
 }
 
 q4gsw_status q4gsw_debug_pin_routes(int gemv, int gemm) {
-  if (gemv < kGemvAuto || gemv > kGemvTma || gemm < kGemmAuto || gemm > kGemmSs2) return Q4GSW_ERR_SHAPE;
+  if (gemv < kGemvAuto || gemv > kGemvTmaXs || gemm < kGemmAuto || gemm > kGemmSs2) return Q4GSW_ERR_SHAPE;
   route_pins().gemv = gemv;
   route_pins().gemm = gemm;
   return Q4GSW_OK;

@@ -44,7 +44,11 @@ constexpr int CTL_BYTES = 256;
 //   L1 and L2, and each of them would cost the TMA unit a tiny box per stage.
 //   ST: the ring depth that keeps a CTA near 56 KB, so that two CTAs of this
 //   launch and two of the next fit on one SM.
-template <int NT, int SPG, bool F32S>
+//   XS: the activations travel in the stage too, four [8 NT tokens][64 fp16]
+//   boxes (128-byte swizzle, rows past the batch zero-filled) after the codes,
+//   so they arrive ST stages ahead like the weights; the ring then holds four
+//   stages (NT = 1, four CTAs per SM) or five (NT = 2, two CTAs per SM).
+template <int NT, int SPG, bool F32S, bool XS = false>
 struct FwdCfg {
   static constexpr int CW = NT == 2 ? 8 : 4;                 // consumer warps
   static constexpr int RTW = 4 / (CW / 4);                   // row tiles per consumer warp
@@ -53,15 +57,18 @@ struct FwdCfg {
   static constexpr int MINB = NT == 1 ? 4 : 2;
   static constexpr int SB = F32S ? 4 : 2;                    // bytes per scale
   static constexpr int SCB = (SPG == 1 ? 16 : SPG == 2 ? 8 : 4) * 64 * SB;
-  static constexpr int OFF_SC = CODE_BYTES;
+  static constexpr int XBOX = 8 * NT * 128;                  // one activation box
+  static constexpr int OFF_X = CODE_BYTES;
+  static constexpr int OFF_SC = XS ? OFF_X + 4 * XBOX : CODE_BYTES;
   static constexpr int STAGE = (OFF_SC + SCB + 1023) / 1024 * 1024;
-  static constexpr int ST0 = 56 * 1024 / STAGE;
+  static constexpr int ST0 = (XS ? (NT == 1 ? 54 : 100) : 56) * 1024 / STAGE;
   static constexpr int ST = ST0 < 3 ? 3 : ST0 > 8 ? 8 : ST0;
   static constexpr int OFF_CTL = ST * STAGE;
   static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
   static constexpr int RED_FLOATS = 4 * 16 * 64;             // [block][token][row], reuses the ring
   static_assert(RED_FLOATS * 4 <= OFF_CTL, "warp partials fit in the ring");
   static_assert(ST <= 12, "barrier arrays");
+  static_assert(!XS || MINB * (BYTES + 1024) <= 228 * 1024, "resident CTAs");
 };
 
 struct Ctl {
@@ -96,13 +103,13 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 // grid = (ceil(N / 64) row tiles, S contraction splits, ceil(M / 16) token
 // slices), cluster = (1, S, 1).  SPG = 16-column steps per scale group
 // (1: gs 16, 2: gs 32, 4: gs >= 64).
-template <int NT, int SPG, bool F32S>
-__global__ void __launch_bounds__(FwdCfg<NT, SPG, F32S>::THREADS, FwdCfg<NT, SPG, F32S>::MINB)
+template <int NT, int SPG, bool F32S, bool XS>
+__global__ void __launch_bounds__(FwdCfg<NT, SPG, F32S, XS>::THREADS, FwdCfg<NT, SPG, F32S, XS>::MINB)
 q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
-                          const __half* __restrict__ x, OutSplit out, int M, int N, int K, int gs,
-                          int stages_total) {
+                          const __grid_constant__ CUtensorMap map_x, const __half* __restrict__ x, OutSplit out,
+                          int M, int N, int K, int gs, int stages_total) {
   using namespace sm100;
-  using C = FwdCfg<NT, SPG, F32S>;
+  using C = FwdCfg<NT, SPG, F32S, XS>;
   constexpr int RTW = C::RTW;
   constexpr int NGB = SPG == 4 ? 1 : 4 / SPG;   // scale groups per 64-column block
   extern __shared__ uint8_t smem_raw[];
@@ -131,12 +138,13 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     fence_mbar_init();
     prefetch_tmap(&map_pk);
     prefetch_tmap(&map_sc);
+    if (XS) prefetch_tmap(&map_x);
   }
   __syncthreads();
 
   // scale rows per stage: 256 / gs for gs <= 256, else 1
   const int sc_rows = gs < SK ? SK / gs : 1;
-  const uint32_t tx = CODE_BYTES + sc_rows * 64 * C::SB;
+  const uint32_t tx = CODE_BYTES + sc_rows * 64 * C::SB + (XS ? 4 * C::XBOX : 0);
 
   float acc[RTW][NT][4];
 #pragma unroll
@@ -158,6 +166,13 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         tma_load_2d(st + CODE_BYTES / 2, &map_pk, &ctl->full[s], kc + 128, n0 / 2);
         tma_load_2d(st + C::OFF_SC, &map_sc, &ctl->full[s], n0, kc >> gsl);
       };
+      auto load_x = [&](int it) {   // XS: the stage's activation boxes
+        const int s = it % C::ST;
+        const int kc = (st_begin + it) * SK;
+        uint8_t* st = smem + s * C::STAGE + C::OFF_X;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(st + b * C::XBOX, &map_x, &ctl->full[s], kc + 64 * b, tok0);
+      };
       // the packed weight is constant: the ring is filled before (and while)
       // the consumers wait for the kernel that produces x
       const int pre = nit < C::ST ? nit : C::ST;
@@ -165,12 +180,17 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         mbar_arrive_expect_tx(&ctl->full[it], tx);
         load_weights(it);
       }
+      if (XS) {
+        griddep_wait();
+        for (int it = 0; it < pre; ++it) load_x(it);
+      }
       int issued = pre;
       for (int it = pre; it < nit; ++it) {
         const int s = it % C::ST;
         if (!mbar_wait(&ctl->empty[s], ((it / C::ST) - 1) & 1, abort_flag, &g_device_error, 64u)) break;
         mbar_arrive_expect_tx(&ctl->full[s], tx);
         load_weights(it);
+        if (XS) load_x(it);
         issued = it + 1;
       }
       for (int it = (issued > C::ST ? issued - C::ST : 0); it < issued; ++it)
@@ -197,7 +217,13 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     const __half* xrow[NT];
 #pragma unroll
     for (int j = 0; j < NT; ++j) xrow[j] = x + (size_t)(tok0 + min(8 * j + g, Mz - 1)) * K + 64 * w + 4 * t;
+    // XS: the same fragment from the stage's box w, row 8 j + g, 16-byte
+    // chunk 2 i + t / 2 under the 128-byte swizzle, half t % 2 of it
+    uint32_t x_row[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) x_row[j] = C::OFF_X + w * C::XBOX + (8 * j + g) * 128 + 8 * (t & 1);
     auto load_xf = [&](int it, uint2 (&d)[NT][4]) {
+      if (XS) return;
       const int kb = (st_begin + it) * SK;   // the warp's block starts at kb + 64 w
       const bool in = kb + 64 * w < K;       // K % 64 == 0: a block is wholly inside or outside
 #pragma unroll
@@ -219,10 +245,16 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     bool fresh = true;   // the next MMA starts a new group (zero accumulator)
     // one stage: wait for its codes and scales, then dequantise and multiply;
     // false when a wait ran out
-    auto stage = [&](int it, const uint2 (&xv)[NT][4]) -> bool {
+    auto stage = [&](int it, const uint2 (&xg)[NT][4]) -> bool {
       const int s = it % C::ST;
       if (!mbar_wait(&ctl->full[s], (it / C::ST) & 1, abort_flag, &g_device_error, 128u)) return false;
       const uint32_t st = sbase + s * C::STAGE;
+      uint2 xv[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          xv[j][i] = XS ? lds64(st + x_row[j] + 16 * ((2 * i + (t >> 1)) ^ g)) : xg[j][i];
       uint4 wv[RTW];
 #pragma unroll
       for (int rt = 0; rt < RTW; ++rt) wv[rt] = lds128(st + code_off[rt]);
@@ -573,12 +605,12 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int NT, int SPG, bool F32S>
-static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUtensorMap& map_sc, const __half* x,
-                                           OutSplit out, int M, int N, int K, int gs, int stages_total, dim3 grid,
-                                           cudaStream_t stream) {
-  using C = gv::FwdCfg<NT, SPG, F32S>;
-  auto kern = gv::q4gsw_gemv_fwd_tma_kernel<NT, SPG, F32S>;
+template <int NT, int SPG, bool F32S, bool XS>
+static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUtensorMap& map_sc,
+                                           const CUtensorMap& map_x, const __half* x, OutSplit out, int M, int N,
+                                           int K, int gs, int stages_total, dim3 grid, cudaStream_t stream) {
+  using C = gv::FwdCfg<NT, SPG, F32S, XS>;
+  auto kern = gv::q4gsw_gemv_fwd_tma_kernel<NT, SPG, F32S, XS>;
   static PerDeviceOnce attr_once;
   {
     cudaError_t e = once_per_device(attr_once, current_device(), [&] {
@@ -600,7 +632,7 @@ static cudaError_t launch_gemv_tma_variant(const CUtensorMap& map_pk, const CUte
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, x, out, M, N, K, gs, stages_total);
+  return cudaLaunchKernelEx(&cfg, kern, map_pk, map_sc, map_x, x, out, M, N, K, gs, stages_total);
 }
 
 cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f32s, const uint16_t* x, int M,
@@ -622,26 +654,41 @@ cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f
   S = S < 1 ? 1 : (S > 8 ? 8 : S);
   while (S > 1 && stages_total / S < 2) --S;
   const int sc_rows = gs < gv::SK ? gv::SK / gs : 1;
-  CUtensorMap map_pk, map_sc;
+  // Activations staged in the ring (see FwdCfg) for 9..16 tokens or at least
+  // six stages per split; from global memory otherwise, where the smaller ring
+  // of the staged form has little to prefetch.  Measured on B200 (us per
+  // launch, from global -> staged): 16 x 14336 x 4096 17.1 -> 15.3,
+  // 16 x 4096 x 14336 18.0 -> 15.0, 1 x 4096 x 14336 12.2 -> 11.3,
+  // 1 x 8192 x 2048 5.8 -> 6.0.  Pins: 2 from global memory, 3 staged.
+  const int pin = route_pins().gemv;
+  const bool xs = pin == kGemvTmaXs || (pin != kGemvTma && (NT == 2 || stages_total / S >= 6));
+  CUtensorMap map_pk, map_sc, map_x;
   const bool ok =
       make_map_2d(&map_pk, CU_TENSOR_MAP_DATA_TYPE_UINT8, pk, K, N / 2, K, 128, gv::RP, CU_TENSOR_MAP_SWIZZLE_128B) &&
       make_map_2d(&map_sc, f32s ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                  pk + L.scales_offset, N, G, (uint64_t)N * sb, 64, sc_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+                  pk + L.scales_offset, N, G, (uint64_t)N * sb, 64, sc_rows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      (!xs || make_map_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, K, M, (uint64_t)K * 2, 64, 8 * NT,
+                          CU_TENSOR_MAP_SWIZZLE_128B));
   if (!ok) return cudaErrorInvalidValue;
+  if (!xs) map_x = map_pk;   // not read
   const dim3 grid(tiles, S, zs);
   cudaError_t e;
   const __half* xh = reinterpret_cast<const __half*>(x);
-#define Q4_TMA_FWD(NT_, SPG_)                                                                                    \
-  (f32s ? launch_gemv_tma_variant<NT_, SPG_, true>(map_pk, map_sc, xh, out, M, N, K, gs, stages_total, grid, stream) \
-        : launch_gemv_tma_variant<NT_, SPG_, false>(map_pk, map_sc, xh, out, M, N, K, gs, stages_total, grid, stream))
+#define Q4_TMA_FWD_X(NT_, SPG_, XS_)                                                                           \
+  (f32s ? launch_gemv_tma_variant<NT_, SPG_, true, XS_>(map_pk, map_sc, map_x, xh, out, M, N, K, gs, stages_total, \
+                                                        grid, stream)                                          \
+        : launch_gemv_tma_variant<NT_, SPG_, false, XS_>(map_pk, map_sc, map_x, xh, out, M, N, K, gs,          \
+                                                         stages_total, grid, stream))
+#define Q4_TMA_FWD(NT_, SPG_) (xs ? Q4_TMA_FWD_X(NT_, SPG_, true) : Q4_TMA_FWD_X(NT_, SPG_, false))
   if (NT == 1)
     e = spg == 1 ? Q4_TMA_FWD(1, 1) : spg == 2 ? Q4_TMA_FWD(1, 2) : Q4_TMA_FWD(1, 4);
   else
     e = spg == 1 ? Q4_TMA_FWD(2, 1) : spg == 2 ? Q4_TMA_FWD(2, 2) : Q4_TMA_FWD(2, 4);
 #undef Q4_TMA_FWD
+#undef Q4_TMA_FWD_X
   if (route)
-    snprintf(route, route_len, "gemv_tma_fwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S,
-             zs, stages_total);
+    snprintf(route, route_len, "gemv_tma_fwd launches=1 nt=%d tiles=%d splits=%d zslices=%d stages=%d%s", NT, tiles,
+             S, zs, stages_total, xs ? " x=staged" : "");
   return e;
 }
 

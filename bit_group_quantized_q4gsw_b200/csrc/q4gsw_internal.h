@@ -11,7 +11,7 @@ namespace q4gsw {
 
 // Route pins of the calling host thread (set by q4gsw_debug_pin_routes; 0
 // everywhere means the launchers choose).  Thread-local, like the route string.
-enum GemvPin { kGemvAuto = 0, kGemvReg = 1, kGemvTma = 2 };
+enum GemvPin { kGemvAuto = 0, kGemvReg = 1, kGemvTma = 2, kGemvTmaXs = 3 };
 enum GemmPin { kGemmAuto = 0, kGemmTs = 1, kGemmSs = 2, kGemmSs1 = 3, kGemmSs2 = 4 };
 struct RoutePins {
   int gemv = kGemvAuto;

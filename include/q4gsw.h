@@ -372,7 +372,8 @@ Q4GSW_API q4gsw_status q4gsw_dequant(const void *packed, int N, int K, int group
 /*
  * Debug export (tests and tuning): pins the kernel route of the calls this
  * host thread makes from now on.
- *   gemv  calls with M <= 16:  0 automatic, 1 register-fed GEMV, 2 TMA-ring GEMV
+ *   gemv  calls with M <= 16:  0 automatic, 1 register-fed GEMV, 2 TMA-ring GEMV,
+ *         3 TMA-ring GEMV whose forward stages the activations in the ring too
  *         (the input gradient has no TMA-ring/register choice other than these two)
  *   gemm  calls with M > 16:   0 automatic, 1 tensor-memory GEMM, 2 shared-memory
  *         GEMM (accumulators per CTA chosen), 3 shared-memory GEMM with one

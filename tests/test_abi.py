@@ -122,10 +122,10 @@ def test_embedding_token_ids_are_seeded_and_in_range():
 def test_debug_route_pins_are_checked_and_thread_local():
     import threading
     lib = b.library()
-    assert lib.q4gsw_debug_pin_routes(3, 0) == 2          # gemv pin out of range
+    assert lib.q4gsw_debug_pin_routes(4, 0) == 2          # gemv pin out of range
     assert lib.q4gsw_debug_pin_routes(0, 5) == 2          # gemm pin out of range
     assert lib.q4gsw_debug_pin_routes(-1, 0) == 2
-    for gemv in range(3):
+    for gemv in range(4):
         for gemm in range(5):
             assert lib.q4gsw_debug_pin_routes(gemv, gemm) == 0
     seen = []

@@ -209,9 +209,10 @@ def test_odd_weight_shapes(N, K, gs):
     check_bwd(inp, gs)
 
 
-@pytest.fixture(params=["tma", "reg"])
+@pytest.fixture(params=["tma", "tma_xs", "reg"])
 def gemv_variant(request):
-    """Pins the GEMV: TMA-ring weight stream or register-fed (q4gsw_debug_pin_routes)."""
+    """Pins the GEMV: TMA-ring weight stream (activations from global memory, or
+    staged in the ring) or register-fed (q4gsw_debug_pin_routes)."""
     q().q4gsw_debug_pin_routes(gemv=request.param)
     yield request.param
     q().q4gsw_debug_pin_routes()
@@ -224,10 +225,12 @@ def test_gemv_routes(M, N, K, gs, gemv_variant):
     inp = wl.random_inputs(M, N, K, gs, seed=3 * M + N + K)
     check_fwd(inp, gs)
     route = q().q4gsw_last_route()
-    assert route.startswith("gemv_tma_fwd" if gemv_variant == "tma" else "gemv_fwd"), route
+    tma = gemv_variant != "reg"
+    assert route.startswith("gemv_tma_fwd" if tma else "gemv_fwd"), route
+    assert ("x=staged" in route) == (gemv_variant == "tma_xs"), route
     check_bwd(inp, gs)
     route = q().q4gsw_last_route()
-    assert route.startswith("gemv_tma_bwd" if gemv_variant == "tma" else "gemv_bwd"), route
+    assert route.startswith("gemv_tma_bwd" if tma else "gemv_bwd"), route
     inp = wl.integer_exact_inputs(M, N, K, gs, seed=M + 1)
     y, _ = run_fwd(inp, gs)
     ref, _ = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), gs)

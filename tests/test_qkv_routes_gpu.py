@@ -57,10 +57,10 @@ def check_route(M, split_name, gemv="auto", gemm="auto", route_prefix=""):
 
 
 @pytest.mark.parametrize("split_name", ["config", "ragged"])
-@pytest.mark.parametrize("gemv", ["reg", "tma"])
+@pytest.mark.parametrize("gemv", ["reg", "tma", "tma_xs"])
 @pytest.mark.parametrize("M", [1, 4, 9, 16])
 def test_qkv_gemv_routes(M, gemv, split_name):
-    check_route(M, split_name, gemv=gemv, route_prefix="gemv_tma_fwd" if gemv == "tma" else "gemv_fwd")
+    check_route(M, split_name, gemv=gemv, route_prefix="gemv_fwd" if gemv == "reg" else "gemv_tma_fwd")
 
 
 @pytest.mark.parametrize("split_name", ["config", "ragged"])
