@@ -11,10 +11,14 @@
 // then adds u B^T (or v A) as one more 64-deep contraction stage of its
 // accumulator.
 //
-// One CTA per 16 tokens; eight warps split the contraction, each running
-// mma.sync m16n8k16 (A = 16 tokens x 16 contraction indices of the activation,
-// B = 16 contraction indices x 8 rank columns of the projection), and the
-// eight partial tiles are summed in shared memory in a fixed order.
+// A cluster of KS CTAs per 16 tokens splits the contraction (KS <= 8, chosen
+// to give the launch about two CTAs per SM); the eight warps of a CTA split its
+// slice again, each running mma.sync m16n8k16 (A = 16 tokens x 16 contraction
+// indices of the activation, B = 16 contraction indices x 8 rank columns of the
+// projection).  The eight warp tiles are summed in shared memory, and rank rk
+// of the cluster sums token rows [16 rk / KS, 16 (rk + 1) / KS) of the KS CTA
+// tiles through distributed shared memory, both in a fixed order.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -23,6 +27,7 @@
 
 namespace q4gsw {
 namespace ad {
+namespace cg = cooperative_groups;
 
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
@@ -35,13 +40,17 @@ __global__ void __launch_bounds__(kThreads)
 q4gsw_adapter_proj_kernel(const __half* __restrict__ act, const __half* __restrict__ proj, __half* __restrict__ out,
                           int M, int C, int r) {
   __shared__ float red[kWarps][16][kRankMax];
+  __shared__ float cta_sum[16][kRankMax];
   griddep_launch_dependents();
   griddep_wait();   // the activations may come from the previous kernel of the stream
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int m0 = blockIdx.x * 16;
+  const int KS = gridDim.y, ks = blockIdx.y;
   const int steps = (C + 15) / 16;   // C % 8 == 0: the last step may hold only 8 columns
-  const int s_begin = warp * steps / kWarps, s_end = (warp + 1) * steps / kWarps;
+  const int c_begin = ks * steps / KS, c_end = (ks + 1) * steps / KS;
+  const int s_begin = c_begin + warp * (c_end - c_begin) / kWarps;
+  const int s_end = c_begin + (warp + 1) * (c_end - c_begin) / kWarps;
   const int nj = (r + 7) / 8;  // 8-column rank tiles
   // rows past M read row M - 1 (never stored)
   const __half* a0 = act + (size_t)min(m0 + g, M - 1) * C;
@@ -89,12 +98,23 @@ q4gsw_adapter_proj_kernel(const __half* __restrict__ act, const __half* __restri
   __syncthreads();
   for (int e = threadIdx.x; e < 16 * kRankMax; e += kThreads) {
     const int row = e / kRankMax, j = e % kRankMax;
-    if (m0 + row >= M) continue;
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) s += red[w][row][j];
+    cta_sum[row][j] = s;
+  }
+  cg::cluster_group cluster = cg::this_cluster();
+  if (KS > 1) cluster.sync();
+  else __syncthreads();
+  const int rb = ks * 16 / KS, re = (ks + 1) * 16 / KS;
+  for (int e = rb * kRankMax + threadIdx.x; e < re * kRankMax; e += kThreads) {
+    const int row = e / kRankMax, j = e % kRankMax;
+    if (m0 + row >= M) continue;
+    float s = 0.f;
+    for (int q = 0; q < KS; ++q) s += (KS > 1 ? cluster.map_shared_rank(&cta_sum[0][0], q) : &cta_sum[0][0])[e];
     out[(size_t)(m0 + row) * kRankMax + j] = j < r ? __float2half_rn(s) : __float2half_rn(0.f);
   }
+  if (KS > 1) cluster.sync();   // no CTA leaves while another reads its tile
 }
 
 }  // namespace ad
@@ -123,15 +143,26 @@ cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
 
 cudaError_t launch_adapter_proj(const uint16_t* act, const uint16_t* proj, bool by_rows, int M, int C, int r,
                                 void* workspace, cudaStream_t stream) {
+  // contraction splits: about two CTAs per SM, at least two 16-column steps
+  // per warp, clusters of at most 8
+  const int tiles = (M + 15) / 16;
+  const int steps = (C + 15) / 16;
+  int KS = (2 * sm_count(current_device()) + tiles - 1) / tiles;
+  KS = KS > 8 ? 8 : KS;
+  while (KS > 1 && steps / KS < 2 * ad::kWarps) --KS;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((M + 15) / 16, 1, 1);
+  cfg.gridDim = dim3(tiles, KS, 1);
   cfg.blockDim = dim3(ad::kThreads, 1, 1);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = KS;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const __half* a = reinterpret_cast<const __half*>(act);
   const __half* p = reinterpret_cast<const __half*>(proj);
   __half* o = static_cast<__half*>(workspace);
