@@ -233,6 +233,14 @@ q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __
 #pragma unroll
         for (int h = 0; h < 2; ++h) sw[h][rt] = lds32(st + sc_off[h] + 32 * rt);
       }
+      {
+        uint32_t dep = 0u;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) dep ^= qv[j].x ^ qv[j].y ^ qv[j].z ^ qv[j].w;
+#pragma unroll
+        for (int rt = 0; rt < RTW; ++rt) dep ^= wv[rt].x ^ wv[rt].y ^ wv[rt].z ^ wv[rt].w ^ sw[0][rt] ^ sw[1][rt];
+        stage_reads_done(dep);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
       const int k0 = (st_begin + it) * SK + 64 * w;

@@ -598,6 +598,11 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
   }
   attr[0].val.clusterDim.z = best_S;
   cfg.gridDim = dim3(tiles_f, tiles_t, best_S);
+  // With split-K the threads sum the S partial tiles through distributed
+  // shared memory and write the outputs (fixed order), instead of rank 0's
+  // tensor store followed, once it has completed, by the other ranks'
+  // reduce-adds.
+  if (best_S > 1) a.tma_out = 0;
   if (route)
     snprintf(route, route_len, "tcgen05_ts_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d out=%s%s",
              BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, WST, tiles_f, tiles_t, best_S, a.tma_out ? "tma" : "st",

@@ -266,6 +266,21 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
           const uint32_t a = st + sc_off[q] + 16 * C::SB * rt;
           sw[rt][q] = F32S ? lds64(a) : make_uint2(lds32(a), 0u);
         }
+      {
+        uint32_t dep = 0u;
+#pragma unroll
+        for (int rt = 0; rt < RTW; ++rt) {
+          dep ^= wv[rt].x ^ wv[rt].y ^ wv[rt].z ^ wv[rt].w;
+#pragma unroll
+          for (int q = 0; q < NGB; ++q) dep ^= sw[rt][q].x ^ sw[rt][q].y;
+        }
+        if (XS)
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dep ^= xv[j][i].x ^ xv[j][i].y;
+        stage_reads_done(dep);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
 
@@ -528,6 +543,14 @@ q4gsw_gemv_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
       for (int q = 0; q < SPB; ++q) {
         sa[q] = F32S ? lds64(st + scA[q]) : make_uint2(lds32(st + scA[q]), 0u);
         sb[q] = F32S ? lds64(st + scB[q]) : make_uint2(lds32(st + scB[q]), 0u);
+      }
+      {
+        uint32_t dep = va.x ^ va.y ^ va.z ^ va.w ^ vb.x ^ vb.y ^ vb.z ^ vb.w;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) dep ^= bfr[j][0] ^ bfr[j][1];
+#pragma unroll
+        for (int q = 0; q < SPB; ++q) dep ^= sa[q].x ^ sa[q].y ^ sb[q].x ^ sb[q].y;
+        stage_reads_done(dep);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers

@@ -143,6 +143,18 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor-core operand reads).
+// Release of a ring stage whose words a warp has loaded into registers:
+// `dep` folds every loaded word, so the warp waits here until its loads have
+// returned, and the proxy fence orders those reads before the TMA writes of
+// the stage's next fill.  Without both, a refill could land before a lagging
+// load had read (measured on B200: wrong partial sums in about one launch in
+// six of a 2-CTA-per-SM, 2-split backward GEMV).  Call before the __syncwarp
+// that precedes the warp's arrive on the stage's "empty" barrier.
+__device__ __forceinline__ void stage_reads_done(uint32_t dep) {
+  asm volatile("" ::"r"(dep));
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
