@@ -568,7 +568,7 @@ def time_shape(q, sh, kind, device, flush, peaks):
     first = q.q4gsw_prepack(codes, scales, sh.group_size)
     del codes, scales
     wb = weight_bytes(sh)
-    R = max(2, math.ceil(3 * L2_BYTES / wb))
+    R = max(2, math.ceil(max(3 * L2_BYTES, 512 * 2**20) / wb))   # at least 512 MB of weight copies
     packs = [first] + [first.clone() for _ in range(R - 1)]
     src = inp.d_out if kind in ("bwd", "ad_bwd") else inp.x
     a = torch.from_numpy(src).to(device)
@@ -641,7 +641,7 @@ def time_shape(q, sh, kind, device, flush, peaks):
            "frac_tc": fl / t / 1e12 / peaks["tflops"], "frac_hbm_measured": by / t / 1e9 / peaks["hbm_gbs"],
            "frac_hbm_8tbs": by / t / 8e12, "us_single_cold": t1, "route": route, "copies": R,
            "timing": f"CUDA graph of {iters} back-to-back launches over {R} rotating weight copies "
-                     f"(> 3x L2), {reps} replays; us_single_cold: one launch after a 256 MB L2 flush"}
+                     f"(>= 512 MB, > 3x L2), {reps} replays; us_single_cold: one launch after a 256 MB L2 flush"}
     ridge = peaks["tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if kind != "emb" and fl / by >= ridge:
         rec["roofline"] = {"bound": "tensor", "achieved": fl / t / 1e12, "peak": peaks["tflops"], "unit": "TFLOP/s",
