@@ -720,7 +720,7 @@ def run_case(args):
     inp = wl.make_inputs(sh, M=M)
     pk = q.q4gsw_prepack(torch.from_numpy(inp.codes).to(device), torch.from_numpy(inp.scales).to(device),
                          sh.group_size)
-    a = torch.from_numpy(inp.d_out if kind == "bwd" else inp.x).to(device)
+    a = torch.from_numpy(inp.d_out if kind in ("bwd", "ad_bwd") else inp.x).to(device)
     for _ in range(args.iters):
         if kind == "qkv":
             Nq, Nk, Nv = sh.splits
@@ -729,6 +729,16 @@ def run_case(args):
             q.q4gsw_linear_fwd(pk, sh.N, sh.K, sh.group_size, a)
         elif kind == "emb":
             q.q4gsw_embedding(pk, sh.N, sh.K, sh.group_size, torch.from_numpy(wl.embedding_indices(sh, M)).to(device))
+        elif kind == "dq8ca":
+            q.q4gsw_linear_dq8ca_fwd(pk, sh.N, sh.K, sh.group_size, a)
+        elif kind in ("ad_fwd", "ad_bwd"):
+            rng = np.random.default_rng(sh.seed + 1)
+            A = torch.from_numpy((rng.standard_normal((ADAPTER_RANK, sh.K)) * 0.05).astype(np.float16)).to(device)
+            B = torch.from_numpy((rng.standard_normal((sh.N, ADAPTER_RANK)) * 0.05).astype(np.float16)).to(device)
+            if kind == "ad_fwd":
+                q.q4gsw_adapter_fwd(pk, sh.N, sh.K, sh.group_size, A, B, a)
+            else:
+                q.q4gsw_adapter_bwd_input(pk, sh.N, sh.K, sh.group_size, A, B, a)
         else:
             q.q4gsw_linear_bwd_input(pk, sh.N, sh.K, sh.group_size, a)
     torch.cuda.synchronize()
