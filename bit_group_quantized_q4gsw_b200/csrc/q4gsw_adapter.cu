@@ -35,7 +35,14 @@ constexpr int kRankMax = 64;
 
 // act [M][C] fp16 row-major; the projection P(c, j) is proj[j * C + c] when
 // BY_ROWS (forward: A [r, C]) or proj[c * r + j] (backward: B [C, r]).
-template <bool BY_ROWS>
+__device__ __forceinline__ uint4 ldg_nc_v4h(const __half* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// NJ: 8-column rank tiles held per lane (2, 4 or 8: ranks up to 16, 32, 64)
+template <bool BY_ROWS, int NJ>
 __global__ void __launch_bounds__(kThreads)
 q4gsw_adapter_proj_kernel(const __half* __restrict__ act, const __half* __restrict__ proj, __half* __restrict__ out,
                           int M, int C, int r) {
@@ -47,17 +54,17 @@ q4gsw_adapter_proj_kernel(const __half* __restrict__ act, const __half* __restri
   const int g = lane >> 2, t = lane & 3;
   const int m0 = blockIdx.x * 16;
   const int KS = gridDim.y, ks = blockIdx.y;
-  const int steps = (C + 15) / 16;   // C % 8 == 0: the last step may hold only 8 columns
-  const int c_begin = ks * steps / KS, c_end = (ks + 1) * steps / KS;
+  const int chunks = (C + 63) / 64;   // 64-column chunks; C % 8 == 0, so an 8-column group is wholly in or out
+  const int c_begin = ks * chunks / KS, c_end = (ks + 1) * chunks / KS;
   const int s_begin = c_begin + warp * (c_end - c_begin) / kWarps;
   const int s_end = c_begin + (warp + 1) * (c_end - c_begin) / kWarps;
   const int nj = (r + 7) / 8;  // 8-column rank tiles
   // rows past M read row M - 1 (never stored)
   const __half* a0 = act + (size_t)min(m0 + g, M - 1) * C;
   const __half* a1 = act + (size_t)min(m0 + g + 8, M - 1) * C;
-  float acc[8][4];
+  float acc[NJ][4];
 #pragma unroll
-  for (int jt = 0; jt < 8; ++jt)
+  for (int jt = 0; jt < NJ; ++jt)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[jt][c] = 0.f;
   auto pval = [&](int c, int j) -> uint32_t {   // P(c, j) as fp16 bits, zero past the rank
@@ -65,35 +72,64 @@ q4gsw_adapter_proj_kernel(const __half* __restrict__ act, const __half* __restri
     const __half v = BY_ROWS ? proj[(size_t)j * C + c] : proj[(size_t)c * r + j];
     return __half_as_ushort(v);
   };
-#pragma unroll 2
-  for (int st = s_begin; st < s_end; ++st) {
-    const int c0 = 16 * st;
-    const bool hi_ok = c0 + 8 < C;   // columns c0 + 8 .. c0 + 15 exist
-    const uint32_t af[4] = {ldg_nc_u32(a0 + c0 + 2 * t), ldg_nc_u32(a1 + c0 + 2 * t),
-                            hi_ok ? ldg_nc_u32(a0 + c0 + 2 * t + 8) : 0u, hi_ok ? ldg_nc_u32(a1 + c0 + 2 * t + 8) : 0u};
+  // Chunk of 64 columns: lane t loads columns c0 + 16 t .. + 15 of its two
+  // token rows as two 16-byte vectors each, and MMA step s (0..3) takes the
+  // column pairs (16 t + 2 s, + 1) as contraction indices (2t, 2t + 1) and
+  // (16 t + 8 + 2 s, + 1) as (2t + 8, 2t + 9).  The permutation depends on t
+  // only, so the projection's fragments follow it (16-byte loads of A's rows
+  // in the forward).  Every load of a chunk is issued before its MMAs.
+  for (int ch = s_begin; ch < s_end; ++ch) {
+    const int c0 = 64 * ch + 16 * t;
+    const bool in0 = c0 + 8 <= C, in1 = c0 + 16 <= C;
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    uint4 x0[2], x1[2];   // rows g and g + 8, columns c0 .. c0 + 7 and c0 + 8 .. c0 + 15
+    x0[0] = in0 ? ldg_nc_v4h(a0 + c0) : z4;
+    x0[1] = in1 ? ldg_nc_v4h(a0 + c0 + 8) : z4;
+    x1[0] = in0 ? ldg_nc_v4h(a1 + c0) : z4;
+    x1[1] = in1 ? ldg_nc_v4h(a1 + c0 + 8) : z4;
+    uint4 p[NJ][2];   // projection column j = 8 jt + g at the same columns
 #pragma unroll
-    for (int jt = 0; jt < 8; ++jt) {
-      if (jt >= nj) break;
+    for (int jt = 0; jt < NJ; ++jt) {
       const int j = 8 * jt + g;
-      uint32_t bf[2];
-      if (BY_ROWS) {
-        // A[j][c], A[j][c + 1] are adjacent
-        bf[0] = j < r ? ldg_nc_u32(proj + (size_t)j * C + c0 + 2 * t) : 0u;
-        bf[1] = (j < r && hi_ok) ? ldg_nc_u32(proj + (size_t)j * C + c0 + 2 * t + 8) : 0u;
+      if (jt < nj && j < r) {
+        if (BY_ROWS) {
+          p[jt][0] = in0 ? ldg_nc_v4h(proj + (size_t)j * C + c0) : z4;
+          p[jt][1] = in1 ? ldg_nc_v4h(proj + (size_t)j * C + c0 + 8) : z4;
+        } else {
+          uint32_t w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = c0 + 2 * (e & 3) + 8 * (e >> 2);
+            w[e] = c + 2 <= C ? pval(c, j) | (pval(c + 1, j) << 16) : 0u;
+          }
+          p[jt][0] = make_uint4(w[0], w[1], w[2], w[3]);
+          p[jt][1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       } else {
-        bf[0] = pval(c0 + 2 * t, j) | (pval(c0 + 2 * t + 1, j) << 16);
-        bf[1] = hi_ok ? pval(c0 + 2 * t + 8, j) | (pval(c0 + 2 * t + 9, j) << 16) : 0u;
+        p[jt][0] = p[jt][1] = z4;
       }
-      mma_16816(acc[jt], af, bf);
+    }
+    const uint32_t* r0 = reinterpret_cast<const uint32_t*>(x0);
+    const uint32_t* r1 = reinterpret_cast<const uint32_t*>(x1);
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+      const uint32_t af[4] = {r0[st], r1[st], r0[4 + st], r1[4 + st]};
+#pragma unroll
+      for (int jt = 0; jt < NJ; ++jt) {
+        if (jt >= nj) break;
+        const uint32_t* pj = reinterpret_cast<const uint32_t*>(p[jt]);
+        const uint32_t bf[2] = {pj[st], pj[4 + st]};
+        mma_16816(acc[jt], af, bf);
+      }
     }
   }
   // D fragment: rows g, g + 8 (tokens), columns 2t, 2t + 1 of rank tile jt
 #pragma unroll
-  for (int jt = 0; jt < 8; ++jt) {
-    red[warp][g][8 * jt + 2 * t] = acc[jt][0];
-    red[warp][g][8 * jt + 2 * t + 1] = acc[jt][1];
-    red[warp][g + 8][8 * jt + 2 * t] = acc[jt][2];
-    red[warp][g + 8][8 * jt + 2 * t + 1] = acc[jt][3];
+  for (int jt = 0; jt < 8; ++jt) {   // rank tiles past NJ hold zeros
+    red[warp][g][8 * jt + 2 * t] = jt < NJ ? acc[jt < NJ ? jt : 0][0] : 0.f;
+    red[warp][g][8 * jt + 2 * t + 1] = jt < NJ ? acc[jt < NJ ? jt : 0][1] : 0.f;
+    red[warp][g + 8][8 * jt + 2 * t] = jt < NJ ? acc[jt < NJ ? jt : 0][2] : 0.f;
+    red[warp][g + 8][8 * jt + 2 * t + 1] = jt < NJ ? acc[jt < NJ ? jt : 0][3] : 0.f;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < 16 * kRankMax; e += kThreads) {
@@ -143,13 +179,13 @@ cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
 
 cudaError_t launch_adapter_proj(const uint16_t* act, const uint16_t* proj, bool by_rows, int M, int C, int r,
                                 void* workspace, cudaStream_t stream) {
-  // contraction splits: about two CTAs per SM, at least two 16-column steps
+  // contraction splits: about two CTAs per SM, at least one 64-column chunk
   // per warp, clusters of at most 8
   const int tiles = (M + 15) / 16;
-  const int steps = (C + 15) / 16;
+  const int chunks = (C + 63) / 64;
   int KS = (2 * sm_count(current_device()) + tiles - 1) / tiles;
   KS = KS > 8 ? 8 : KS;
-  while (KS > 1 && steps / KS < 2 * ad::kWarps) --KS;
+  while (KS > 1 && chunks / KS < ad::kWarps) --KS;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles, KS, 1);
   cfg.blockDim = dim3(ad::kThreads, 1, 1);
@@ -166,8 +202,11 @@ cudaError_t launch_adapter_proj(const uint16_t* act, const uint16_t* proj, bool 
   const __half* a = reinterpret_cast<const __half*>(act);
   const __half* p = reinterpret_cast<const __half*>(proj);
   __half* o = static_cast<__half*>(workspace);
-  return by_rows ? cudaLaunchKernelEx(&cfg, ad::q4gsw_adapter_proj_kernel<true>, a, p, o, M, C, r)
-                 : cudaLaunchKernelEx(&cfg, ad::q4gsw_adapter_proj_kernel<false>, a, p, o, M, C, r);
+  const int nj = (r + 7) / 8;
+#define Q4_PROJ(BR, NJ_) cudaLaunchKernelEx(&cfg, ad::q4gsw_adapter_proj_kernel<BR, NJ_>, a, p, o, M, C, r)
+  if (by_rows) return nj <= 2 ? Q4_PROJ(true, 2) : nj <= 4 ? Q4_PROJ(true, 4) : Q4_PROJ(true, 8);
+  return nj <= 2 ? Q4_PROJ(false, 2) : nj <= 4 ? Q4_PROJ(false, 4) : Q4_PROJ(false, 8);
+#undef Q4_PROJ
 }
 
 }  // namespace q4gsw
