@@ -195,7 +195,7 @@ def test_empty_batch_leaves_outputs_untouched():
     assert m.q4gsw_last_route() == "empty"
 
 
-@pytest.mark.parametrize("M", [1, 2, 7, 8, 9, 15, 16, 17, 33, 127, 129])
+@pytest.mark.parametrize("M", [1, 2, 7, 8, 9, 15, 16, 17, 33, 127, 129, 511, 512, 513])
 def test_ragged_token_counts(M):
     inp = wl.random_inputs(M, 72, 192, 64, seed=100 + M)
     check_fwd(inp, 64)
@@ -281,6 +281,19 @@ def test_gemm_route_tails(M, N, K, gs, gemm_variant):
     check_bwd(inp, gs)
     route = q().q4gsw_last_route()
     assert _route_ok(route, "bwd", gemm_variant), route
+
+
+@pytest.mark.parametrize("M,route", [(16, "gemv_tma"), (17, "tcgen05_ts_gemm"), (512, "tcgen05_ts_gemm"),
+                                     (513, "tcgen05_gemm")])
+def test_one_group_over_all_of_k_at_every_route_boundary(M, route):
+    # gs == K: a single scale group per output feature; each side of the
+    # GEMV / tensor-memory GEMM / shared-memory GEMM switches
+    q().q4gsw_debug_pin_routes()
+    inp = wl.random_inputs(M, 136, 512, 512, seed=M + 1)
+    check_fwd(inp, 512)
+    assert q().q4gsw_last_route().startswith(route + "_fwd"), q().q4gsw_last_route()
+    check_bwd(inp, 512)
+    assert q().q4gsw_last_route().startswith(route + "_bwd"), q().q4gsw_last_route()
 
 
 def test_gemm_default_routes():
