@@ -64,15 +64,29 @@ __device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A * B (the first MMA of a group: no accumulator to clear)
+__device__ __forceinline__ void mma_s8_zero(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
+
 // 16 (c - 8) as signed bytes from the nibble pairs of one code word: the low
 // nibbles (even row) and the high nibbles (odd row); c << 4 ^ 0x80 = 16 (c - 8).
 __device__ __forceinline__ uint32_t even16(uint32_t w) { return ((w << 4) & 0xF0F0F0F0u) ^ 0x80808080u; }
 __device__ __forceinline__ uint32_t odd16(uint32_t w) { return (w & 0xF0F0F0F0u) ^ 0x80808080u; }
 
+// ONES (at most 7 tokens, NT = 1): B column 7 is a spare token column (its q
+// row is zero-filled), so lanes g = 7 put ones there and column 7 of the
+// product MMA gives C = sum 16 (c - 8) of each row: no separate ones-MMA.
 // grid = (ceil(N / 64) row blocks, S contraction splits (one cluster), ceil(M / 16)).
 // q: int8 [M][K] in the codes' order (inside each 64-column block, the 16 bytes
 // at 16 t hold columns 4 t + 16 i + (0, 2, 1, 3), i = 0..3); a_s fp32 [M]; a_z int32 [M].
-template <int NT>
+// GM: where groups start, fixed at compile time where gs allows it:
+//   0 (gs 32): every 32-column step is a group;  1 (gs 64, 128): every block of
+//   the warp (its two steps) lies in one group;  2 (gs >= 256): a group spans
+//   blocks of several stages (tracked at run time).
+template <int NT, bool ONES, int GM>
 __global__ void __launch_bounds__(Cfg<NT>::THREADS, Cfg<NT>::MINB)
 q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
                             const __grid_constant__ CUtensorMap map_q, const float* __restrict__ a_s,
@@ -189,22 +203,16 @@ q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __
     for (int h = 0; h < 2; ++h)
       sc_off[h] = C::OFF_SC + (uint32_t)(gs < SK ? ((64 * w + 32 * h) >> gsl) : 0) * 64 * 2 + 4 * pair_of(rt0, g);
 
+    static_assert(!ONES || NT == 1, "the spare column exists for up to 7 tokens");
     int pq[RTW][NT][4], pc[RTW][4];
-    auto zero_parts = [&] {
-#pragma unroll
-      for (int rt = 0; rt < RTW; ++rt) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) pc[rt][c] = 0;
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) pq[rt][j][c] = 0;
-      }
-    };
-    zero_parts();
+    bool gstart = true;   // no MMA since the last flush: the next one starts a group
     auto flush = [&](const uint32_t (&sw)[RTW]) {
 #pragma unroll
       for (int rt = 0; rt < RTW; ++rt) {
+        if (ONES) {   // C of row g (even) and g + 8 (odd) from lane (g, 3), D column 7
+          pc[rt][0] = pc[rt][1] = __shfl_sync(0xffffffffu, pq[rt][0][1], (g << 2) | 3);
+          pc[rt][2] = pc[rt][3] = __shfl_sync(0xffffffffu, pq[rt][0][3], (g << 2) | 3);
+        }
         const float2 sp = __half22float2(*reinterpret_cast<const __half2*>(&sw[rt]));
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
@@ -215,7 +223,7 @@ q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __
           acc[rt][j][3] = fmaf((float)((pq[rt][j][3] - az1[j] * pc[rt][3]) >> 4), sp.y, acc[rt][j][3]);
         }
       }
-      zero_parts();
+      gstart = true;
     };
     constexpr uint32_t kOnes = 0x01010101u;
     auto stage = [&](int it) -> bool {
@@ -225,6 +233,7 @@ q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __
       uint4 qv[NT];
 #pragma unroll
       for (int j = 0; j < NT; ++j) qv[j] = lds128(st + q_off[j]);
+      if (ONES && g == 7) qv[0] = make_uint4(kOnes, kOnes, kOnes, kOnes);
       uint4 wv[RTW];
       uint32_t sw[2][RTW];
 #pragma unroll
@@ -250,19 +259,37 @@ q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __
 #pragma unroll
       for (int h = 0; h < 2; ++h) {   // 32-column steps: code words 2h, 2h + 1; q words likewise
 #pragma unroll
-        for (int rt = 0; rt < RTW && in; ++rt) {
-          const uint32_t w0 = h == 0 ? wv[rt].x : wv[rt].z, w1 = h == 0 ? wv[rt].y : wv[rt].w;
-          const uint32_t a[4] = {even16(w0), odd16(w0), even16(w1), odd16(w1)};
-          mma_s8(pc[rt], a, kOnes, kOnes);
+        if (in) {
 #pragma unroll
-          for (int j = 0; j < NT; ++j)
-            mma_s8(pq[rt][j], a, h == 0 ? qv[j].x : qv[j].z, h == 0 ? qv[j].y : qv[j].w);
+          for (int rt = 0; rt < RTW; ++rt) {
+            const uint32_t w0 = h == 0 ? wv[rt].x : wv[rt].z, w1 = h == 0 ? wv[rt].y : wv[rt].w;
+            const uint32_t a[4] = {even16(w0), odd16(w0), even16(w1), odd16(w1)};
+            // the first MMA of a group takes a zero accumulator
+            const bool zero = GM == 0 ? true : GM == 1 ? h == 0 : gstart;
+            if (!ONES) {
+              if (zero) mma_s8_zero(pc[rt], a, kOnes, kOnes);
+              else mma_s8(pc[rt], a, kOnes, kOnes);
+            }
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+              const uint32_t b0 = h == 0 ? qv[j].x : qv[j].z, b1 = h == 0 ? qv[j].y : qv[j].w;
+              if (zero) mma_s8_zero(pq[rt][j], a, b0, b1);
+              else mma_s8(pq[rt][j], a, b0, b1);
+            }
+          }
+          gstart = false;
         }
-        // a group ends with this step: gs == 32 at every step, else at the
-        // warp's block end when its next block (256 columns on) starts another
-        // group, or the split ends
-        if (gs == 32) flush(sw[h]);
-        else if (h == 1 && (((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1)) flush(sw[0]);
+        // a group ends with this step: at every step (GM 0), at the block end
+        // (GM 1), else when the warp's next block (256 columns on) starts
+        // another group or the split ends; blocks past K took no MMA and add
+        // nothing (they come last, after the warp's final flush, for GM 0 and 1)
+        if (GM == 0) {
+          if (in) flush(sw[h]);
+        } else if (GM == 1) {
+          if (in && h == 1) flush(sw[0]);
+        } else if (h == 1 && !gstart && (((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1)) {
+          flush(sw[0]);
+        }
       }
       return true;
     };
@@ -319,12 +346,12 @@ q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __
 
 }  // namespace dqt
 
-template <int NT>
+template <int NT, bool ONES, int GM>
 static cudaError_t launch_dq8ca_variant(const CUtensorMap& map_pk, const CUtensorMap& map_sc, const CUtensorMap& map_q,
                                         const float* a_s, const int* a_z, OutSplit out, int M, int N, int K, int gs,
                                         int stages_total, dim3 grid, cudaStream_t stream) {
   using C = dqt::Cfg<NT>;
-  auto kern = dqt::q4gsw_dq8ca_gemv_tma_kernel<NT>;
+  auto kern = dqt::q4gsw_dq8ca_gemv_tma_kernel<NT, ONES, GM>;
   static PerDeviceOnce attr_once;
   {
     cudaError_t e = once_per_device(attr_once, current_device(), [&] {
@@ -376,12 +403,19 @@ cudaError_t launch_dq8ca_gemv(const void* packed, int N, int K, int gs, int M, c
   const float* a_s = reinterpret_cast<const float*>(ws + dq8ca_scale_offset(M, K));
   const int* a_z = reinterpret_cast<const int*>(ws + dq8ca_zero_offset(M, K));
   const dim3 grid(tiles, S, zs);
-  const cudaError_t e =
-      NT == 1 ? launch_dq8ca_variant<1>(map_pk, map_sc, map_q, a_s, a_z, out, M, N, K, gs, stages_total, grid, stream)
-              : launch_dq8ca_variant<2>(map_pk, map_sc, map_q, a_s, a_z, out, M, N, K, gs, stages_total, grid, stream);
+  const int gm = gs == 32 ? 0 : gs < gv::SK ? 1 : 2;
+#define Q4_DQ(NT_, ONES_)                                                                                          \
+  (gm == 0   ? launch_dq8ca_variant<NT_, ONES_, 0>(map_pk, map_sc, map_q, a_s, a_z, out, M, N, K, gs, stages_total, \
+                                                   grid, stream)                                                   \
+   : gm == 1 ? launch_dq8ca_variant<NT_, ONES_, 1>(map_pk, map_sc, map_q, a_s, a_z, out, M, N, K, gs, stages_total, \
+                                                   grid, stream)                                                   \
+             : launch_dq8ca_variant<NT_, ONES_, 2>(map_pk, map_sc, map_q, a_s, a_z, out, M, N, K, gs, stages_total, \
+                                                   grid, stream))
+  const cudaError_t e = NT == 2 ? Q4_DQ(2, false) : M <= 7 ? Q4_DQ(1, true) : Q4_DQ(1, false);
+#undef Q4_DQ
   if (route)
-    snprintf(route, route_len, "int8_gemv_tma nt=%d tiles=%d splits=%d zslices=%d stages=%d", NT, tiles, S, zs,
-             NT == 1 ? dqt::Cfg<1>::ST : dqt::Cfg<2>::ST);
+    snprintf(route, route_len, "int8_gemv_tma nt=%d tiles=%d splits=%d zslices=%d stages=%d%s", NT, tiles, S, zs,
+             NT == 1 ? dqt::Cfg<1>::ST : dqt::Cfg<2>::ST, NT == 1 && M <= 7 ? " ones_column=7" : "");
   return e;
 }
 
