@@ -102,7 +102,8 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 
 // grid = (ceil(N / 64) row tiles, S contraction splits, ceil(M / 16) token
 // slices), cluster = (1, S, 1).  SPG = 16-column steps per scale group
-// (1: gs 16, 2: gs 32, 4: gs >= 64).
+// (1: gs 16, 2: gs 32, 4: gs 64 or 128, where a warp's 64-column block is one
+// group; 8: gs >= 256, where a group spans the warp's blocks of several stages).
 template <int NT, int SPG, bool F32S, bool XS>
 __global__ void __launch_bounds__(FwdCfg<NT, SPG, F32S, XS>::THREADS, FwdCfg<NT, SPG, F32S, XS>::MINB)
 q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __grid_constant__ CUtensorMap map_sc,
@@ -111,7 +112,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
   using namespace sm100;
   using C = FwdCfg<NT, SPG, F32S, XS>;
   constexpr int RTW = C::RTW;
-  constexpr int NGB = SPG == 4 ? 1 : 4 / SPG;   // scale groups per 64-column block
+  constexpr int NGB = SPG >= 4 ? 1 : 4 / SPG;   // scale groups per 64-column block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
@@ -237,7 +238,7 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
     uint32_t sc_off[NGB];
 #pragma unroll
     for (int q = 0; q < NGB; ++q) {
-      const int col = 64 * w + (SPG == 4 ? 0 : 16 * SPG * q);
+      const int col = 64 * w + (SPG >= 4 ? 0 : 16 * SPG * q);
       sc_off[q] = C::OFF_SC + (uint32_t)(gs < SK ? (col >> gsl) : 0) * 64 * C::SB + 2 * C::SB * pair_of(rt0, g);
     }
 
@@ -300,7 +301,9 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
       };
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const bool first = SPG == 4 ? (i == 0 && fresh) : (i % SPG == 0);
+        // the first MMA of a group starts from a zero accumulator; where the
+        // groups start is fixed at compile time except for groups over stages
+        const bool first = SPG == 8 ? (i == 0 && fresh) : SPG == 4 ? i == 0 : (i % SPG == 0);
 #pragma unroll
         for (int rt = 0; rt < RTW; ++rt) {
           const uint32_t word = i == 0 ? wv[rt].x : i == 1 ? wv[rt].y : i == 2 ? wv[rt].z : wv[rt].w;
@@ -315,7 +318,8 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         }
         if (SPG < 4 && (i % SPG) == SPG - 1) flush(i / SPG);
       }
-      if (SPG == 4) {
+      if (SPG == 4) flush(0);   // the block is one group (gs 64 or 128)
+      if (SPG == 8) {
         // this warp's block of the next stage starts another group, or the split ends here
         const int k0 = (st_begin + it) * SK + 64 * w;
         fresh = ((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1;
@@ -668,7 +672,7 @@ cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f
   const int zs = (M + 15) / 16;
   const int tiles = (N + 63) / 64;
   const int stages_total = (K + gv::SK - 1) / gv::SK;
-  const int spg = gs == 16 ? 1 : gs == 32 ? 2 : 4;
+  const int spg = gs == 16 ? 1 : gs == 32 ? 2 : gs < gv::SK ? 4 : 8;
   // Contraction splits: as many CTAs as the SMs hold at once (each CTA's
   // stages are consumed at a bounded rate, so the stream needs many of them),
   // at least two stages per split, clusters of at most 8.
@@ -704,9 +708,9 @@ cudaError_t launch_gemv_tma_fwd(const void* packed, int N, int K, int gs, bool f
                                                          stages_total, grid, stream))
 #define Q4_TMA_FWD(NT_, SPG_) (xs ? Q4_TMA_FWD_X(NT_, SPG_, true) : Q4_TMA_FWD_X(NT_, SPG_, false))
   if (NT == 1)
-    e = spg == 1 ? Q4_TMA_FWD(1, 1) : spg == 2 ? Q4_TMA_FWD(1, 2) : Q4_TMA_FWD(1, 4);
+    e = spg == 1 ? Q4_TMA_FWD(1, 1) : spg == 2 ? Q4_TMA_FWD(1, 2) : spg == 4 ? Q4_TMA_FWD(1, 4) : Q4_TMA_FWD(1, 8);
   else
-    e = spg == 1 ? Q4_TMA_FWD(2, 1) : spg == 2 ? Q4_TMA_FWD(2, 2) : Q4_TMA_FWD(2, 4);
+    e = spg == 1 ? Q4_TMA_FWD(2, 1) : spg == 2 ? Q4_TMA_FWD(2, 2) : spg == 4 ? Q4_TMA_FWD(2, 4) : Q4_TMA_FWD(2, 8);
 #undef Q4_TMA_FWD
 #undef Q4_TMA_FWD_X
   if (route)
