@@ -49,7 +49,7 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
 # dram__bytes_write.sum), with the hash of the kernel sources they were taken
 # on: reported only while the sources still match, null otherwise.
-NCU_TRAFFIC = {"sources_sha": "ed63c1fc9c001ed9", "bytes_per_launch": {'up_fwd': 11561472, 'up_bwd': 17852672, 'down_fwd': 17852928, 'down_bwd': 11561216, 'qkv_fwd': 5662976}}
+NCU_TRAFFIC = {"sources_sha": "64442abd1e55e568", "bytes_per_launch": {'qkv_fwd': 5668000, 'up_fwd': 11566000, 'down_fwd': 17858000, 'down_bwd': 11568000, 'up_bwd': 17859000}}
 
 
 def sources_sha() -> str:
