@@ -47,15 +47,19 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
             "+ down and up input grads; M=512 tokens, group_size 32")
 
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
-# dram__bytes_write.sum), with the hash of the kernel sources they were taken
-# on: reported only while the sources still match, null otherwise.
-NCU_TRAFFIC = {"sources_sha": "64442abd1e55e568", "bytes_per_launch": {'qkv_fwd': 5668000, 'up_fwd': 11566000, 'down_fwd': 17858000, 'down_bwd': 11568000, 'up_bwd': 17859000}}
+# dram__bytes_write.sum), with the hash of the tensor-memory GEMM's sources they
+# were taken on: reported only while those sources still match, null otherwise.
+NCU_TRAFFIC = {"sources_sha": "5657920991ed5f96", "bytes_per_launch": {'qkv_fwd': 5668000, 'up_fwd': 11566000, 'down_fwd': 17858000, 'down_bwd': 11568000, 'up_bwd': 17859000}}
+
+
+# the files the tensor-memory GEMM (every op of the step) is built from
+TS_SOURCES = ("q4gsw_gemm_ts.cuh", "q4gsw_sm100.cuh", "q4gsw_common.cuh", "q4gsw_internal.h")
 
 
 def sources_sha() -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "bit_group_quantized_q4gsw_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in TS_SOURCES:
+        h.update(open(os.path.join(ROOT, "bit_group_quantized_q4gsw_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 

@@ -31,18 +31,25 @@ __host__ __device__ inline size_t off_as(int M, int K) { return round_up((size_t
 __host__ __device__ inline size_t off_az(int M, int K) { return off_as(M, K) + round_up((size_t)4 * M, 256); }
 __host__ __device__ inline size_t ws_bytes(int M, int K) { return off_az(M, K) + round_up((size_t)4 * M, 256); }
 
-// q of one value, the fp32 steps of the reading
-__device__ __forceinline__ uint32_t quant_byte(float v, float as, int az) {
-  int qv = (int)rintf(__fdiv_rn(v, as)) + az;
+// q of one value: rint of the correctly rounded quotient v / a_s, plus a_z,
+// clamped.  The quotient is taken as v times the rounded reciprocal inv of a_s;
+// for |v / a_s| <= 256 that product lies within 2^-14 of the correctly rounded
+// quotient (three roundings of at most 2^-24 relative each), so wherever it
+// is farther than 1e-4 from a half-integer both round to the same integer, and
+// only near a tie is the quotient divided out exactly.
+__device__ __forceinline__ uint32_t quant_byte(float v, float as, float inv, int az) {
+  float r = v * inv;
+  if (fabsf(fabsf(r - rintf(r)) - 0.5f) < 1e-4f) r = __fdiv_rn(v, as);
+  int qv = (int)rintf(r) + az;
   qv = qv < -128 ? -128 : qv > 127 ? 127 : qv;
   return (uint32_t)(qv & 0xFF);
 }
 
 // four consecutive values -> one word in the packed codes' byte order (+0, +2, +1, +3)
-__device__ __forceinline__ uint32_t quant_word(__half2 a, __half2 b, float as, int az) {
+__device__ __forceinline__ uint32_t quant_word(__half2 a, __half2 b, float as, float inv, int az) {
   const float2 fa = __half22float2(a), fb = __half22float2(b);
-  return quant_byte(fa.x, as, az) | quant_byte(fb.x, as, az) << 8 | quant_byte(fa.y, as, az) << 16 |
-         quant_byte(fb.y, as, az) << 24;
+  return quant_byte(fa.x, as, inv, az) | quant_byte(fb.x, as, inv, az) << 8 | quant_byte(fa.y, as, inv, az) << 16 |
+         quant_byte(fb.y, as, inv, az) << 24;
 }
 
 __device__ __forceinline__ void range_of(const uint4& v, float& lo, float& hi) {
@@ -57,11 +64,11 @@ __device__ __forceinline__ void range_of(const uint4& v, float& lo, float& hi) {
 
 // columns 8 i .. 8 i + 7 of the row -> their q bytes: block i / 8, 16-column
 // step (i % 8) / 2, lanes t = 2 (i % 2) and 2 (i % 2) + 1 of that step
-__device__ __forceinline__ void store_q(uint8_t* qrow, int i, const uint4& v, float as, int az) {
+__device__ __forceinline__ void store_q(uint8_t* qrow, int i, const uint4& v, float as, float inv, int az) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
   uint8_t* dst = qrow + 64 * (i >> 3) + 32 * (i & 1) + 4 * ((i & 7) >> 1);
-  *reinterpret_cast<uint32_t*>(dst) = quant_word(h[0], h[1], as, az);
-  *reinterpret_cast<uint32_t*>(dst + 16) = quant_word(h[2], h[3], as, az);
+  *reinterpret_cast<uint32_t*>(dst) = quant_word(h[0], h[1], as, inv, az);
+  *reinterpret_cast<uint32_t*>(dst + 16) = quant_word(h[2], h[3], as, inv, az);
 }
 
 // One CTA per token: the row's 16-byte vectors stay in registers between the
@@ -69,7 +76,7 @@ __device__ __forceinline__ void store_q(uint8_t* qrow, int i, const uint4& v, fl
 __global__ void __launch_bounds__(kQThreads)
 q4gsw_dq8ca_quantize_kernel(const __half* __restrict__ x, uint8_t* __restrict__ ws, int M, int K) {
   __shared__ float s_lo[kQThreads / 32], s_hi[kQThreads / 32];
-  __shared__ float s_as;
+  __shared__ float s_as, s_inv;
   __shared__ int s_az;
   griddep_launch_dependents();
   griddep_wait();   // x may come from the previous kernel of the stream
@@ -109,21 +116,22 @@ q4gsw_dq8ca_quantize_kernel(const __half* __restrict__ x, uint8_t* __restrict__ 
       float z = rintf(__fsub_rn(-128.f, __fdiv_rn(lo, as)));
       z = fminf(127.f, fmaxf(-128.f, z));
       s_as = as;
+      s_inv = __fdiv_rn(1.f, as);
       s_az = (int)z;
       reinterpret_cast<float*>(ws + off_as(M, K))[m] = as;
       reinterpret_cast<int*>(ws + off_az(M, K))[m] = (int)z;
     }
   }
   __syncthreads();
-  const float as = s_as;
+  const float as = s_as, inv = s_inv;
   const int az = s_az;
   uint8_t* qrow = ws + (size_t)m * K;
 #pragma unroll
   for (int u = 0; u < kQVec; ++u) {
     const int i = threadIdx.x + u * kQThreads;
-    if (i < V) store_q(qrow, i, v[u], as, az);
+    if (i < V) store_q(qrow, i, v[u], as, inv, az);
   }
-  for (int i = threadIdx.x + kQVec * kQThreads; i < V; i += kQThreads) store_q(qrow, i, row[i], as, az);
+  for (int i = threadIdx.x + kQVec * kQThreads; i < V; i += kQThreads) store_q(qrow, i, row[i], as, inv, az);
 }
 
 }  // namespace dq
