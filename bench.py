@@ -49,7 +49,7 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
 # dram__bytes_write.sum), with the hash of the tensor-memory GEMM's sources they
 # were taken on: reported only while those sources still match, null otherwise.
-NCU_TRAFFIC = {"sources_sha": "5657920991ed5f96", "bytes_per_launch": {'qkv_fwd': 5668000, 'up_fwd': 11566000, 'down_fwd': 17858000, 'down_bwd': 11568000, 'up_bwd': 17859000}}
+NCU_TRAFFIC = {"sources_sha": "434cb93ceaf6c46b", "bytes_per_launch": {'qkv_fwd': 5668000, 'up_fwd': 11566000, 'down_fwd': 17858000, 'down_bwd': 11567000, 'up_bwd': 17859000}}
 
 
 # the files the tensor-memory GEMM (every op of the step) is built from

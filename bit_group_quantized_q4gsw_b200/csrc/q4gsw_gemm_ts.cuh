@@ -70,7 +70,7 @@ struct Args {
   int stages_total;
   int sc_bytes;       // bytes of the scale box of one stage
   int bt;             // tokens per tile
-  int tma_out;        // outputs written by tensor store / reduce-add (map_y*), else by threads
+  int tma_out;        // outputs written by one tensor store (map_y*; no split-K), else by threads
   // Low-rank adapter stage (ad_r > 0): one more 64-deep stage of the last
   // split whose weight operand is the adapter matrix (forward: rows of B
   // [N, r]; backward: columns of A [r, K]; leading dimension ad_ld) and whose
@@ -374,39 +374,16 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     }
   }
   if (args.tma_out) {
-    // Tensor store of the [bt][128] fp32 tile (rows past M and features past
-    // the output clipped by the map).  With split-K, rank 0 stores its partial
-    // and, once that store has completed, the other ranks add theirs at L2
-    // (tensor reduce-add), so no CTA reads another's shared memory and each
-    // leaves as soon as its tile has been read out of shared memory.  The
-    // order of the S-1 additions is not fixed.
+    // One CTA per tile (no split-K): one tensor store of the [bt][128] fp32
+    // tile (rows past M and features past the output clipped by the map).
     const CUtensorMap* my = f0 < o.n1 ? &map_y0 : (f0 < o.n2 ? &map_y1 : &map_y2);
     const int c0 = f0 < o.n1 ? f0 : (f0 < o.n2 ? f0 - o.n1 : f0 - o.n2);
     fence_proxy_async_smem();
     __syncthreads();
-    const bool ok = !*abort_flag;
-    if (S == 1) {
-      if (threadIdx.x == 0 && ok) {
-        tma_store_2d(my, stage_f32, c0, t0);
-        bulk_commit();
-        bulk_wait_read_all();
-      }
-    } else {
-      cg::cluster_group cluster = cg::this_cluster();
-      const int rk = (int)cluster.block_rank();
-      if (rk == 0 && threadIdx.x == 0 && ok) {
-        tma_store_2d(my, stage_f32, c0, t0);
-        bulk_commit();
-        bulk_wait_all();
-        fence_proxy_async_global();
-      }
-      cluster.sync();   // every thread of every CTA of the cluster, aborted or not
-      if (rk != 0 && threadIdx.x == 0 && ok) {
-        fence_proxy_async_global();
-        tma_reduce_add_2d(my, stage_f32, c0, t0);
-        bulk_commit();
-        bulk_wait_read_all();
-      }
+    if (threadIdx.x == 0 && !*abort_flag) {
+      tma_store_2d(my, stage_f32, c0, t0);
+      bulk_commit();
+      bulk_wait_read_all();
     }
   } else {
     // Copy-out: one warp writes 512 contiguous bytes (128 features of one
