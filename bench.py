@@ -394,10 +394,10 @@ def run_gpu(args, rank, world, local_rank):
     # ---- device-resident timed region
     # Consecutive launches overlap (programmatic dependent launch); an event
     # between two launches removes that overlap.  So per-operation events are
-    # recorded on every 8th step only (the sampled steps); the other steps run
-    # back to back.  ms_per_step covers all K steps.
+    # recorded on every 25th step only (the sampled steps, 8 of the default
+    # 200); the other steps run back to back.  ms_per_step covers all K steps.
     nops = len(ops)
-    SAMPLE = 8
+    SAMPLE = 25
     sampled = [i for i in range(args.steps) if i % SAMPLE == SAMPLE - 1] or [args.steps - 1]
     ev = {i: [torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for i in sampled}
     for i in range(args.warmup):
