@@ -334,3 +334,25 @@ def test_gemm_split_k_cluster_reduction(gemm_variant):
 
 def test_no_kernel_wait_ran_out():
     q().q4gsw_device_error_check()
+
+
+@pytest.mark.parametrize("M,N,K,gs,f32", [(1, 64, 64, 32, 0), (3, 264, 448, 16, 0), (8, 4096, 1024, 32, 0),
+                                          (9, 1032, 2048, 128, 0), (16, 512, 4096, 256, 0), (16, 14336, 4096, 128, 0),
+                                          (5, 520, 1088, 64, 1), (13, 2048, 2048, 16, 1)])
+def test_staged_and_global_activations_agree_bit_for_bit(M, N, K, gs, f32):
+    # the forward TMA ring takes its activation fragments from the stage (pin
+    # "tma_xs") or from global memory (pin "tma"); the MMAs are the same, so
+    # the outputs are identical
+    inp = wl.random_inputs(M, N, K, gs, seed=M + N)
+    scales = inp.scales.astype(np.float32) if f32 else inp.scales
+    blob = q().q4gsw_prepack(cuda(inp.codes), cuda(scales), gs)
+    outs = []
+    try:
+        for pin in ("tma", "tma_xs"):
+            q().q4gsw_debug_pin_routes(gemv=pin)
+            outs.append(q().q4gsw_linear_fwd(blob, N, K, gs, cuda(inp.x), f32s=bool(f32)).cpu())
+            assert ("x=staged" in q().q4gsw_last_route()) == (pin == "tma_xs")
+    finally:
+        q().q4gsw_debug_pin_routes()
+    q().q4gsw_device_error_check()
+    assert torch.equal(outs[0], outs[1])
