@@ -564,8 +564,18 @@ def time_shape(q, sh, kind, device, flush, peaks):
     """One operation of one configuration shape: mean time per launch over a
     CUDA graph of back-to-back launches whose packed weights rotate through
     copies totalling > 3x the L2, plus one launch timed alone after an L2 flush.
-    Returns the JSON record with both rooflines."""
+    Returns the JSON record with both rooflines.  A kind "fwd@ts" / "fwd@ss"
+    pins the tensor-core GEMM route (tensor-memory or shared-memory tile)."""
     import torch
+    if "@" in kind:
+        kind, pin = kind.split("@")
+        q.q4gsw_debug_pin_routes(gemm=pin)
+        try:
+            rec = time_shape(q, sh, kind, device, flush, peaks)
+        finally:
+            q.q4gsw_debug_pin_routes()
+        rec["dir"] = f"{kind}@{pin}"
+        return rec
     inp = wl.make_inputs(sh)
     codes = torch.from_numpy(inp.codes).to(device)
     scales = torch.from_numpy(inp.scales).to(device)
@@ -662,7 +672,9 @@ def time_shape(q, sh, kind, device, flush, peaks):
 # metric (decode M=1; the sweep's M=1 and M=16 on both 8B-class matrices) and
 # the largest compute-bound shapes (the sweep's M=4096); the adapter and the
 # int8-activation product (dq8ca: algorithmic bytes as the fp16 forward, the
-# quantised copy of x in the workspace counts as overhead).
+# quantised copy of x in the workspace counts as overhead); and at M=512 the
+# two tensor-core GEMM routes side by side (dequantised tile in tensor memory,
+# the default up to 512 tokens, or in shared memory).
 SHAPE_LEGS = [("decode_N2048_K2048", "fwd"), ("decode_N8192_K2048", "fwd"), ("decode_N2048_K8192", "fwd"),
               ("sweep_M1_N14336_K4096", "fwd"), ("sweep_M1_N14336_K4096", "bwd"),
               ("sweep_M1_N4096_K14336", "fwd"), ("sweep_M1_N4096_K14336", "bwd"),
@@ -673,7 +685,8 @@ SHAPE_LEGS = [("decode_N2048_K2048", "fwd"), ("decode_N8192_K2048", "fwd"), ("de
               ("adapter_up_M512", "ad_fwd"), ("adapter_up_M512", "ad_bwd"),
               ("adapter_down_M512", "ad_fwd"), ("adapter_down_M512", "ad_bwd"),
               ("decode_N8192_K2048", "dq8ca"), ("sweep_M1_N4096_K14336", "dq8ca"),
-              ("sweep_M16_N14336_K4096", "dq8ca")]
+              ("sweep_M16_N14336_K4096", "dq8ca"),
+              ("adapter_up_M512", "fwd@ts"), ("adapter_up_M512", "fwd@ss")]
 
 
 def shape_legs(device, peaks, world):
