@@ -16,8 +16,10 @@
  *        weights and scales, scattered into three distinct outputs; outside the
  *        accepted shapes the ordinary routes run.
  *   [P1] "Upstream the Gemma 4 Vulkan support we carry on our ExecuTorch fork",
- *        software-mansion/react-native-executorch issue #1361, comment of
- *        Oct 20, 2026: fp16 weight scales.
+ *        software-mansion/react-native-executorch issue #1361: the fork's
+ *        shader list (linear_q4gsw, linear_dq8ca_q4gsw,
+ *        linear_fp32_scale_dq_acc, embedding_q4gsw) and the comment of Oct 20,
+ *        2026: fp16 weight scales.
  *
  * Notation: M tokens, K input features, N output features, gs = group_size,
  * G = K / gs.  code[n,k] in 0..15, scale[g,n] fp16,
@@ -26,7 +28,9 @@
  * Conventions for every entry point
  *   - Every pointer argument is a DEVICE pointer on the current CUDA device,
  *     except where stated.  The caller allocates and owns every buffer; the
- *     library allocates no device memory.  Its state: per host thread, the
+ *     library allocates no device memory when called (its one fixed array, the
+ *     1 MiB of q4gsw_adapter_fwd_noalloc, is part of its device image).  Its
+ *     state: per host thread, the
  *     route string (q4gsw_last_route) and the debug route pins
  *     (q4gsw_debug_pin_routes); per device, one status word shared by every
  *     stream and thread (see q4gsw_device_error_check) and caches of kernel
@@ -40,7 +44,9 @@
  *     error nothing is enqueued and outputs are untouched.  A launch failure
  *     reported by the CUDA runtime returns Q4GSW_ERR_CUDA.
  *   - No CPU fallback exists: every result is computed by this library's
- *     CUDA kernels.  Calls may be made from several host threads at once
+ *     CUDA kernels.  Results are deterministic: every reduction (warp slices,
+ *     split-K CTAs of a cluster) runs in a fixed order, so a call repeated on
+ *     the same inputs and route returns the same bits.  Calls may be made from several host threads at once
  *     (first-use caches are filled under std::call_once or atomics).
  *   - The compute calls launch with programmatic dependent launch: a call may
  *     start while the previous kernel on `stream` is still finishing.  It waits
