@@ -258,7 +258,6 @@ q4gsw_dq8ca_gemv_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __
       const bool in = k0 < K;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {   // 32-column steps: code words 2h, 2h + 1; q words likewise
-#pragma unroll
         if (in) {
 #pragma unroll
           for (int rt = 0; rt < RTW; ++rt) {

@@ -25,9 +25,9 @@
 //   warp 1       allocates tensor memory (fp32 accumulator in columns 0..255,
 //                a ring of WST dequantised stages of 32 columns after it) and
 //                issues tcgen05.mma from one thread;
-//   warps 2..17  warp w writes TMEM lanes 32 (w % 4) .. +31 (weight rows) and
-//                the 16-deep contraction slice (w - 2) / 4 of every stage, then
-//                runs the epilogue for the same lanes.
+//   warps 2..17  warp w writes TMEM lanes 32 (w % 4) .. +31 (weight rows) of
+//                every fourth stage (stages (w - 2) / 4 + 4 i, TMEM slot
+//                (w - 2) / 4), then runs the epilogue for the same lanes.
 // Every consumer waits on every phase of the barriers it uses.
 #pragma once
 
@@ -83,7 +83,7 @@ struct Args {
 struct Ctl {
   uint64_t full[8];       // stage s loaded (TMA transaction bytes)
   uint64_t consumed[8];   // the MMAs of the stage in slot s completed (one commit per stage)
-  uint64_t wready[WST];   // dequantised stage in TMEM slot w written (all dequantisation warps)
+  uint64_t wready[WST];   // dequantised stage in TMEM slot w written (one warp per lane quadrant)
   uint64_t accfull;
   uint64_t drain;
   uint32_t tmem_base;
@@ -113,6 +113,60 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
 __device__ __forceinline__ uint32_t nibbles_minus8(uint32_t v) {
   const __half2 kSub = u32_as_h2(0x64086408u);   // 1032, 1032
   return h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(v, 0x000F000Fu, 0x64006400u)), kSub));
+}
+
+// Rows [row_b, row_e) of the tile, summed over the S partial tiles parked in
+// the shared memory of the cluster's CTAs (ranks 0 .. S-1, added in rank
+// order), written as float4 to the output.  Each thread first issues the
+// loads of up to kPer items (S loads each, most of them remote), then adds
+// and stores: the reads of distributed shared memory are latency-bound, and
+// one item at a time left ~4 of those latencies in a row per thread.
+template <int S>
+__device__ __forceinline__ void copy_out(const float* stage_f32, int row_b, int row_e, int t0, int f0,
+                                         const Args& args) {
+  using namespace sm100;
+  constexpr int kPer = S == 1 ? 8 : (12 / S > 0 ? 12 / S : 1);   // at most 12 float4 in flight
+  const OutSplit& o = args.out;
+  uint32_t src[S];   // the staging tile of every rank, in the cluster's shared window
+#pragma unroll
+  for (int qq = 0; qq < S; ++qq) src[qq] = S == 1 ? smem_u32(stage_f32) : mapa_u32(smem_u32(stage_f32), qq);
+  const int total = (row_e - row_b) * (BW / 4);
+  for (int base = threadIdx.x; base < total; base += kThreads * kPer) {
+    float4 part[kPer][S];
+    bool ok[kPer];
+    int offs[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = base + u * kThreads;
+      const int row = row_b + idx / (BW / 4), c4 = idx % (BW / 4);
+      offs[u] = row * BW + 4 * c4;
+      ok[u] = idx < total && t0 + row < args.M && f0 + 4 * c4 < args.rows_out;
+      if (ok[u]) {
+#pragma unroll
+        for (int qq = 0; qq < S; ++qq)
+          part[u][qq] = S == 1 ? *reinterpret_cast<const float4*>(stage_f32 + offs[u])
+                               : ld_dsmem_v4(src[qq] + 4u * (uint32_t)offs[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (!ok[u]) continue;
+      float4 acc = part[u][0];
+#pragma unroll
+      for (int qq = 1; qq < S; ++qq) {
+        acc.x += part[u][qq].x;
+        acc.y += part[u][qq].y;
+        acc.z += part[u][qq].z;
+        acc.w += part[u][qq].w;
+      }
+      const int m = t0 + offs[u] / BW, f = f0 + offs[u] % BW;
+      float* dst;
+      if (f < o.n1) dst = o.y0 + (size_t)m * o.n1 + f;
+      else if (f < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (f - o.n1);
+      else dst = o.y2 + (size_t)m * (o.N - o.n2) + (f - o.n2);
+      *reinterpret_cast<float4*>(dst) = acc;
+    }
+  }
 }
 
 template <bool BWD, int ST, bool F32S>
@@ -147,7 +201,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       mbar_init(&ctl->full[i], 1);
       mbar_init(&ctl->consumed[i], 1);
     }
-    for (int i = 0; i < WST; ++i) mbar_init(&ctl->wready[i], kDequantWarps);
+    for (int i = 0; i < WST; ++i) mbar_init(&ctl->wready[i], kDequantWarps / WST);   // one warp per lane quadrant
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -215,27 +269,57 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // The tensor core accepts little more than the MMA it is executing, so
-    // every cycle this thread spends between stages is a bubble: it waits on
-    // wready alone (each dequantisation warp saw the stage's full barrier
-    // before arriving, so wready covers the activation tile too), tests the
-    // next stage's barrier while the last MMA of this stage is queued, and
-    // commits once per stage.
+    // Every cycle this thread spends between stages is a bubble of the tensor
+    // pipe, and the MMAs issue at the pipe's rate only from straight-line code
+    // whose operand addresses are fixed offsets: measured on B200 with the
+    // stage and slot indices taken modulo at run time, four MMAs and their
+    // commit took ~570 cycles at every token width, against ~330 (64 tokens)
+    // and 512 (256 tokens, the MMA's own time) from the unrolled form below.
+    // So the loop runs in blocks of U = lcm(ST, WST) stages, in which stage j
+    // of the block uses shared-memory stage j % ST and TMEM slot j % WST as
+    // constants; the last nitx mod U stages take the generic loop.  Each stage
+    // waits on wready alone (each dequantisation warp saw the stage's full
+    // barrier before arriving, so wready covers the activation tile too) and
+    // commits once.
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(BW, args.bt, false);
-      bool next_ready = false;
-      for (int it = 0; it < nitx; ++it) {
-        const int s = it % ST, w = it % WST;
-        if (!next_ready && !mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
-        tc_fence_after();
-        const uint32_t x0 = sbase + SM::OFF_X + s * X_BYTES;
+      // The descriptor's start address field is address / 16 in its low 14
+      // bits (shared addresses stay below 256 KB), so the descriptor of the
+      // activation tile of stage s at depth 16 ks is the stage-0 descriptor
+      // plus (s X_BYTES + 32 ks) / 16: an immediate add, no register per stage.
+      const uint64_t d0 = smem_desc_sw128(sbase + SM::OFF_X, 16, 1024);
+      const uint32_t ab = tmem + ACC_COLS;
+      auto issue = [&](uint32_t s, uint32_t w, bool first) {
 #pragma unroll
-        for (int ks = 0; ks < TK / 16; ++ks) {
-          if (ks == TK / 16 - 1)
-            next_ready = it + 1 < nitx && mbar_test_wait(&ctl->wready[(it + 1) % WST], ((it + 1) / WST) & 1);
-          const uint64_t bd = smem_desc_sw128(x0 + 32 * ks, 16, 1024);
-          mma_f16_ts(tmem, tmem + ACC_COLS + w * A_COLS + 8 * ks, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < TK / 16; ++ks)
+          mma_f16_ts(tmem, ab + w * A_COLS + 8 * ks, d0 + ((s * X_BYTES + 32 * ks) >> 4), idesc,
+                     (first && ks == 0) ? 0u : 1u);
+      };
+      constexpr int U = ST * WST / (ST % WST == 0 ? WST : ST % 2 == 0 ? 2 : 1);   // lcm(ST, WST), WST = 4
+      static_assert(U % ST == 0 && U % WST == 0, "block of stages");
+      bool ok = true;
+      const int nblk = nitx / U;
+      for (int b = 0; b < nblk && ok; ++b) {
+        const int it0 = b * U;
+        const uint32_t ph = (uint32_t)(it0 / WST) & 1u;
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+          const uint32_t pw = (ph + (uint32_t)(j / WST)) & 1u;
+          if (!mbar_try_wait(&ctl->wready[j % WST], pw) &&
+              !mbar_wait(&ctl->wready[j % WST], pw, abort_flag, &g_device_error, 4u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue(j % ST, j % WST, it0 + j == 0);
+          mma_commit(&ctl->consumed[j % ST]);
         }
+      }
+      for (int it = nblk * U; it < nitx && ok; ++it) {
+        const int s = it % ST, w = it % WST;
+        if (!mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
+        tc_fence_after();
+        issue(s, w, it == 0);
         mma_commit(&ctl->consumed[s]);
       }
       mma_commit(&ctl->accfull);
@@ -244,39 +328,46 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     }
   } else {
     // ------------------------------------------------------------ dequantisation
-    // Thread = weight row r of the tile (its TMEM lane); the warp's slice kq
-    // covers contraction columns 16 kq .. 16 kq + 15 of each stage, i.e. the
-    // 8 TMEM columns 8 kq .. 8 kq + 7 of the stage (two fp16 per column, lower
-    // index in the low half).
+    // Thread = weight row r of the tile (its TMEM lane 32 q + lane).  The
+    // four warps of lane quadrant q take whole stages in turn: warp kq
+    // dequantises stages kq, kq + 4, kq + 8, ... (all 64 contraction columns,
+    // i.e. the 32 TMEM columns of slot it % WST = kq; two fp16 per column,
+    // lower index in the low half).  A warp thus pays the latency of its two
+    // barrier waits (~140 cycles each, measured, even on a completed phase)
+    // once per four stages; with every warp on every stage that chain bounded
+    // the stage rate at ~650 cycles.
+    static_assert(kDequantWarps == 4 * WST, "warp kq of a lane quadrant owns TMEM slot kq");
     const int q = warp & 3, kq = (warp - 2) >> 2;
     const int r = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    uint32_t off[8];
-    uint32_t sc_off, shift = 0;
+    const uint32_t slot = tmem + lane_base + (uint32_t)(ACC_COLS + kq * A_COLS);
+    uint32_t off[4] = {0u, 0u, 0u, 0u};
+    uint32_t sc_off[4] = {0u, 0u, 0u, 0u};
+    uint32_t shift = 0, boff = 0, sc_base = 0;
     if (!BWD) {
-      // Row r = 2 p + odd of pair p.  Word kq of the 16-byte chunk t of the
-      // pair row holds columns 16 kq + 4 t + (0, 2, 1, 3) in its byte slots;
+      // Row r = 2 p + odd of pair p.  Word c of the 16-byte chunk t of the
+      // pair row holds columns 16 c + 4 t + (0, 2, 1, 3) in its byte slots;
       // the chunk sits at 16 (t ^ ((p >> 1) & 3)) under the 64-byte swizzle.
       const int p = r >> 1;
       shift = 4 * (r & 1);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) off[t] = p * 64 + 16 * (t ^ ((p >> 1) & 3)) + 4 * kq;
-      // the 16 columns share one scale: row ((kc mod gs) + 16 kq) >> gsl of
-      // the stage's box (stages start on 64-column boundaries)
-      sc_off = (args.gs < 64 ? ((16 * kq) >> gsl) : 0) * BW * SB + SB * r;
+      for (int t = 0; t < 4; ++t) off[t] = p * 64 + 16 * (t ^ ((p >> 1) & 3));
+      // columns 16 c .. 16 c + 15 share one scale: row (16 c) >> gsl of the
+      // stage's box (stages start on 64-column boundaries)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sc_off[c] = (args.gs < 64 ? ((16 * c) >> gsl) : 0) * BW * SB + SB * r;
     } else {
       // Row r = output feature k = f0 + r.  Pair row p (contraction rows 2p,
       // 2p+1) holds it in byte column_offset(r) of its 128-byte box row; the
-      // scale of both rows sits in scale row ((f0 mod gs) + r) >> gsl.
-      const uint32_t boff = (uint32_t)column_offset(r);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) off[j] = (8 * kq + j) * 128 + boff;
-      sc_off = (uint32_t)((((f0 & (args.gs - 1)) + r) >> gsl) * TK * SB + 2 * SB * 8 * kq);
+      // scales of pair p sit at 2 SB p of scale row ((f0 mod gs) + r) >> gsl.
+      boff = (uint32_t)column_offset(r);
+      sc_base = (uint32_t)((((f0 & (args.gs - 1)) + r) >> gsl) * TK * SB);
     }
-    for (int it = 0; it < nitx; ++it) {
-      const int s = it % ST, w = it % WST;
+    for (int it = kq; it < nitx; it += WST) {
+      const int s = it % ST;
       if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
-      // TMEM slot w is free once the MMAs of stage it - WST completed
+      // TMEM slot kq is free once the MMAs of stage it - WST (this warp's
+      // previous stage) completed
       if (it >= WST &&
           !mbar_wait(&ctl->consumed[(it - WST) % ST], ((it - WST) / ST) & 1, abort_flag, &g_device_error, 32u))
         break;
@@ -285,63 +376,80 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       const uint32_t sc = sbase + SM::OFF_SC + s * SC_BYTES;
       uint32_t v[8];
       if (it >= nit) {
-        // The adapter stage: rank columns j = 16 kq .. 16 kq + 15 of this
-        // thread's output feature, straight from the fp16 adapter matrix
-        // (forward B[f][j], backward A[j][f]; zero past the rank or the extent).
+        // The adapter stage: rank columns j = 0 .. 63 of this thread's output
+        // feature, straight from the fp16 adapter matrix (forward B[f][j],
+        // backward A[j][f]; zero past the rank or the extent).
         const int f = f0 + r;
         const bool fin = f < args.rows_out;
         const unsigned short* am = reinterpret_cast<const unsigned short*>(args.ad_mat);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int j = 16 * kq + 2 * m;
-          uint32_t lo = 0u, hi = 0u;
-          if (fin && j < args.ad_r)
-            lo = BWD ? __ldg(am + (size_t)j * args.ad_ld + f) : __ldg(am + (size_t)f * args.ad_ld + j);
-          if (fin && j + 1 < args.ad_r)
-            hi = BWD ? __ldg(am + (size_t)(j + 1) * args.ad_ld + f) : __ldg(am + (size_t)f * args.ad_ld + j + 1);
-          v[m] = lo | (hi << 16);
+          for (int m = 0; m < 8; ++m) {
+            const int j = 16 * c + 2 * m;
+            uint32_t lo = 0u, hi = 0u;
+            if (fin && j < args.ad_r)
+              lo = BWD ? __ldg(am + (size_t)j * args.ad_ld + f) : __ldg(am + (size_t)f * args.ad_ld + j);
+            if (fin && j + 1 < args.ad_r)
+              hi = BWD ? __ldg(am + (size_t)(j + 1) * args.ad_ld + f) : __ldg(am + (size_t)f * args.ad_ld + j + 1);
+            v[m] = lo | (hi << 16);
+          }
+          tmem_st_32x32b_x8(slot + 8 * c, v);
         }
       } else if (!BWD) {
-        uint32_t wd[4];
+        uint4 wv[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) wd[t] = lds32(pk + off[t]);
-        if (F32S) {
-          const float sf = __uint_as_float(lds32(sc + sc_off));
+        for (int t = 0; t < 4; ++t) wv[t] = lds128_u32addr(pk + off[t]);
+        uint32_t sraw[4];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const uint32_t W = wd[t] >> shift;                                           // this row's nibbles
-            v[2 * t] = weight_pair_f32s(u32_as_h2(nibbles_minus8(W)), sf, sf);          // columns 4t, 4t+1
-            v[2 * t + 1] = weight_pair_f32s(u32_as_h2(nibbles_minus8(W >> 8)), sf, sf); // 4t+2, 4t+3
-          }
-        } else {
-          const uint32_t sb = lds_u16(sc + sc_off);
-          const __half2 s2 = u32_as_h2(sb | (sb << 16));
+        for (int c = 0; c < 4; ++c) sraw[c] = F32S ? lds32(sc + sc_off[c]) : lds_u16(sc + sc_off[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            const uint32_t W = wd[t] >> shift;                                      // this row's nibbles
-            v[2 * t] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W)), s2));       // columns 4t, 4t+1
-            v[2 * t + 1] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W >> 8)), s2));  // 4t+2, 4t+3
+            const uint32_t word = c == 0 ? wv[t].x : c == 1 ? wv[t].y : c == 2 ? wv[t].z : wv[t].w;
+            const uint32_t W = word >> shift;   // this row's nibbles
+            if (F32S) {
+              const float sf = __uint_as_float(sraw[c]);
+              v[2 * t] = weight_pair_f32s(u32_as_h2(nibbles_minus8(W)), sf, sf);          // columns 4t, 4t+1
+              v[2 * t + 1] = weight_pair_f32s(u32_as_h2(nibbles_minus8(W >> 8)), sf, sf); // 4t+2, 4t+3
+            } else {
+              const __half2 s2 = u32_as_h2(sraw[c] | (sraw[c] << 16));
+              v[2 * t] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W)), s2));            // columns 4t, 4t+1
+              v[2 * t + 1] = h2_as_u32(__hmul2(u32_as_h2(nibbles_minus8(W >> 8)), s2));   // 4t+2, 4t+3
+            }
           }
+          tmem_st_32x32b_x8(slot + 8 * c, v);
         }
       } else {
+        // four slices of 8 pairs (16 contraction rows), each slice's 8 code
+        // bytes and their scales loaded before any is used (fp32 scales: one
+        // slice at a time, within the register budget)
+#pragma unroll (F32S ? 1 : 4)
+        for (int c = 0; c < 4; ++c) {
+          uint32_t b[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t b = lds_u8(pk + off[j]);                 // code[2p, k] | code[2p+1, k] << 4
-          const __half2 c2 = u32_as_h2(nibbles_minus8(b * 0x1001u));
-          if (F32S) {
-            const uint32_t a = sc + sc_off + 8 * j;                 // s32[g, 2p], s32[g, 2p+1]
-            v[j] = weight_pair_f32s(c2, __uint_as_float(lds32(a)), __uint_as_float(lds32(a + 4)));
-          } else {
-            const uint32_t s2 = lds32(sc + sc_off + 4 * j);        // s[g, 2p], s[g, 2p+1]
-            v[j] = h2_as_u32(__hmul2(c2, u32_as_h2(s2)));
+          for (int j = 0; j < 8; ++j) b[j] = lds_u8(pk + (8 * c + j) * 128 + boff);   // pair p = 8 c + j: code[2p, k] | code[2p+1, k] << 4
+          constexpr int NV = F32S ? 4 : 2;   // 16-byte scale vectors of 8 pairs
+          uint4 sv[NV];
+#pragma unroll
+          for (int u = 0; u < NV; ++u) sv[u] = lds128_u32addr(sc + sc_base + 2 * SB * 8 * c + 16 * u);
+          const uint32_t* sw = reinterpret_cast<const uint32_t*>(sv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const __half2 c2 = u32_as_h2(nibbles_minus8(b[j] * 0x1001u));
+            if (F32S)   // s32[g, 2p], s32[g, 2p+1]
+              v[j] = weight_pair_f32s(c2, __uint_as_float(sw[2 * j]), __uint_as_float(sw[2 * j + 1]));
+            else        // s[g, 2p], s[g, 2p+1]
+              v[j] = h2_as_u32(__hmul2(c2, u32_as_h2(sw[j])));
           }
+          tmem_st_32x32b_x8(slot + 8 * c, v);
         }
       }
-      tmem_st_32x32b_x8(tmem + lane_base + (uint32_t)(ACC_COLS + w * A_COLS + 8 * kq), v);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->wready[w]);
+      if (lane == 0) mbar_arrive(&ctl->wready[kq]);
     }
   }
 
@@ -388,47 +496,28 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
   } else {
     // Copy-out: one warp writes 512 contiguous bytes (128 features of one
     // token); with split-K, rank rk sums rows [rk bt / S, (rk + 1) bt / S) of
-    // the S partial tiles, loading all S before adding them in rank order.
+    // the S partial tiles in rank order.
     // Every thread of every CTA of the cluster passes the barriers, aborted or not.
     cg::cluster_group cluster = cg::this_cluster();
-    if (S > 1) cluster.sync();
+    if (S > 1) cluster_barrier();
     else __syncthreads();
     {
       const int rk = S > 1 ? (int)cluster.block_rank() : 0;
       const int row_b = rk * args.bt / S, row_e = (rk + 1) * args.bt / S;
       if (!(S > 1 ? cluster_any_abort(cluster, &ctl->abort, S) : *abort_flag)) {
-        for (int idx = threadIdx.x; idx < (row_e - row_b) * (BW / 4); idx += kThreads) {
-          const int row = row_b + idx / (BW / 4), c4 = idx % (BW / 4);
-          const int m = t0 + row, f = f0 + 4 * c4;
-          if (m >= args.M || f >= args.rows_out) continue;
-          const int offs = row * BW + 4 * c4;
-          float4 acc;
-          if (S == 1) {
-            acc = *reinterpret_cast<const float4*>(stage_f32 + offs);
-          } else {
-            float4 part[8];
-#pragma unroll
-            for (int qq = 0; qq < 8; ++qq)
-              if (qq < S) part[qq] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(stage_f32, qq) + offs);
-            acc = part[0];
-#pragma unroll
-            for (int qq = 1; qq < 8; ++qq)
-              if (qq < S) {
-                acc.x += part[qq].x;
-                acc.y += part[qq].y;
-                acc.z += part[qq].z;
-                acc.w += part[qq].w;
-              }
-          }
-          float* dst;
-          if (f < o.n1) dst = o.y0 + (size_t)m * o.n1 + f;
-          else if (f < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (f - o.n1);
-          else dst = o.y2 + (size_t)m * (o.N - o.n2) + (f - o.n2);
-          *reinterpret_cast<float4*>(dst) = acc;
+        switch (S) {
+          case 1: copy_out<1>(stage_f32, row_b, row_e, t0, f0, args); break;
+          case 2: copy_out<2>(stage_f32, row_b, row_e, t0, f0, args); break;
+          case 3: copy_out<3>(stage_f32, row_b, row_e, t0, f0, args); break;
+          case 4: copy_out<4>(stage_f32, row_b, row_e, t0, f0, args); break;
+          case 5: copy_out<5>(stage_f32, row_b, row_e, t0, f0, args); break;
+          case 6: copy_out<6>(stage_f32, row_b, row_e, t0, f0, args); break;
+          case 7: copy_out<7>(stage_f32, row_b, row_e, t0, f0, args); break;
+          default: copy_out<8>(stage_f32, row_b, row_e, t0, f0, args); break;
         }
       }
     }
-    if (S > 1) cluster.sync();
+    if (S > 1) cluster_barrier();   // no CTA leaves while another reads its tile
   }
   tc_fence_before();
   __syncthreads();

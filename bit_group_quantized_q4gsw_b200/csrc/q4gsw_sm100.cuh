@@ -99,6 +99,27 @@ __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parit
   return true;
 }
 
+// Cluster-wide barrier of every thread of every CTA of the cluster: arrive
+// with release, wait with acquire (orders the shared-memory writes before it
+// with the distributed-shared-memory reads after it).
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in the CTA of cluster rank
+// `rank` (32-bit shared::cluster window), and a 16-byte load from it.
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t caddr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(caddr) : "memory");
+  return v;
+}
+
 // Called between two cluster barriers (every CTA's main loop is over): true if
 // the wait of any CTA of the cluster ran out, so that no CTA stores sums that
 // include another CTA's unfinished partial tile.
