@@ -23,11 +23,12 @@
 //   warp 0       TMA producer: activation tile [bt][64] fp16 (128-byte
 //                swizzle), packed codes and scale rows of each 64-deep stage;
 //   warp 1       allocates tensor memory (fp32 accumulator in columns 0..255,
-//                a ring of WST dequantised stages of 32 columns after it) and
-//                issues tcgen05.mma from one thread;
+//                after it one 32-column slot of dequantised weights per
+//                shared-memory stage) and issues tcgen05.mma from one thread;
 //   warps 2..17  warp w writes TMEM lanes 32 (w % 4) .. +31 (weight rows) of
-//                every fourth stage (stages (w - 2) / 4 + 4 i, TMEM slot
-//                (w - 2) / 4), then runs the epilogue for the same lanes.
+//                every fourth stage (stages (w - 2) / 4 + 4 i, each into the
+//                slot of its shared-memory stage), then runs the epilogue for
+//                the same lanes.
 // Every consumer waits on every phase of the barriers it uses.
 #pragma once
 
@@ -37,7 +38,7 @@ namespace ts {
 constexpr int BW = 128;                    // weight rows per tile (MMA M)
 constexpr int BT_MAX = 256;                // tokens per tile (MMA N)
 constexpr int TK = 64;                     // contraction depth per stage
-constexpr int WST = 4;                     // tensor-memory ring of dequantised stages
+constexpr int kMaxST = 8;                  // shared-memory stages (and TMEM slots) at most
 constexpr int kDequantWarps = 16;
 constexpr int kThreads = 32 * (2 + kDequantWarps);
 constexpr int X_BYTES = BT_MAX * TK * 2;   // activation tile, 32 KB
@@ -46,7 +47,7 @@ constexpr int CTL_BYTES = 256;
 constexpr int ACC_COLS = 256;              // fp32 accumulator columns (tokens)
 constexpr int A_COLS = TK / 2;             // one dequantised stage: 64 fp16 per lane = 32 columns
 constexpr int TMEM_COLS = 512;
-static_assert(ACC_COLS + WST * A_COLS <= TMEM_COLS, "tensor memory budget");
+static_assert(ACC_COLS + kMaxST * A_COLS <= TMEM_COLS, "tensor memory budget");
 
 // ST stages; SCB bytes of scale rows per stage (1 KB for fp16 scales, 2 KB for
 // fp32 scales, packed layout version 2).
@@ -81,9 +82,9 @@ struct Args {
 };
 
 struct Ctl {
-  uint64_t full[8];       // stage s loaded (TMA transaction bytes)
-  uint64_t consumed[8];   // the MMAs of the stage in slot s completed (one commit per stage)
-  uint64_t wready[WST];   // dequantised stage in TMEM slot w written (one warp per lane quadrant)
+  uint64_t full[kMaxST];       // stage s loaded (TMA transaction bytes)
+  uint64_t consumed[kMaxST];   // the MMAs of the stage in slot s completed (one commit per stage)
+  uint64_t wready[kMaxST];     // dequantised stage in TMEM slot s written (one warp per lane quadrant)
   uint64_t accfull;
   uint64_t drain;
   uint32_t tmem_base;
@@ -176,6 +177,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
                      const __grid_constant__ CUtensorMap map_y1, const __grid_constant__ CUtensorMap map_y2,
                      const __grid_constant__ CUtensorMap map_ad, const Args args) {
   using namespace sm100;
+  static_assert(ST <= kMaxST, "barrier arrays and TMEM slots");
   using SM = Smem<ST, F32S ? 2048 : 1024>;
   constexpr int SC_BYTES = SM::SC_BYTES;
   constexpr int SB = F32S ? 4 : 2;   // bytes per scale
@@ -200,8 +202,8 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     for (int i = 0; i < ST; ++i) {
       mbar_init(&ctl->full[i], 1);
       mbar_init(&ctl->consumed[i], 1);
+      mbar_init(&ctl->wready[i], 4);   // one warp per lane quadrant
     }
-    for (int i = 0; i < WST; ++i) mbar_init(&ctl->wready[i], kDequantWarps / WST);   // one warp per lane quadrant
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -275,12 +277,11 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     // stage and slot indices taken modulo at run time, four MMAs and their
     // commit took ~570 cycles at every token width, against ~330 (64 tokens)
     // and 512 (256 tokens, the MMA's own time) from the unrolled form below.
-    // So the loop runs in blocks of U = lcm(ST, WST) stages, in which stage j
-    // of the block uses shared-memory stage j % ST and TMEM slot j % WST as
-    // constants; the last nitx mod U stages take the generic loop.  Each stage
-    // waits on wready alone (each dequantisation warp saw the stage's full
-    // barrier before arriving, so wready covers the activation tile too) and
-    // commits once.
+    // So the loop runs in blocks of ST stages, in which stage j of the block
+    // uses shared-memory stage and TMEM slot j as constants; the last nitx mod
+    // ST stages take the generic loop.  Each stage waits on wready alone (each
+    // dequantisation warp saw the stage's full barrier before arriving, so
+    // wready covers the activation tile too) and commits once.
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(BW, args.bt, false);
       // The descriptor's start address field is address / 16 in its low 14
@@ -289,37 +290,33 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       // plus (s X_BYTES + 32 ks) / 16: an immediate add, no register per stage.
       const uint64_t d0 = smem_desc_sw128(sbase + SM::OFF_X, 16, 1024);
       const uint32_t ab = tmem + ACC_COLS;
-      auto issue = [&](uint32_t s, uint32_t w, bool first) {
+      auto issue = [&](uint32_t s, bool first) {
 #pragma unroll
         for (int ks = 0; ks < TK / 16; ++ks)
-          mma_f16_ts(tmem, ab + w * A_COLS + 8 * ks, d0 + ((s * X_BYTES + 32 * ks) >> 4), idesc,
+          mma_f16_ts(tmem, ab + s * A_COLS + 8 * ks, d0 + ((s * X_BYTES + 32 * ks) >> 4), idesc,
                      (first && ks == 0) ? 0u : 1u);
       };
-      constexpr int U = ST * WST / (ST % WST == 0 ? WST : ST % 2 == 0 ? 2 : 1);   // lcm(ST, WST), WST = 4
-      static_assert(U % ST == 0 && U % WST == 0, "block of stages");
       bool ok = true;
-      const int nblk = nitx / U;
+      const int nblk = nitx / ST;
       for (int b = 0; b < nblk && ok; ++b) {
-        const int it0 = b * U;
-        const uint32_t ph = (uint32_t)(it0 / WST) & 1u;
+        const uint32_t ph = (uint32_t)b & 1u;
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-          const uint32_t pw = (ph + (uint32_t)(j / WST)) & 1u;
-          if (!mbar_try_wait(&ctl->wready[j % WST], pw) &&
-              !mbar_wait(&ctl->wready[j % WST], pw, abort_flag, &g_device_error, 4u)) {
+        for (int j = 0; j < ST; ++j) {
+          if (!mbar_try_wait(&ctl->wready[j], ph) &&
+              !mbar_wait(&ctl->wready[j], ph, abort_flag, &g_device_error, 4u)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue(j % ST, j % WST, it0 + j == 0);
-          mma_commit(&ctl->consumed[j % ST]);
+          issue(j, b == 0 && j == 0);
+          mma_commit(&ctl->consumed[j]);
         }
       }
-      for (int it = nblk * U; it < nitx && ok; ++it) {
-        const int s = it % ST, w = it % WST;
-        if (!mbar_wait(&ctl->wready[w], (it / WST) & 1, abort_flag, &g_device_error, 4u)) break;
+      for (int it = nblk * ST; it < nitx && ok; ++it) {
+        const int s = it % ST;
+        if (!mbar_wait(&ctl->wready[s], (it / ST) & 1, abort_flag, &g_device_error, 4u)) break;
         tc_fence_after();
-        issue(s, w, it == 0);
+        issue(s, it == 0);
         mma_commit(&ctl->consumed[s]);
       }
       mma_commit(&ctl->accfull);
@@ -331,16 +328,19 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     // Thread = weight row r of the tile (its TMEM lane 32 q + lane).  The
     // four warps of lane quadrant q take whole stages in turn: warp kq
     // dequantises stages kq, kq + 4, kq + 8, ... (all 64 contraction columns,
-    // i.e. the 32 TMEM columns of slot it % WST = kq; two fp16 per column,
-    // lower index in the low half).  A warp thus pays the latency of its two
-    // barrier waits (~140 cycles each, measured, even on a completed phase)
-    // once per four stages; with every warp on every stage that chain bounded
-    // the stage rate at ~650 cycles.
-    static_assert(kDequantWarps == 4 * WST, "warp kq of a lane quadrant owns TMEM slot kq");
+    // i.e. the 32 TMEM columns of the slot of the stage's shared-memory ring
+    // index; two fp16 per column, lower index in the low half).  A warp thus
+    // pays the latency of its barrier wait (~140 cycles, measured, even on a
+    // completed phase) once per four stages; with every warp on every stage
+    // that chain bounded the stage rate at ~650 cycles.
+    //
+    // One wait suffices: stage it's slot was last read by the MMAs of stage
+    // it - ST, and the producer refilled the stage (completing full) only
+    // after those MMAs had committed.
+    static_assert(kDequantWarps == 16, "four warps per lane quadrant");
     const int q = warp & 3, kq = (warp - 2) >> 2;
     const int r = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    const uint32_t slot = tmem + lane_base + (uint32_t)(ACC_COLS + kq * A_COLS);
     uint32_t off[4] = {0u, 0u, 0u, 0u};
     uint32_t sc_off[4] = {0u, 0u, 0u, 0u};
     uint32_t shift = 0, boff = 0, sc_base = 0;
@@ -363,15 +363,11 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       boff = (uint32_t)column_offset(r);
       sc_base = (uint32_t)((((f0 & (args.gs - 1)) + r) >> gsl) * TK * SB);
     }
-    for (int it = kq; it < nitx; it += WST) {
+    for (int it = kq; it < nitx; it += 4) {
       const int s = it % ST;
       if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
-      // TMEM slot kq is free once the MMAs of stage it - WST (this warp's
-      // previous stage) completed
-      if (it >= WST &&
-          !mbar_wait(&ctl->consumed[(it - WST) % ST], ((it - WST) / ST) & 1, abort_flag, &g_device_error, 32u))
-        break;
       tc_fence_after();
+      const uint32_t slot = tmem + lane_base + (uint32_t)(ACC_COLS + s * A_COLS);
       const uint32_t pk = sbase + SM::OFF_P + s * P_BYTES;
       const uint32_t sc = sbase + SM::OFF_SC + s * SC_BYTES;
       uint32_t v[8];
@@ -449,7 +445,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->wready[kq]);
+      if (lane == 0) mbar_arrive(&ctl->wready[s]);
     }
   }
 
@@ -694,7 +690,7 @@ static cudaError_t launch_gemm_ts_impl(const void* packed, int N, int K, int gs,
   cfg.gridDim = dim3(tiles_f, tiles_t, best_S);
   if (route)
     snprintf(route, route_len, "tcgen05_ts_gemm_%s launches=1 tile=%dx%dx%d stages=%d+%d grid=%dx%dx%d out=%s%s",
-             BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, WST, tiles_f, tiles_t, best_S, a.tma_out ? "tma" : "st",
+             BWD ? "bwd" : "fwd", BW, a.bt, TK, ST, ST, tiles_f, tiles_t, best_S, a.tma_out ? "tma" : "st",
              ad ? " adapter_stage=1" : "");
   return cudaLaunchKernelEx(&cfg, kern, map_act, map_pk, map_sc, map_y[0], map_y[1], map_y[2], map_ad, a);
 }
