@@ -49,7 +49,7 @@ WORKLOAD = ("adapter-training step of one 1B-class decoder layer on a frozen q4g
 # DRAM bytes per launch from one ncu capture of each op (dram__bytes_read.sum +
 # dram__bytes_write.sum), with the hash of the tensor-memory GEMM's sources they
 # were taken on: reported only while those sources still match, null otherwise.
-NCU_TRAFFIC = {"sources_sha": "434cb93ceaf6c46b", "bytes_per_launch": {'qkv_fwd': 5668000, 'up_fwd': 11566000, 'down_fwd': 17858000, 'down_bwd': 11567000, 'up_bwd': 17859000}}
+NCU_TRAFFIC = {"sources_sha": "f8936914d313ffc8", "bytes_per_launch": {'qkv_fwd': 5706000, 'up_fwd': 11604000, 'down_fwd': 17896000, 'down_bwd': 11604000, 'up_bwd': 17896000}}
 
 
 # the files the tensor-memory GEMM (every op of the step) is built from
@@ -425,6 +425,8 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize(device)
     barrier(world)
     torch.cuda.synchronize(device)
+    # a bounded wait that ran out inside the timed region makes its time meaningless
+    gs.q.q4gsw_device_error_check()
     ms_total = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
@@ -534,6 +536,7 @@ def run_gpu(args, rank, world, local_rank):
     e1.record(s_comp)
     torch.cuda.synchronize(device)
     barrier(world)
+    gs.q.q4gsw_device_error_check()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     e2e = {"value": job_throughput(world, flops_step, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
@@ -552,6 +555,7 @@ def run_gpu(args, rank, world, local_rank):
             "routes": {k: v[1] for k, v in per_call.items()}}
     if not args.no_shapes:
         line["shapes"] = shape_legs(device, peaks, world)
+        gs.q.q4gsw_device_error_check()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inputs)
     if rank == 0:

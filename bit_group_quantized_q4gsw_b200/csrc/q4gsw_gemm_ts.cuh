@@ -29,7 +29,8 @@
 //                every fourth stage (stages (w - 2) / 4 + 4 i, each into the
 //                slot of its shared-memory stage), then runs the epilogue for
 //                the same lanes.
-// Every consumer waits on every phase of the barriers it uses.
+// A parity wait is only sound while its barrier is at most one phase behind
+// the phase waited for; each wait below states why that holds.
 #pragma once
 
 namespace q4gsw {
@@ -334,9 +335,18 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     // completed phase) once per four stages; with every warp on every stage
     // that chain bounded the stage rate at ~650 cycles.
     //
-    // One wait suffices: stage it's slot was last read by the MMAs of stage
-    // it - ST, and the producer refilled the stage (completing full) only
-    // after those MMAs had committed.
+    // A warp sees only every fourth phase of a stage's barriers, so before
+    // waiting for stage it's full phase it first waits for the commit of
+    // stage it - ST's MMAs (consumed): those MMAs followed the wready of all
+    // four quadrant warps of stage it - ST, each of which had seen that
+    // stage's full phase, so full[s] is then at most one phase behind.
+    // (Without it, a load of stage it - ST landing after this warp's stage
+    // it - 4 left full[s] two phases behind: the parity test passed on the
+    // older phase, and the wready counts shifted until a warp waited on its
+    // own arrival.)  consumed[s] itself is at most one phase behind: this
+    // warp's stage it - 4 needed full(it - 4), which the producer issued
+    // after the commit of stage it - 4 - ST >= the one before it - ST.  The
+    // same commit frees the stage's TMEM slot, last read by those MMAs.
     static_assert(kDequantWarps == 16, "four warps per lane quadrant");
     const int q = warp & 3, kq = (warp - 2) >> 2;
     const int r = 32 * q + lane;
@@ -365,6 +375,7 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     }
     for (int it = kq; it < nitx; it += 4) {
       const int s = it % ST;
+      if (it >= ST && !mbar_wait(&ctl->consumed[s], ((it / ST) - 1) & 1, abort_flag, &g_device_error, 32u)) break;
       if (!mbar_wait(&ctl->full[s], (it / ST) & 1, abort_flag, &g_device_error, 8u)) break;
       tc_fence_after();
       const uint32_t slot = tmem + lane_base + (uint32_t)(ACC_COLS + s * A_COLS);
