@@ -61,7 +61,7 @@ struct Smem {
   static constexpr int OFF_CTL = OFF_SC + ST * SCB;
   static constexpr int BYTES = OFF_CTL + CTL_BYTES + 1024;
   static_assert(OFF_P % 1024 == 0 && OFF_SC % 1024 == 0, "1024-byte aligned regions");
-  static_assert(BT_MAX * BW * 4 <= OFF_SC, "split-K staging must fit below the scale slots");
+  static_assert((BT_MAX + 7) * BW * 4 <= OFF_SC, "split-K receive slots must fit below the scale slots");
   static_assert(BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -117,21 +117,26 @@ __device__ __forceinline__ uint32_t nibbles_minus8(uint32_t v) {
   return h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(v, 0x000F000Fu, 0x64006400u)), kSub));
 }
 
-// Rows [row_b, row_e) of the tile, summed over the S partial tiles parked in
-// the shared memory of the cluster's CTAs (ranks 0 .. S-1, added in rank
-// order), written as float4 to the output.  Each thread first issues the
-// loads of up to kPer items (S loads each, most of them remote), then adds
-// and stores: the reads of distributed shared memory are latency-bound, and
-// one item at a time left ~4 of those latencies in a row per thread.
+// Rows [row_b, row_e) of the tile, summed over the S partial tiles in rank
+// order and written as float4 to the output.  pushed: the partials sit in
+// this CTA's shared memory, rank qq's at stage_f32 + qq * slot_floats with
+// rows relative to row_b; otherwise each rank's whole [token][128] tile is
+// parked in its own shared memory and read through the cluster window.  Each
+// thread first issues the loads of up to kPer items (S each), then adds and
+// stores: remote loads are latency-bound, and one item at a time left ~4 of
+// those latencies in a row per thread.
 template <int S>
-__device__ __forceinline__ void copy_out(const float* stage_f32, int row_b, int row_e, int t0, int f0,
-                                         const Args& args) {
+__device__ __forceinline__ void copy_out(const float* stage_f32, bool pushed, int slot_floats, int row_b, int row_e,
+                                         int t0, int f0, const Args& args) {
   using namespace sm100;
   constexpr int kPer = S == 1 ? 8 : (12 / S > 0 ? 12 / S : 1);   // at most 12 float4 in flight
   const OutSplit& o = args.out;
-  uint32_t src[S];   // the staging tile of every rank, in the cluster's shared window
+  uint32_t src[S];   // rank qq's partial rows, in the cluster's shared window
 #pragma unroll
-  for (int qq = 0; qq < S; ++qq) src[qq] = S == 1 ? smem_u32(stage_f32) : mapa_u32(smem_u32(stage_f32), qq);
+  for (int qq = 0; qq < S; ++qq)
+    src[qq] = pushed ? smem_u32(stage_f32 + qq * slot_floats)
+                     : (S == 1 ? smem_u32(stage_f32) : mapa_u32(smem_u32(stage_f32), (uint32_t)qq));
+  const int r0 = pushed ? 0 : row_b;   // row of row_b in the source layout
   const int total = (row_e - row_b) * (BW / 4);
   for (int base = threadIdx.x; base < total; base += kThreads * kPer) {
     float4 part[kPer][S];
@@ -140,14 +145,15 @@ __device__ __forceinline__ void copy_out(const float* stage_f32, int row_b, int 
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int idx = base + u * kThreads;
-      const int row = row_b + idx / (BW / 4), c4 = idx % (BW / 4);
+      const int row = idx / (BW / 4), c4 = idx % (BW / 4);   // row relative to row_b
       offs[u] = row * BW + 4 * c4;
-      ok[u] = idx < total && t0 + row < args.M && f0 + 4 * c4 < args.rows_out;
+      ok[u] = idx < total && t0 + row_b + row < args.M && f0 + 4 * c4 < args.rows_out;
       if (ok[u]) {
+        const uint32_t o4 = 4u * (uint32_t)((r0 + row) * BW + 4 * c4);
 #pragma unroll
         for (int qq = 0; qq < S; ++qq)
-          part[u][qq] = S == 1 ? *reinterpret_cast<const float4*>(stage_f32 + offs[u])
-                               : ld_dsmem_v4(src[qq] + 4u * (uint32_t)offs[u]);
+          part[u][qq] = S == 1 ? *reinterpret_cast<const float4*>(stage_f32 + (r0 + row) * BW + 4 * c4)
+                               : ld_dsmem_v4(src[qq] + o4);
       }
     }
 #pragma unroll
@@ -161,7 +167,7 @@ __device__ __forceinline__ void copy_out(const float* stage_f32, int row_b, int 
         acc.z += part[u][qq].z;
         acc.w += part[u][qq].w;
       }
-      const int m = t0 + offs[u] / BW, f = f0 + offs[u] % BW;
+      const int m = t0 + row_b + offs[u] / BW, f = f0 + offs[u] % BW;
       float* dst;
       if (f < o.n1) dst = o.y0 + (size_t)m * o.n1 + f;
       else if (f < o.n2) dst = o.y1 + (size_t)m * (o.n2 - o.n1) + (f - o.n1);
@@ -473,8 +479,10 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
     if (have_acc) tc_fence_after();
   }
   const OutSplit& o = args.out;
-  float* stage_f32 = reinterpret_cast<float*>(smem);   // staging [256 tokens][128 features]
-  if (epi && have_acc) {
+  float* stage_f32 = reinterpret_cast<float*>(smem);   // the operand ring, idle by now
+  // Park the tile in this CTA's shared memory as [token][128 features].
+  auto park = [&] {
+    if (!(epi && have_acc)) return;
     const int q = warp & 3, cb = (warp - 2) >> 2;
     const int r = 32 * q + lane;
 #pragma unroll 1
@@ -487,44 +495,93 @@ q4gsw_gemm_ts_kernel(const __grid_constant__ CUtensorMap map_act, const __grid_c
 #pragma unroll
       for (int j = 0; j < 32; ++j) stage_f32[(col + j) * BW + r] = __uint_as_float(v[j]);
     }
-  }
-  if (args.tma_out) {
-    // One CTA per tile (no split-K): one tensor store of the [bt][128] fp32
-    // tile (rows past M and features past the output clipped by the map).
-    const CUtensorMap* my = f0 < o.n1 ? &map_y0 : (f0 < o.n2 ? &map_y1 : &map_y2);
-    const int c0 = f0 < o.n1 ? f0 : (f0 < o.n2 ? f0 - o.n1 : f0 - o.n2);
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (threadIdx.x == 0 && !*abort_flag) {
-      tma_store_2d(my, stage_f32, c0, t0);
-      bulk_commit();
-      bulk_wait_read_all();
+  };
+  if (S == 1) {
+    // One tensor store of the [bt][128] fp32 tile (rows past M and features
+    // past the output clipped by the map), or the threads' copy-out.
+    park();
+    if (args.tma_out) {
+      const CUtensorMap* my = f0 < o.n1 ? &map_y0 : (f0 < o.n2 ? &map_y1 : &map_y2);
+      const int c0 = f0 < o.n1 ? f0 : (f0 < o.n2 ? f0 - o.n1 : f0 - o.n2);
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (threadIdx.x == 0 && !*abort_flag) {
+        tma_store_2d(my, stage_f32, c0, t0);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+    } else {
+      __syncthreads();
+      if (!*abort_flag) copy_out<1>(stage_f32, false, 0, 0, args.bt, t0, f0, args);
     }
   } else {
-    // Copy-out: one warp writes 512 contiguous bytes (128 features of one
-    // token); with split-K, rank rk sums rows [rk bt / S, (rk + 1) bt / S) of
-    // the S partial tiles in rank order.
-    // Every thread of every CTA of the cluster passes the barriers, aborted or not.
+    // Split-K: rank rk owns token rows [rk bt / S, (rk + 1) bt / S) and adds
+    // the S partial tiles' rows in rank order.  Two ways to bring them over,
+    // chosen by the tile's width (measured on B200, M=512 MLP projections and
+    // Q/K/V):
+    //  - wide tiles (bt >= 192): once every CTA of the cluster is past its main
+    //    loop (first barrier: all operand rings idle), each CTA stores its
+    //    partial rows straight from tensor memory into the owner's receive
+    //    slot for its rank (remote stores are posted, no round trip); after the
+    //    second barrier each owner adds its slots from its own shared memory.
+    //    This spares parking the 128 KB tile and reading 3/4 of it remotely
+    //    (4-way split, 256 tokens: 21.0 -> 19.9 us);
+    //  - narrower tiles: each CTA parks its tile before the first barrier,
+    //    overlapping the cluster's slowest main loop, and the owners read the
+    //    other ranks' rows through the cluster window; after the second barrier
+    //    no CTA reads another's shared memory, so any may leave.
+    // Every thread of every CTA of the cluster passes both barriers, aborted or not.
     cg::cluster_group cluster = cg::this_cluster();
-    if (S > 1) cluster_barrier();
-    else __syncthreads();
-    {
-      const int rk = S > 1 ? (int)cluster.block_rank() : 0;
-      const int row_b = rk * args.bt / S, row_e = (rk + 1) * args.bt / S;
-      if (!(S > 1 ? cluster_any_abort(cluster, &ctl->abort, S) : *abort_flag)) {
-        switch (S) {
-          case 1: copy_out<1>(stage_f32, row_b, row_e, t0, f0, args); break;
-          case 2: copy_out<2>(stage_f32, row_b, row_e, t0, f0, args); break;
-          case 3: copy_out<3>(stage_f32, row_b, row_e, t0, f0, args); break;
-          case 4: copy_out<4>(stage_f32, row_b, row_e, t0, f0, args); break;
-          case 5: copy_out<5>(stage_f32, row_b, row_e, t0, f0, args); break;
-          case 6: copy_out<6>(stage_f32, row_b, row_e, t0, f0, args); break;
-          case 7: copy_out<7>(stage_f32, row_b, row_e, t0, f0, args); break;
-          default: copy_out<8>(stage_f32, row_b, row_e, t0, f0, args); break;
+    const int me = (int)cluster.block_rank();
+    const int row_b = me * args.bt / S, row_e = (me + 1) * args.bt / S;
+    const bool push = args.bt >= 192;
+    const int rmax = (args.bt + S - 1) / S;   // rows of the largest owner's range: one receive slot
+    if (!push) park();
+    cluster_barrier();
+    const bool aborted = cluster_any_abort(cluster, &ctl->abort, S);
+    if (push) {
+      if (epi && have_acc && !aborted) {
+        const int q = warp & 3, cb = (warp - 2) >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t mine = smem_u32(stage_f32) + 4u * (uint32_t)(me * rmax * BW + r);   // my slot, my feature
+#pragma unroll 1
+        for (int c32 = 0; c32 < 2; ++c32) {
+          const int col = 64 * cb + 32 * c32;
+          if (col >= args.bt) break;
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, v);
+          tmem_wait_ld();
+          int owner = ((col + 1) * S - 1) / args.bt;          // largest rank with rank bt / S <= col
+          int ob = owner * args.bt / S, oe = (owner + 1) * args.bt / S;
+          uint32_t dst = mapa_u32(mine, (uint32_t)owner);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = col + j;
+            if (t >= args.bt) break;
+            if (t >= oe) {   // the next owner's rows (uniform over the warp)
+              ++owner;
+              ob = oe;
+              oe = (owner + 1) * args.bt / S;
+              dst = mapa_u32(mine, (uint32_t)owner);
+            }
+            st_dsmem_f32(dst + 4u * (uint32_t)((t - ob) * BW), __uint_as_float(v[j]));
+          }
         }
       }
+      cluster_barrier();   // every partial row delivered
     }
-    if (S > 1) cluster_barrier();   // no CTA leaves while another reads its tile
+    if (!aborted) {
+      switch (S) {
+        case 2: copy_out<2>(stage_f32, push, rmax * BW, row_b, row_e, t0, f0, args); break;
+        case 3: copy_out<3>(stage_f32, push, rmax * BW, row_b, row_e, t0, f0, args); break;
+        case 4: copy_out<4>(stage_f32, push, rmax * BW, row_b, row_e, t0, f0, args); break;
+        case 5: copy_out<5>(stage_f32, push, rmax * BW, row_b, row_e, t0, f0, args); break;
+        case 6: copy_out<6>(stage_f32, push, rmax * BW, row_b, row_e, t0, f0, args); break;
+        case 7: copy_out<7>(stage_f32, push, rmax * BW, row_b, row_e, t0, f0, args); break;
+        default: copy_out<8>(stage_f32, push, rmax * BW, row_b, row_e, t0, f0, args); break;
+      }
+    }
+    if (!push) cluster_barrier();   // no CTA leaves while another reads its tile
   }
   tc_fence_before();
   __syncthreads();
