@@ -332,6 +332,27 @@ def test_gemm_split_k_cluster_reduction(gemm_variant):
     assert np.array_equal(dx.astype(np.float64), ref)
 
 
+@pytest.mark.parametrize("kind,M,N,K,gs", [("fwd", 512, 2048, 8192, 32), ("bwd", 512, 8192, 2048, 32),
+                                            ("fwd", 400, 2048, 8192, 64)])
+def test_split_k_wide_tiles_push_partials_bit_exact(kind, M, N, K, gs):
+    # split-K with tiles of at least 192 tokens: each CTA stores its partial
+    # rows into the owning rank's shared memory (the other split-K tests run
+    # narrower tiles, whose owners read the partials remotely instead); the
+    # 400-token case has a 208-token tile whose last rows lie past M
+    inp = wl.integer_exact_inputs(M, N, K, gs, seed=M + N)
+    if kind == "fwd":
+        y, route = run_fwd(inp, gs)
+        ref, _ = o.linear_fwd(bits(inp.x), inp.codes, bits(inp.scales), gs)
+    else:
+        y, route = run_bwd(inp, gs)
+        ref, _ = o.linear_bwd_input(bits(inp.d_out), inp.codes, bits(inp.scales), gs)
+    assert route.startswith("tcgen05_ts_gemm"), route
+    bt = int(route.split("tile=128x")[1].split("x")[0])
+    splits = int(route.split("grid=")[1].split()[0].split("x")[2])
+    assert bt >= 192 and splits > 1, route
+    assert np.array_equal(y.astype(np.float64), ref)
+
+
 def test_no_kernel_wait_ran_out():
     q().q4gsw_device_error_check()
 
