@@ -244,6 +244,11 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
 
     float part[RTW][NT][4];
     bool fresh = true;   // the next MMA starts a new group (zero accumulator)
+    // Release of a stage: with 16 tokens (NT = 2) after its MMAs, whose
+    // operands are then known to be in registers (M=16, 14336x4096 forward:
+    // 14.5 -> 13.9 us); with 8 tokens as soon as its words are loaded, which
+    // measured as fast or faster there (the refill starts earlier).
+    constexpr bool kLateRelease = NT == 2;
     // one stage: wait for its codes and scales, then dequantise and multiply;
     // false when a wait ran out
     auto stage = [&](int it, const uint2 (&xg)[NT][4]) -> bool {
@@ -280,10 +285,12 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
           for (int j = 0; j < NT; ++j)
 #pragma unroll
             for (int i = 0; i < 4; ++i) dep ^= xv[j][i].x ^ xv[j][i].y;
-        stage_reads_done(dep);
+        if (!kLateRelease) stage_reads_done(dep);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
+      if (!kLateRelease) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->empty[s]);   // the stage is in registers
+      }
 
       auto flush = [&](int q) {   // scale the finished group of every row tile into acc
 #pragma unroll
@@ -324,6 +331,18 @@ q4gsw_gemv_fwd_tma_kernel(const __grid_constant__ CUtensorMap map_pk, const __gr
         const int k0 = (st_begin + it) * SK + 64 * w;
         fresh = ((k0 + SK) >> gsl) != (k0 >> gsl) || it == nit - 1;
         if (fresh) flush(0);
+      }
+      if (kLateRelease) {
+        // the MMAs consumed the codes and activations; the scale words of a
+        // group that continues into the next stage (gs >= 256) may be unused
+        uint32_t dep = 0u;
+#pragma unroll
+        for (int rt = 0; rt < RTW; ++rt)
+#pragma unroll
+          for (int q = 0; q < NGB; ++q) dep ^= sw[rt][q].x ^ sw[rt][q].y;
+        stage_reads_done(dep);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->empty[s]);
       }
       return true;
     };
